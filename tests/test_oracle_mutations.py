@@ -1,0 +1,147 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and show the pins catch them.
+
+Each mutation swaps one oracle function for a wrong variant — a dropped term,
+a wrong sign, index or constant, a transposed operand — and at least one
+check of tests/test_oracle_pins.py must then fail.
+"""
+import numpy as np
+import pytest
+
+from oracle import bitnet_oracle as O
+import test_oracle_pins as pins
+
+F32 = np.float32
+_orig = {name: getattr(O, name) for name in dir(O) if callable(getattr(O, name))}
+
+
+def _absmax_128(y, qmax, qmin):
+    return _orig["absmax_quantize"](y, qmax + 1 if qmax == 127 else qmax, qmin)
+
+
+def _absmax_no_rint(y, qmax, qmin):
+    y = np.asarray(y, np.float32)
+    s = F32(qmax) / np.maximum(np.max(np.abs(y), axis=-1), O.SCALE_FLOOR)
+    return np.clip(np.trunc(y * s[..., None]), qmin, qmax).astype(np.int8), s
+
+
+def _scale_is_mean(w):
+    mean, _ = _orig["weight_scale"](w)
+    return mean, F32(mean)
+
+
+def _scale_absmax(w):
+    m = F32(np.max(np.abs(w)))
+    return m, F32(1.0) / m
+
+
+def _sum_drops_last(w):
+    return _orig["exact_sum_abs"](np.asarray(w).ravel()[:-1])
+
+
+def _fwht_wrong_sign(y, block):
+    y = np.asarray(y, np.float32)
+    M, K = y.shape
+    u = y.reshape(M, K // block, block)
+    h = 1
+    while h < block:
+        v = u.reshape(M, K // block, block // (2 * h), 2, h)
+        a, c = v[..., 0, :], v[..., 1, :]
+        u = np.stack([a + c, c - a], axis=-2).reshape(M, K // block, block)
+        h *= 2
+    return u.reshape(M, K)
+
+
+def _fwht_adjacent_only(y, block):
+    y = np.asarray(y, np.float32)
+    M, K = y.shape
+    u = y.reshape(M, K // block, block)
+    for _ in range(int(np.log2(block))):
+        v = u.reshape(M, K // block, block // 2, 2)
+        a, c = v[..., 0], v[..., 1]
+        u = np.stack([a + c, a - c], axis=-1).reshape(M, K // block, block)
+    return u.reshape(M, K)
+
+
+def _no_norm_const(block):
+    return F32(1.0)
+
+
+def _pack_transposed(q):
+    q = np.asarray(q, np.int8)
+    N, K = q.shape
+    f = (q.astype(np.int64) & 3).reshape(N, K // 16, 4, 4)
+    word = np.zeros((N, K // 16), np.uint64)
+    for j in range(4):
+        for i in range(4):
+            word |= (f[:, :, j, i] << (8 * j + 2 * i)).astype(np.uint64)
+    return np.ascontiguousarray(word.astype("<u4")).view(np.uint8).reshape(N, K // 4)
+
+
+def _pack_int4_swapped(q):
+    q = np.asarray(q, np.int8).astype(np.int64)
+    return ((q[:, 1::2] & 0xF) | ((q[:, 0::2] & 0xF) << 4)).astype(np.uint8)
+
+
+def _sequential_sum(v):
+    v = np.asarray(v, np.float32)
+    acc = np.zeros(v.shape[:-1], np.float32)
+    for k in range(v.shape[-1]):
+        acc = acc + v[..., k]
+    return acc
+
+
+def _rms_no_eps(x, gamma=None, eps=O.DEFAULT_EPS):
+    return _orig["rms_norm"](x, gamma, 0.0)
+
+
+def _rms_mean_of_abs(x, gamma=None, eps=O.DEFAULT_EPS):
+    x = np.asarray(x, np.float32)
+    ms = O.pairwise_sum_f32(np.abs(x)) / F32(x.shape[-1])
+    r = F32(1.0) / np.sqrt(ms + F32(eps))
+    y = x * r[..., None]
+    return (y * gamma if gamma is not None else y), r
+
+
+def _matmul_drop_last_k(qx, qw):
+    return _orig["int_matmul"](np.asarray(qx)[:, :-1], np.asarray(qw)[:, :-1])
+
+
+def _dequant_times(acc, s_x, s_w):
+    return np.asarray(acc, np.float32) * (np.asarray(s_x, np.float32)[:, None] * F32(s_w))
+
+
+def _ternarize_no_clamp(w, s_w):
+    return np.rint(np.asarray(w, np.float32) * F32(s_w)).astype(np.int8)
+
+
+MUTATIONS = {
+    "absmax_numerator_128": ("absmax_quantize", _absmax_128),
+    "absmax_truncates": ("absmax_quantize", _absmax_no_rint),
+    "weight_scale_is_mean": ("weight_scale", _scale_is_mean),
+    "weight_scale_absmax": ("weight_scale", _scale_absmax),
+    "weight_sum_drops_term": ("exact_sum_abs", _sum_drops_last),
+    "ternarize_no_clamp": ("ternarize", _ternarize_no_clamp),
+    "fwht_wrong_sign": ("fwht_f32", _fwht_wrong_sign),
+    "fwht_wrong_pairs": ("fwht_f32", _fwht_adjacent_only),
+    "hadamard_unnormalised": ("hadamard_norm_const", _no_norm_const),
+    "pack_ternary_transposed": ("pack_ternary", _pack_transposed),
+    "pack_int4_nibbles_swapped": ("pack_int4", _pack_int4_swapped),
+    "sum_sequential": ("pairwise_sum_f32", _sequential_sum),
+    "rms_no_eps": ("rms_norm", _rms_no_eps),
+    "rms_mean_abs": ("rms_norm", _rms_mean_of_abs),
+    "matmul_drops_term": ("int_matmul", _matmul_drop_last_k),
+    "dequant_multiplies": ("dequantize", _dequant_times),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name, monkeypatch):
+    attr, fn = MUTATIONS[name]
+    monkeypatch.setattr(O, attr, fn)
+    caught = []
+    for check in pins.CHECKS:
+        try:
+            check()
+        except Exception:
+            caught.append(check.__name__)
+    assert caught, f"no pin catches the planted mistake {name}"
