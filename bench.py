@@ -1,0 +1,459 @@
+"""Benchmark of the BitLinear hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|hbitlinear|tiny]
+                    [--impl ours|reference]
+
+One step = one BitLinear forward over one batch: the activation quantiser
+(RMSNorm + absmax int8, or RMSNorm + Hadamard + int4) and the ternary product
+with its dequantisation.  Weights are quantised offline, outside the timed
+region.  The default workload is the decode GEMV: X bf16 [16, 2560],
+W ternary [6912, 2560].  Rank 0 prints one JSON line.
+
+Device timing: the K timed steps are captured in one CUDA graph and replayed
+between CUDA events on the launching stream, with a barrier and a device
+synchronise on both sides; each step reads the next of a ring of weight copies
+whose total size exceeds twice the 126 MB L2.  The dominant kernel is timed the
+same way on its own for the roofline.  e2e: the same steps through the Python
+API with pinned host input/output buffers, the host<->device copies inside the
+timed region.  The CPU oracle is timed on a bounded sample on the host.
+
+Under torchrun (N > 1) each rank runs its own batches (independent tokens:
+weak scaling, no data-path collective); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bitlinear_bitnet_quant_b200 import workloads as wl  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "BitLinear tokens/sec and GB/s|TOPS vs HBM/int8 roofline, 1xB200"
+
+
+# ----------------------------------------------------------------------------
+# workloads
+# ----------------------------------------------------------------------------
+
+WORKLOADS = {
+    # name: (builder, eps)
+    "decode": lambda: wl.decode(16, with_weights=False),
+    "prefill": lambda: wl.prefill(with_weights=False),
+    "hbitlinear": lambda: wl.hbitlinear(with_weights=False),
+    "tiny": lambda: wl.tiny(),
+}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bitlinear_bitnet_quant_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profiled_traffic(kernel_tag: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.txt")
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("kernel_source_hash") != kernel_source_hash():
+            return None
+        return float(kv["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=2)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=1)
+        sm, mx, reasons = [], 0.0, set()
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                 f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# our implementation
+# ----------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from bitlinear_bitnet_quant_b200 import api, build_lib
+
+    build_lib.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+
+    c = WORKLOADS[args.workload]()
+    M, K, N, bits = c["M"], c["K"], c["N"], c["act_bits"]
+    eps = 1e-6
+    out_dtype = torch.bfloat16 if args.workload == "prefill" else torch.float32
+    out_bytes = 2 if out_dtype == torch.bfloat16 else 4
+
+    # ---- weights: quantised offline, a ring of copies larger than 2x L2 ----
+    packed_bytes = N * K // 4
+    copies = max(2, min(64, math.ceil(2.2 * L2_BYTES / packed_bytes)))
+    rng = np.random.default_rng(1234 + rank)
+    base_w = torch.from_numpy(wl.weights(N, K, seed=rank)).to(dev)
+    ring = []
+    for i in range(copies):
+        w = base_w if i == 0 else base_w[torch.from_numpy(rng.permutation(N)).to(dev)]
+        pk, s_w = api.bitnet_quantize_weights(w.contiguous())
+        ring.append((pk, s_w))
+    del base_w
+    torch.cuda.synchronize()
+
+    x_host = c["x"]
+    if c["x_dtype"] == "bf16":
+        x = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).to(dev)
+    else:
+        x = torch.from_numpy(x_host).to(dev)
+    # preallocated outputs (the graph reuses them)
+    if bits == 8:
+        xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    else:
+        xq = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    s_x = torch.empty((M,), dtype=torch.float32, device=dev)
+    Y = torch.empty((M, N), dtype=out_dtype, device=dev)
+
+    def quant():
+        if bits == 8:
+            api.bitnet_quant_act(x, None, eps, Xq=xq, s_x=s_x, stream=stream)
+        else:
+            api.bitnet_hadamard_quant_act(x, None, eps, c.get("had_block", 0), Xq4=xq, s_x=s_x, stream=stream)
+
+    def linear(i):
+        pk, s_w = ring[i % copies]
+        api.bitnet_linear(xq, bits, s_x, pk, s_w, Y=Y, stream=stream)
+
+    def step(i):
+        quant()
+        linear(i)
+
+    warmup = max(3, args.warmup)
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    def graph_of(fn, count):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(count):
+                fn(i)
+        return g
+
+    def timed(g):
+        g.replay()                      # untimed replay: warms the graph itself
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    steps = args.steps
+    g_step = graph_of(step, steps)
+    g_lin = graph_of(linear, steps)
+    g_q = graph_of(lambda i: quant(), steps)
+
+    visible = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    clocks = ClockSampler(visible[local_rank] if local_rank < len(visible) else str(local_rank))
+    clocks.start()
+    t_step = timed(g_step)
+    t_lin = timed(g_lin)
+    t_q = timed(g_q)
+    clk = clocks.stop()
+
+    # ---- e2e through the public API with pinned host buffers ----
+    x_pin = torch.empty_like(x, device="cpu").pin_memory()
+    x_pin.copy_(x.cpu())
+    y_pin = torch.empty((M, N), dtype=out_dtype).pin_memory()
+    h2d = x_pin.numel() * x_pin.element_size()
+    d2h = y_pin.numel() * y_pin.element_size()
+
+    def e2e_step(i):
+        x.copy_(x_pin, non_blocking=True)
+        pk, s_w = ring[i % copies]
+        Yo = api.bitlinear_forward(x, pk, s_w, act_bits=bits, eps=eps, had_block=c.get("had_block", 0),
+                                   out_dtype=out_dtype, stream=stream)
+        y_pin.copy_(Yo, non_blocking=True)
+
+    for i in range(warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([t_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_e2e = float(t.item())
+        dist.barrier()
+
+    if rank != 0:
+        return None
+
+    tokens_per_step = M * world
+    value = tokens_per_step * steps / (t_step / 1e3)
+    ms_per_step = t_step / steps
+    peaks, peak_src = load_peaks()
+    lin_s = t_lin / steps / 1e3
+    q_s = t_q / steps / 1e3
+    x_in_bytes = M * K * (2 if c["x_dtype"] == "bf16" else 4)
+    xq_bytes = M * K if bits == 8 else M * K // 2
+    if args.workload in ("decode", "tiny"):
+        alg_bytes = packed_bytes + xq_bytes + 4 * M + 4 + M * N * out_bytes
+        roof = {"bound": "hbm", "achieved": alg_bytes / lin_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "kernel": "bitnet_linear (tcgen05)" if M > 2 else "bitnet_linear (dp4a)",
+                "algorithmic_bytes_per_launch": alg_bytes}
+        tag = f"linear_{args.workload}"
+    else:
+        ops = 2.0 * M * N * K
+        int8_peak = 2.0 * peaks["bf16_tflops"]          # nominal int8 : bf16 = 4.5 : 2.25
+        roof = {"bound": "tensor", "achieved": ops / lin_s / 1e12, "peak": int8_peak, "unit": "TOPS",
+                "kernel": "bitnet_linear (tcgen05 kind::i8)", "algorithmic_ops_per_launch": ops,
+                "peak_note": "2 x measured bf16 burst (nominal int8/bf16 ratio)"}
+        tag = f"linear_{args.workload}"
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = profiled_traffic(tag)
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    quant_bytes = x_in_bytes + xq_bytes + 4 * M
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8xternary->int32" if bits == 8 else "int4xternary->int32",
+        "data": "synthetic",
+        "config": {"workload": c["name"], "M_tokens": M, "K": K, "N": N, "act_bits": bits,
+                   "x_dtype": c["x_dtype"], "out_dtype": "bf16" if out_bytes == 2 else "f32",
+                   "l2": f"ring of {copies} packed-weight copies ({copies * packed_bytes / 1e6:.0f} MB > 2x L2)",
+                   "timing": "CUDA graph of the K steps, CUDA events on the launching stream",
+                   "parallelism": f"dp{world} (independent batches per rank)"},
+        "roofline": roof,
+        "kernels_us": {"quant": q_s * 1e6, "linear": lin_s * 1e6},
+        "quant_roofline": {"bound": "hbm", "achieved": quant_bytes / q_s / 1e9, "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": quant_bytes / q_s / 1e9 / peaks["hbm_gbs"]},
+        "e2e": {"value": tokens_per_step * steps / (t_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * steps,
+        "clocks": clk,
+    }
+    return line
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle (the reference arm and the cpu_baseline leg)
+# ----------------------------------------------------------------------------
+
+def oracle_step_fn(c):
+    from oracle import bitnet_oracle as O
+    w = wl.weights(c["N"], c["K"], seed=0)
+    _, s_w, qw = O.quantize_weights(w)
+    x = O.bf16_bits_to_f32(c["x"]) if c["x_dtype"] == "bf16" else c["x"]
+
+    def step(rows):
+        xs = x[rows]
+        if c["act_bits"] == 8:
+            q, s = O.quant_act(xs, None, 1e-6)
+        else:
+            _, s, q, _ = O.hadamard_quant_act(xs, None, 1e-6, c.get("had_block", 0))
+        O.linear(q, s, qw, s_w)
+        return len(xs)
+    return step
+
+
+def sample_rows(c):
+    """Rows of one sampled step: the whole batch when small, else 8 tokens."""
+    return np.arange(c["M"]) if c["M"] <= 16 else np.arange(8)
+
+
+def cpu_baseline(c, budget_s=10.0):
+    step = oracle_step_fn(c)
+    rows = sample_rows(c)
+    step(rows[:1])                                   # warm-up (allocations)
+    t0 = time.perf_counter()
+    tokens, n = 0, 0
+    while True:
+        tokens += step(rows)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} oracle steps of {len(rows)} tokens of {c['name']} (numpy, single thread)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    c = WORKLOADS[args.workload]()
+    step = oracle_step_fn(c)
+    rows = sample_rows(c)
+    for _ in range(max(3, args.warmup)):
+        step(rows)
+    t0 = time.perf_counter()
+    tokens = 0
+    for _ in range(args.steps):
+        tokens += step(rows)
+    dt = time.perf_counter() - t0
+    value = tokens / dt
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8xternary->int64" if c["act_bits"] == 8 else "int4xternary->int64",
+            "data": "synthetic",
+            "config": {"workload": c["name"], "M_tokens": c["M"], "K": c["K"], "N": c["N"],
+                       "act_bits": c["act_bits"], "parallelism": "rank 0 only (CPU oracle)"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"each step: {len(rows)} tokens of {c['name']} through the numpy oracle"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        world = max(world, 1)
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    pg = False
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+        pg = True
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if line is not None:
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(WORKLOADS[args.workload]())
+            print(json.dumps(line), flush=True)
+    finally:
+        if pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

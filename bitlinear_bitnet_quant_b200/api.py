@@ -1,0 +1,189 @@
+"""Thin Python binding of libbitnet.so (include/bitnet.h).
+
+Argument marshalling only: every step of the BitLinear path runs in the
+library's CUDA kernels.  PyTorch supplies device memory and the current
+stream.  The functions keep the C names; outputs not passed in are allocated
+with torch on the input's device.  Any nonzero status raises BitnetError.
+If the library is missing, loading raises instead of falling back.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+from . import build_lib
+
+_c_void_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+
+BITNET_F32 = 0
+BITNET_BF16 = 1
+
+_lib = None
+
+# argument types of every entry point declared in include/bitnet.h
+_SIGNATURES = {
+    "bitnet_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "bitnet_abi_version": (ctypes.c_int, []),
+    "bitnet_quantize_weights_workspace_size": (ctypes.c_size_t, [_i64, _i64]),
+    "bitnet_quantize_weights": (ctypes.c_int, [_c_void_p, ctypes.c_int, _i64, _i64, _c_void_p, _c_void_p,
+                                               _c_void_p, ctypes.c_size_t, _c_void_p]),
+    "bitnet_quant_act": (ctypes.c_int, [_c_void_p, ctypes.c_int, _i64, _i64, _c_void_p, ctypes.c_float,
+                                        _c_void_p, _c_void_p, _c_void_p]),
+    "bitnet_hadamard_quant_act": (ctypes.c_int, [_c_void_p, ctypes.c_int, _i64, _i64, _c_void_p, ctypes.c_float,
+                                                 ctypes.c_int, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "bitnet_linear": (ctypes.c_int, [_c_void_p, ctypes.c_int, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64,
+                                     _c_void_p, ctypes.c_int, _c_void_p, _c_void_p]),
+    "bitnet_set_linear_path": (ctypes.c_int, [ctypes.c_int]),
+    "bitnet_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
+}
+
+
+class BitnetError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: status {status} ({status_string(status)})")
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/bitnet.h declares."""
+    with open(os.path.join(build_lib.INCLUDE, "bitnet.h")) as f:
+        text = f.read()
+    return re.findall(r"^BITNET_API\s+[\w\s\*]+?\b(bitnet_\w+)\s*\(", text, flags=re.M)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbitnet.so (built in-tree by build_lib); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        path = build_lib.LIB
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
+                               "`python -m bitlinear_bitnet_quant_b200.build_lib`")
+        L = ctypes.CDLL(path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().bitnet_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise BitnetError(fn, status)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return BITNET_F32
+    if t.dtype == torch.bfloat16:
+        return BITNET_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: fp32 or bf16 expected")
+
+
+def _require(t: torch.Tensor, name: str):
+    if not (t.is_cuda and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+# ---------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------
+
+def bitnet_quantize_weights_workspace_size(N: int, K: int) -> int:
+    return int(lib().bitnet_quantize_weights_workspace_size(N, K))
+
+
+def bitnet_quantize_weights(W: torch.Tensor, pkW=None, s_w=None, workspace=None, stream=None):
+    """Absmean ternarisation + packing.  Returns (pkW uint8 [N, K/4], s_w fp32 [1])."""
+    _require(W, "W")
+    N, K = W.shape
+    dev = W.device
+    pkW = torch.empty((N, K // 4), dtype=torch.uint8, device=dev) if pkW is None else pkW
+    s_w = torch.empty((1,), dtype=torch.float32, device=dev) if s_w is None else s_w
+    ws_bytes = bitnet_quantize_weights_workspace_size(N, K)
+    workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev) if workspace is None else workspace
+    _check("bitnet_quantize_weights", lib().bitnet_quantize_weights(
+        _ptr(W), _dtype_code(W), N, K, _ptr(pkW), _ptr(s_w), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return pkW, s_w
+
+
+def bitnet_quant_act(X: torch.Tensor, gamma=None, eps: float = 1e-6, Xq=None, s_x=None, stream=None):
+    """RMSNorm + per-token absmax int8.  Returns (Xq int8 [M, K], s_x fp32 [M])."""
+    _require(X, "X")
+    M, K = X.shape
+    Xq = torch.empty((M, K), dtype=torch.int8, device=X.device) if Xq is None else Xq
+    s_x = torch.empty((M,), dtype=torch.float32, device=X.device) if s_x is None else s_x
+    _check("bitnet_quant_act", lib().bitnet_quant_act(
+        _ptr(X), _dtype_code(X), M, K, _ptr(gamma), float(eps), _ptr(Xq), _ptr(s_x), _stream(stream)))
+    return Xq, s_x
+
+
+def bitnet_hadamard_quant_act(X: torch.Tensor, gamma=None, eps: float = 1e-6, had_block: int = 0,
+                              Xq4=None, s_x=None, want_t: bool = False, stream=None):
+    """RMSNorm + Hadamard + per-token int4.  Returns (Xq4 uint8 [M, K/2], s_x [M], t or None)."""
+    _require(X, "X")
+    M, K = X.shape
+    Xq4 = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device) if Xq4 is None else Xq4
+    s_x = torch.empty((M,), dtype=torch.float32, device=X.device) if s_x is None else s_x
+    T = torch.empty((M, K), dtype=torch.float32, device=X.device) if want_t else None
+    _check("bitnet_hadamard_quant_act", lib().bitnet_hadamard_quant_act(
+        _ptr(X), _dtype_code(X), M, K, _ptr(gamma), float(eps), int(had_block), _ptr(Xq4), _ptr(s_x),
+        _ptr(T), _stream(stream)))
+    return Xq4, s_x, T
+
+
+def bitnet_linear(Xq: torch.Tensor, act_bits: int, s_x: torch.Tensor, pkW: torch.Tensor, s_w: torch.Tensor,
+                  out_dtype=torch.float32, Y=None, want_acc: bool = False, stream=None):
+    """Ternary x int8/int4 product + dequantisation.  Returns (Y [M, N], acc int32 or None)."""
+    _require(Xq, "Xq")
+    _require(pkW, "pkW")
+    M = Xq.shape[0]
+    N, KB = pkW.shape
+    K = KB * 4
+    Y = torch.empty((M, N), dtype=out_dtype, device=Xq.device) if Y is None else Y
+    acc = torch.empty((M, N), dtype=torch.int32, device=Xq.device) if want_acc else None
+    _check("bitnet_linear", lib().bitnet_linear(
+        _ptr(Xq), int(act_bits), _ptr(s_x), _ptr(pkW), _ptr(s_w), M, N, K, _ptr(Y), _dtype_code(Y),
+        _ptr(acc), _stream(stream)))
+    return Y, acc
+
+
+def bitnet_set_linear_path(path: int) -> None:
+    _check("bitnet_set_linear_path", lib().bitnet_set_linear_path(int(path)))
+
+
+def bitnet_device_error() -> int:
+    code = ctypes.c_int(0)
+    _check("bitnet_device_error", lib().bitnet_device_error(ctypes.byref(code)))
+    return code.value
+
+
+def bitlinear_forward(X: torch.Tensor, pkW: torch.Tensor, s_w: torch.Tensor, act_bits: int = 8, gamma=None,
+                      eps: float = 1e-6, had_block: int = 0, out_dtype=torch.float32, stream=None):
+    """One BitLinear forward: quantise the activations, then the ternary product."""
+    if act_bits == 8:
+        Xq, s_x = bitnet_quant_act(X, gamma, eps, stream=stream)
+    else:
+        Xq, s_x, _ = bitnet_hadamard_quant_act(X, gamma, eps, had_block, stream=stream)
+    Y, _ = bitnet_linear(Xq, act_bits, s_x, pkW, s_w, out_dtype=out_dtype, stream=stream)
+    return Y

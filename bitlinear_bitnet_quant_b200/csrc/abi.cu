@@ -1,0 +1,170 @@
+// extern "C" entry points declared in include/bitnet.h: host-side validation,
+// then dispatch to the kernels.  Nothing here allocates device memory.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "../../include/bitnet.h"
+
+namespace bitnet {
+__device__ int g_device_error = 0;
+
+cudaError_t run_quantize_weights(const void* W, int bf16, int64_t N, int64_t K, uint8_t* pkW,
+                                 float* s_w, void* ws, cudaStream_t st);
+size_t weights_workspace_bytes();
+cudaError_t run_quant_act_i8(const void* X, int bf16, int M, int K, const float* gamma, float eps,
+                             int8_t* Xq, float* s_x, cudaStream_t st);
+cudaError_t run_hadamard_quant_i4(const void* X, int bf16, int M, int K, int L, const float* gamma,
+                                  float eps, uint8_t* Xq4, float* s_x, float* T_dbg, cudaStream_t st);
+cudaError_t run_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
+                       int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, int path, cudaStream_t st);
+bool tensor_map_encoder_available();
+}  // namespace bitnet
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_dev_ok[kMaxDevices];   // 0 unknown, 1 sm_100, 2 other
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return BITNET_ERR_CUDA; }
+  if (dev < 0 || dev >= kMaxDevices) return BITNET_ERR_UNSUPPORTED;
+  int s = g_dev_ok[dev].load(std::memory_order_relaxed);
+  if (s == 0) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return BITNET_ERR_CUDA;
+    }
+    s = major == 10 ? 1 : 2;
+    g_dev_ok[dev].store(s, std::memory_order_relaxed);
+  }
+  return s == 1 ? BITNET_OK : BITNET_ERR_UNSUPPORTED;
+}
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return BITNET_OK;
+  cudaGetLastError();
+  return BITNET_ERR_CUDA;
+}
+
+// 0 = automatic, 1 = SIMT, 2 = tcgen05 (set by bitnet_set_linear_path).
+std::atomic<int> g_linear_path{0};
+int linear_path() { return g_linear_path.load(std::memory_order_relaxed); }
+
+}  // namespace
+
+extern "C" {
+
+const char* bitnet_status_string(int status) {
+  switch (status) {
+    case BITNET_OK: return "ok";
+    case BITNET_ERR_NULL: return "a required pointer is NULL";
+    case BITNET_ERR_SHAPE: return "a size breaks the documented limits";
+    case BITNET_ERR_ALIGN: return "a tensor pointer is not 16-byte aligned";
+    case BITNET_ERR_DTYPE: return "unknown dtype or act_bits value";
+    case BITNET_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case BITNET_ERR_UNSUPPORTED: return "no sm_100 device or TMA encoder unavailable";
+    case BITNET_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int bitnet_abi_version(void) { return 1; }
+
+size_t bitnet_quantize_weights_workspace_size(int64_t N, int64_t K) {
+  (void)N; (void)K;
+  return bitnet::weights_workspace_bytes();
+}
+
+int bitnet_quantize_weights(const void* W, int w_dtype, int64_t N, int64_t K, uint8_t* pkW, float* s_w,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (!W || !pkW || !s_w) return BITNET_ERR_NULL;
+  if (w_dtype != BITNET_F32 && w_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (N < 1 || K < 16 || K % 16 != 0 || N * K >= (int64_t(1) << 31)) return BITNET_ERR_SHAPE;
+  if (!workspace || workspace_bytes < bitnet::weights_workspace_bytes()) return BITNET_ERR_WORKSPACE;
+  if (!aligned16(W) || !aligned16(pkW) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(s_w) & 3u))
+    return BITNET_ERR_ALIGN;
+  int d = check_device();
+  if (d != BITNET_OK) return d;
+  return cuda_status(bitnet::run_quantize_weights(W, w_dtype == BITNET_BF16, N, K, pkW, s_w, workspace,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
+int bitnet_quant_act(const void* X, int x_dtype, int64_t M, int64_t K, const float* gamma, float eps,
+                     int8_t* Xq, float* s_x, void* stream) {
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (M < 0 || M > (int64_t(1) << 30) || K < 16 || K > 16384 || K % 16 != 0) return BITNET_ERR_SHAPE;
+  if (M == 0) return BITNET_OK;
+  if (!X || !Xq || !s_x) return BITNET_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Xq) || (gamma && !aligned16(gamma)) || (reinterpret_cast<uintptr_t>(s_x) & 3u))
+    return BITNET_ERR_ALIGN;
+  int d = check_device();
+  if (d != BITNET_OK) return d;
+  return cuda_status(bitnet::run_quant_act_i8(X, x_dtype == BITNET_BF16, (int)M, (int)K, gamma, eps, Xq, s_x,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int bitnet_hadamard_quant_act(const void* X, int x_dtype, int64_t M, int64_t K, const float* gamma, float eps,
+                              int had_block, uint8_t* Xq4, float* s_x, float* T_dbg, void* stream) {
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (M < 0 || M > (int64_t(1) << 30) || K < 128 || K > 16384 || K % 128 != 0) return BITNET_ERR_SHAPE;
+  int64_t b = had_block;
+  if (b == 0) b = K & (-K);
+  if (b < 32 || b > 8192 || (b & (b - 1)) != 0 || K % b != 0) return BITNET_ERR_SHAPE;
+  if (M == 0) return BITNET_OK;
+  if (!X || !Xq4 || !s_x) return BITNET_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Xq4) || (gamma && !aligned16(gamma)) || (T_dbg && !aligned16(T_dbg)) ||
+      (reinterpret_cast<uintptr_t>(s_x) & 3u))
+    return BITNET_ERR_ALIGN;
+  int d = check_device();
+  if (d != BITNET_OK) return d;
+  int L = 0;
+  while ((int64_t(1) << L) < b) ++L;
+  return cuda_status(bitnet::run_hadamard_quant_i4(X, x_dtype == BITNET_BF16, (int)M, (int)K, L, gamma, eps,
+                                                   Xq4, s_x, T_dbg, static_cast<cudaStream_t>(stream)));
+}
+
+int bitnet_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
+                  int64_t M, int64_t N, int64_t K, void* Y, int y_dtype, int32_t* acc_dbg, void* stream) {
+  if (act_bits != 8 && act_bits != 4) return BITNET_ERR_DTYPE;
+  if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (M < 0 || M > (int64_t(1) << 30) || N < 1 || N > (int64_t(1) << 30) || K < 128 || K > 65536 ||
+      K % 128 != 0 || M * N >= (int64_t(1) << 40))
+    return BITNET_ERR_SHAPE;
+  if (M == 0) return BITNET_OK;
+  if (!Xq || !s_x || !pkW || !s_w || !Y) return BITNET_ERR_NULL;
+  if (!aligned16(Xq) || !aligned16(pkW) || !aligned16(Y) || (acc_dbg && !aligned16(acc_dbg)) ||
+      (reinterpret_cast<uintptr_t>(s_x) & 3u) || (reinterpret_cast<uintptr_t>(s_w) & 3u))
+    return BITNET_ERR_ALIGN;
+  int d = check_device();
+  if (d != BITNET_OK) return d;
+  if (!bitnet::tensor_map_encoder_available()) return BITNET_ERR_UNSUPPORTED;
+  return cuda_status(bitnet::run_linear(Xq, act_bits, s_x, pkW, s_w, (int)M, (int)N, (int)K, Y,
+                                        y_dtype == BITNET_BF16, acc_dbg, linear_path(),
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+int bitnet_set_linear_path(int path) {
+  if (path < 0 || path > 2) return BITNET_ERR_SHAPE;
+  g_linear_path.store(path, std::memory_order_relaxed);
+  return BITNET_OK;
+}
+
+int bitnet_device_error(int* code_out) {
+  int code = 0, zero = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) { cudaGetLastError(); return BITNET_ERR_CUDA; }
+  if (cudaMemcpyFromSymbol(&code, bitnet::g_device_error, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(bitnet::g_device_error, &zero, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return BITNET_ERR_CUDA;
+  }
+  if (code_out) *code_out = code;
+  return BITNET_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,435 @@
+// Activation quantisers of the BitLinear forward.
+//
+//  * quant_act_i8: RMSNorm, then per-token absmax int8 ("LLM을 1.58비트로
+//    파인튜닝: BitNet을 이용한 극단적인 양자화", section 양자화 메커니즘:
+//    absmax per token into [-128, 127], layer norm before the quantiser).
+//  * hadamard_quant_i4: RMSNorm, Walsh-Hadamard transform, per-token absmax
+//    int4 ("초저용량 LLM의 진화: BitNet v2 파헤치기", section 방법론: the
+//    H-BitLinear layer applies a Hadamard transform before 4-bit quantisation).
+//
+// Fixed arithmetic (fp32, round-to-nearest-even, no contraction):
+//   ss = sum of x*x by the balanced pairwise tree over element indices
+//        (zero padded to a power of two)
+//   r  = 1 / sqrt(ss / K + eps);  y = (x * r) * gamma
+//   s  = qmax / max(max|y|, 1e-5);  q = clamp(rint(y * s), qmin, qmax)
+// Hadamard: Sylvester order per block of b = 2^L elements, radix-2 stages of
+// stride 1, 2, ..., b/2 (pair (a, c) -> (a + c, a - c)), then times
+// c_b = fp32(1/sqrt(b)).  Codes are then taken from t with qmax = 7.
+#include "common.cuh"
+
+namespace bitnet {
+
+// ---------------------------------------------------------------------------
+// RMSNorm + int8: one CTA of NT threads per token.  Chunk j (16 bytes of
+// input: E elements) goes to thread j % NT in iteration j / NT, so the loads
+// are coalesced; the pairwise tree is then: E elements inside a chunk, the
+// NT threads (warp xor-shuffles, then warps in order), the IT iterations.
+// ---------------------------------------------------------------------------
+template <typename TIn> struct InVec;
+template <> struct InVec<float> {
+  static constexpr int E = 4;
+  static BN_DEV void load(const float* p, float (&v)[4]) {
+    uint4 u = ldg_nc_v4(p);
+    v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+    v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+  }
+};
+template <> struct InVec<uint16_t> {
+  static constexpr int E = 8;
+  static BN_DEV void load(const uint16_t* p, float (&v)[8]) {
+    uint4 u = ldg_nc_v4(p);
+    v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+    v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+  }
+};
+
+// Balanced tree over N (power of two) register values, in index order.
+template <int N>
+BN_DEV float tree_sum(float (&a)[N]) {
+#pragma unroll
+  for (int s = 1; s < N; s <<= 1) {
+#pragma unroll
+    for (int i = 0; i < N; i += 2 * s) a[i] = __fadd_rn(a[i], a[i + s]);
+  }
+  return a[0];
+}
+
+// Tree over the 32 lanes: after offsets 1, 2, 4, 8, 16 every lane holds the
+// sum in which lane pairs (2u, 2u+1), then quads, ... were combined in order.
+BN_DEV float warp_tree_sum(float v) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+template <typename TIn, int NT, int IT>
+__global__ void __launch_bounds__(NT)
+quant_act_i8_kernel(const TIn* __restrict__ X, int K, const float* __restrict__ gamma, float eps,
+                    int8_t* __restrict__ Xq, float* __restrict__ s_x) {
+  constexpr int E = InVec<TIn>::E;
+  constexpr int NW = NT / 32;
+  __shared__ float red[IT][NW];
+  __shared__ float wmax[NW];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int m = blockIdx.x;
+  const int C = K / E;                       // chunks in the row
+  const TIn* xrow = X + (size_t)m * K;
+
+  float v[IT][E];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int j = it * NT + tid;
+    if (j < C) {
+      InVec<TIn>::load(xrow + (size_t)j * E, v[it]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[it][e] = 0.f;
+    }
+  }
+
+  // ---- sum of squares, pairwise over element indices ----
+  float cs[IT];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    float sq[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) sq[e] = __fmul_rn(v[it][e], v[it][e]);
+    const float w = warp_tree_sum(tree_sum<E>(sq));
+    if (lane == 0) red[it][warp] = w;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    float p[NW];
+#pragma unroll
+    for (int w = 0; w < NW; ++w) p[w] = red[it][w];
+    cs[it] = tree_sum<NW>(p);
+  }
+  const float ss = tree_sum<IT>(cs);
+
+  const float ms = __fdiv_rn(ss, (float)K);
+  const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+
+  // ---- normalise, absmax ----
+  float amax = 0.f;
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int j = it * NT + tid;
+    if (gamma != nullptr && j < C) {
+      float g[4 * ((E + 3) / 4)];
+#pragma unroll
+      for (int q = 0; q < E / 4; ++q) {
+        uint4 u = ldg_nc_v4(gamma + (size_t)j * E + 4 * q);
+        g[4 * q] = __uint_as_float(u.x); g[4 * q + 1] = __uint_as_float(u.y);
+        g[4 * q + 2] = __uint_as_float(u.z); g[4 * q + 3] = __uint_as_float(u.w);
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[it][e] = __fmul_rn(__fmul_rn(v[it][e], r), g[e]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[it][e] = __fmul_rn(v[it][e], r);
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[it][e]));
+  }
+  amax = warp_max(amax);
+  if (lane == 0) wmax[warp] = amax;
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < NW; ++w) amax = fmaxf(amax, wmax[w]);
+
+  const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
+
+  // ---- codes ----
+  int8_t* qrow = Xq + (size_t)m * K;
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int j = it * NT + tid;
+    if (j >= C) continue;
+    uint32_t packed[E / 4];
+#pragma unroll
+    for (int q = 0; q < E / 4; ++q) {
+      uint32_t w = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        int c = __float2int_rn(__fmul_rn(v[it][4 * q + e], s));
+        c = max(-128, min(127, c));
+        w |= (uint32_t)(c & 0xFF) << (8 * e);
+      }
+      packed[q] = w;
+    }
+    if constexpr (E == 8) {
+      *reinterpret_cast<uint2*>(qrow + (size_t)j * E) = make_uint2(packed[0], packed[1]);
+    } else {
+      *reinterpret_cast<uint32_t*>(qrow + (size_t)j * E) = packed[0];
+    }
+  }
+  if (tid == 0) s_x[m] = s;
+}
+
+// ---------------------------------------------------------------------------
+// RMSNorm + Hadamard + int4.  Each thread owns 128 consecutive elements of a
+// token (G = K/128 threads per token, rounded up to a power of two GP; TPB
+// tokens per CTA).  Stages of stride < 128 run in registers; the stages of
+// stride 128 .. b/2 run after one transpose through shared memory, in which
+// a thread holds the elements whose index bits [a, 7) and the block index are
+// fixed (a = 14 - L), i.e. in-thread bits [0, a) and [7, L).
+// ---------------------------------------------------------------------------
+constexpr int HT_R = 128;                          // elements per thread
+
+BN_DEV int hpidx(int e) { return e + (e >> 7); }   // one pad word per 128
+
+// In-register radix-2 stages s = S0 .. S1-1 over v[c], where in-thread index
+// bit (s - SHIFT) is the element-index bit s.
+template <int S0, int S1, int SHIFT>
+BN_DEV void fwht_reg(float (&v)[HT_R]) {
+#pragma unroll
+  for (int s = S0; s < S1; ++s) {
+    constexpr int dummy = 0; (void)dummy;
+    const int h = 1 << (s - SHIFT);
+#pragma unroll
+    for (int c = 0; c < HT_R; ++c) {
+      if ((c & h) == 0) {
+        const float a = v[c], b = v[c + h];
+        v[c] = __fadd_rn(a, b);
+        v[c + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+}
+
+// Phase-2 in-thread index c -> element index inside the token row.
+template <int L>
+BN_DEV int phase2_elem(int tprime, int c) {
+  constexpr int A = 14 - L;                        // low in-thread bits
+  constexpr int MIDB = L - 7;                      // thread bits inside a block
+  const int blk = tprime >> MIDB;
+  const int mid = tprime & ((1 << MIDB) - 1);
+  const int within = ((c >> A) << 7) | (mid << A) | (c & ((1 << A) - 1));
+  return (blk << L) | within;
+}
+
+template <typename TIn, int L>
+__global__ void __launch_bounds__(128)
+hadamard_quant_i4_kernel(const TIn* __restrict__ X, int M, int K, int GP,
+                         const float* __restrict__ gamma, float eps, float cb,
+                         uint8_t* __restrict__ Xq4, float* __restrict__ s_x,
+                         float* __restrict__ T_dbg) {
+  extern __shared__ float hsm[];
+  const int G = K / HT_R;
+  const int TPB = blockDim.x / GP;
+  const int g = threadIdx.x / GP;                  // token slot in the CTA
+  const int t = threadIdx.x % GP;                  // thread inside the token
+  const int lane = threadIdx.x & 31;
+  const int m = blockIdx.x * TPB + g;
+  const bool active = (m < M) && (t < G);
+  const int rowpad = K + (K >> 7);
+  float* tok = hsm + (size_t)g * rowpad;
+  float* red = hsm + (size_t)TPB * rowpad;         // [TPB][4] partials
+
+  float v[HT_R];
+  if (active) {
+    const TIn* src = X + (size_t)m * K + (size_t)t * HT_R;
+    constexpr int E = InVec<TIn>::E;
+#pragma unroll
+    for (int q = 0; q < HT_R / E; ++q) {
+      float tmp[E];
+      InVec<TIn>::load(src + q * E, tmp);
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[q * E + e] = tmp[e];
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < HT_R; ++c) v[c] = 0.f;
+  }
+
+  // ---- sum of squares: in-thread subtree of 128, then threads in order ----
+  float part;
+  {
+    float sq[HT_R];
+#pragma unroll
+    for (int c = 0; c < HT_R; ++c) sq[c] = __fmul_rn(v[c], v[c]);
+    part = tree_sum<HT_R>(sq);
+  }
+  const int wl = GP < 32 ? GP : 32;                // lanes of one token inside a warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1)
+    if (o < wl) part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
+  float ss = part;
+  if (GP > 32) {                                   // 2 or 4 warps per token
+    if (lane == 0) red[g * 4 + (t >> 5)] = part;
+    __syncthreads();
+    float p[4] = {red[g * 4], red[g * 4 + 1], 0.f, 0.f};
+    if (GP == 64) {
+      ss = __fadd_rn(p[0], p[1]);
+    } else {
+      p[2] = red[g * 4 + 2]; p[3] = red[g * 4 + 3];
+      ss = __fadd_rn(__fadd_rn(p[0], p[1]), __fadd_rn(p[2], p[3]));
+    }
+  }
+  const float ms = __fdiv_rn(ss, (float)K);
+  const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+  if (active) {
+    if (gamma != nullptr) {
+      const float* gp = gamma + (size_t)t * HT_R;
+#pragma unroll
+      for (int c = 0; c < HT_R; ++c) v[c] = __fmul_rn(__fmul_rn(v[c], r), __ldg(gp + c));
+    } else {
+#pragma unroll
+      for (int c = 0; c < HT_R; ++c) v[c] = __fmul_rn(v[c], r);
+    }
+  }
+
+  // ---- Hadamard stages of stride 1 .. min(b, 128)/2 in registers ----
+  constexpr int P1 = L < 7 ? L : 7;
+  fwht_reg<0, P1, 0>(v);
+
+  if constexpr (L > 7) {
+    __syncthreads();                                // red[] reads above are done
+    if (active) {
+#pragma unroll
+      for (int c = 0; c < HT_R; ++c) tok[hpidx(t * HT_R + c)] = v[c];
+    }
+    __syncthreads();
+    if (active) {
+#pragma unroll
+      for (int c = 0; c < HT_R; ++c) v[c] = tok[hpidx(phase2_elem<L>(t, c))];
+    }
+    fwht_reg<7, L, 7 - (14 - L)>(v);
+    if (active) {
+#pragma unroll
+      for (int c = 0; c < HT_R; ++c) tok[hpidx(phase2_elem<L>(t, c))] = v[c];
+    }
+    __syncthreads();
+    if (active) {
+#pragma unroll
+      for (int c = 0; c < HT_R; ++c) v[c] = tok[hpidx(t * HT_R + c)];
+    }
+  }
+
+  // ---- normalise, absmax over the token ----
+  float amax = 0.f;
+#pragma unroll
+  for (int c = 0; c < HT_R; ++c) {
+    v[c] = __fmul_rn(v[c], cb);
+    amax = fmaxf(amax, fabsf(v[c]));
+  }
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1)
+    if (o < wl) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (GP > 32) {
+    __syncthreads();
+    if (lane == 0) red[g * 4 + (t >> 5)] = amax;
+    __syncthreads();
+    amax = fmaxf(fmaxf(red[g * 4], red[g * 4 + 1]),
+                 GP == 128 ? fmaxf(red[g * 4 + 2], red[g * 4 + 3]) : 0.f);
+  }
+  const float s = __fdiv_rn(7.0f, fmaxf(amax, 1e-5f));
+
+  if (!active) return;
+  if (T_dbg != nullptr) {
+    float* dst = T_dbg + (size_t)m * K + (size_t)t * HT_R;
+#pragma unroll
+    for (int c = 0; c < HT_R; c += 4)
+      *reinterpret_cast<float4*>(dst + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+  }
+  // 128 codes -> 64 bytes: code 2j in the low nibble, 2j+1 in the high nibble
+  uint32_t w[16];
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      int c = __float2int_rn(__fmul_rn(v[8 * q + e], s));
+      c = max(-8, min(7, c));
+      word |= (uint32_t)(c & 0xF) << (4 * e);
+    }
+    w[q] = word;
+  }
+  uint4* dst = reinterpret_cast<uint4*>(Xq4 + (size_t)m * (K / 2) + (size_t)t * (HT_R / 2));
+#pragma unroll
+  for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  if (t == 0) s_x[m] = s;
+}
+
+// ---------------------------------------------------------------------------
+// host launchers (called from abi.cu after validation)
+// ---------------------------------------------------------------------------
+template <typename TIn, int NT, int IT>
+static cudaError_t launch_q8(const void* X, int M, int K, const float* gamma, float eps,
+                             int8_t* Xq, float* s_x, cudaStream_t st) {
+  quant_act_i8_kernel<TIn, NT, IT><<<M, NT, 0, st>>>(static_cast<const TIn*>(X), K, gamma, eps, Xq, s_x);
+  return cudaGetLastError();
+}
+
+template <typename TIn>
+static cudaError_t dispatch_q8(const void* X, int M, int K, const float* gamma, float eps,
+                               int8_t* Xq, float* s_x, cudaStream_t st) {
+  constexpr int E = InVec<TIn>::E;
+  int C = K / E, PC = 1;
+  while (PC < C) PC <<= 1;
+  if (PC <= 1024) {
+    switch (PC <= 128 ? 1 : PC / 128) {
+      case 1: return launch_q8<TIn, 128, 1>(X, M, K, gamma, eps, Xq, s_x, st);
+      case 2: return launch_q8<TIn, 128, 2>(X, M, K, gamma, eps, Xq, s_x, st);
+      case 4: return launch_q8<TIn, 128, 4>(X, M, K, gamma, eps, Xq, s_x, st);
+      case 8: return launch_q8<TIn, 128, 8>(X, M, K, gamma, eps, Xq, s_x, st);
+    }
+  } else {
+    switch (PC / 256) {
+      case 8: return launch_q8<TIn, 256, 8>(X, M, K, gamma, eps, Xq, s_x, st);
+      case 16: return launch_q8<TIn, 256, 16>(X, M, K, gamma, eps, Xq, s_x, st);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t run_quant_act_i8(const void* X, int bf16, int M, int K, const float* gamma, float eps,
+                             int8_t* Xq, float* s_x, cudaStream_t st) {
+  return bf16 ? dispatch_q8<uint16_t>(X, M, K, gamma, eps, Xq, s_x, st)
+              : dispatch_q8<float>(X, M, K, gamma, eps, Xq, s_x, st);
+}
+
+template <typename TIn, int L>
+static cudaError_t launch_h4(const void* X, int M, int K, const float* gamma, float eps,
+                             uint8_t* Xq4, float* s_x, float* T_dbg, cudaStream_t st) {
+  const int G = K / HT_R;
+  int GP = 1;
+  while (GP < G) GP <<= 1;
+  const int TPB = GP >= 128 ? 1 : 128 / GP;
+  const int threads = TPB * GP;
+  const size_t smem = (size_t)TPB * (K + (K >> 7)) * sizeof(float) + (size_t)TPB * 4 * sizeof(float);
+  auto kern = hadamard_quant_i4_kernel<TIn, L>;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  const float cb = (float)(1.0 / sqrt((double)(1 << L)));
+  const int grid = (M + TPB - 1) / TPB;
+  kern<<<grid, threads, smem, st>>>(static_cast<const TIn*>(X), M, K, GP, gamma, eps, cb, Xq4, s_x, T_dbg);
+  return cudaGetLastError();
+}
+
+template <typename TIn>
+static cudaError_t dispatch_h4(const void* X, int M, int K, int L, const float* gamma, float eps,
+                               uint8_t* Xq4, float* s_x, float* T_dbg, cudaStream_t st) {
+  switch (L) {
+    case 5: return launch_h4<TIn, 5>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
+    case 6: return launch_h4<TIn, 6>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
+    case 7: return launch_h4<TIn, 7>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
+    case 8: return launch_h4<TIn, 8>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
+    case 9: return launch_h4<TIn, 9>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
+    case 10: return launch_h4<TIn, 10>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
+    case 11: return launch_h4<TIn, 11>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
+    case 12: return launch_h4<TIn, 12>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
+    case 13: return launch_h4<TIn, 13>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t run_hadamard_quant_i4(const void* X, int bf16, int M, int K, int L, const float* gamma,
+                                  float eps, uint8_t* Xq4, float* s_x, float* T_dbg, cudaStream_t st) {
+  return bf16 ? dispatch_h4<uint16_t>(X, M, K, L, gamma, eps, Xq4, s_x, T_dbg, st)
+              : dispatch_h4<float>(X, M, K, L, gamma, eps, Xq4, s_x, T_dbg, st);
+}
+
+}  // namespace bitnet

@@ -1,0 +1,164 @@
+/*
+ * bitnet.h - C ABI of the B200 (sm_100a) BitNet b1.58 BitLinear forward.
+ *
+ * The BitLinear layer replaces a linear layer by ternary weights {-1, 0, +1}
+ * and 8-bit activations; BitNet v2's H-BitLinear adds a Hadamard transform
+ * and 4-bit activations.  Sources, by page title and section:
+ *   [P1] "초저용량 LLM의 진화: BitNet v2 파헤치기 (1비트 LLM을 위한 4비트 활성화)",
+ *        section 방법론 (Hadamard before 4-bit activation quantisation).
+ *   [P2] "AI 혁신의 선두: 마이크로소프트의 1비트 LLM, BitNet b1.58 2B4T",
+ *        section 주요 아키텍처 혁신 (ternary weights by absmean; no bias terms).
+ *   [P4] "LLM을 1.58비트로 파인튜닝: BitNet을 이용한 극단적인 양자화",
+ *        sections 양자화 메커니즘 (absmean weight scale, per-token absmax int8,
+ *        norm before activation quantisation), 계산 패러다임 (integer matmul),
+ *        주요 결과 (four weights per int8), 추론 최적화 및 커스텀 커널 (unpack
+ *        weights on the fly inside the matmul).
+ *   [P5] "양자화(quantization) 1.58bit" (endplan.ai), absmax paragraph
+ *        (factor 127/absmax; dequantise by dividing by it).
+ *
+ * Conventions for every entry point:
+ *   - Pointers to tensors are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or keeps them.  `stream` is a cudaStream_t (NULL =
+ *     the legacy default stream).  Calls are asynchronous: they only enqueue
+ *     kernels (and, for bitnet_quantize_weights, one memset of the workspace).
+ *   - Row-major layouts: X [M][K] (M tokens, K input features), W [N][K]
+ *     (N output features), Y [M][N].
+ *   - Every argument is validated on the host before anything is enqueued; on
+ *     any error nothing is enqueued and a bitnet_status code is returned.
+ *     Launch failures return BITNET_ERR_CUDA (cudaGetLastError is consumed).
+ *   - Tensor pointers must be 16-byte aligned (BITNET_ERR_ALIGN).
+ *   - The current CUDA device must be sm_100 (BITNET_ERR_UNSUPPORTED).
+ *   - Fixed arithmetic: fp32 with IEEE round-to-nearest-even, no fused
+ *     multiply-add where a result decides an integer code.  Codes, packed
+ *     weights and int32 accumulators are deterministic and bit-exact.
+ */
+#ifndef BITNET_B200_H
+#define BITNET_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BITNET_API __attribute__((visibility("default")))
+#else
+#define BITNET_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BITNET_OK = 0,
+  BITNET_ERR_NULL = 1,         /* a required pointer is NULL */
+  BITNET_ERR_SHAPE = 2,        /* a size breaks the documented limits */
+  BITNET_ERR_ALIGN = 3,        /* a tensor pointer is not 16-byte aligned */
+  BITNET_ERR_DTYPE = 4,        /* unknown dtype or act_bits value */
+  BITNET_ERR_CUDA = 5,         /* a CUDA call or kernel launch failed */
+  BITNET_ERR_UNSUPPORTED = 6,  /* no sm_100 device, or the TMA encoder is missing */
+  BITNET_ERR_WORKSPACE = 7     /* workspace missing or too small */
+} bitnet_status;
+
+typedef enum { BITNET_F32 = 0, BITNET_BF16 = 1 } bitnet_dtype;
+
+/* Static description of a status code; never NULL, thread-safe. */
+BITNET_API const char* bitnet_status_string(int status);
+
+/* Version of this ABI (increments on any signature change). */
+BITNET_API int bitnet_abi_version(void);
+
+/* Bytes of workspace bitnet_quantize_weights needs (a small constant). */
+BITNET_API size_t bitnet_quantize_weights_workspace_size(int64_t N, int64_t K);
+
+/*
+ * Offline absmean ternarisation and packing of a weight matrix [P4 양자화
+ * 메커니즘, 주요 결과; P2 주요 아키텍처 혁신].
+ *   mean = (sum of |W| computed exactly, rounded once to fp64) / (N*K) in fp64,
+ *          rounded to fp32;  s_w = 1 / max(mean, 1e-5) in fp32;
+ *   q    = clamp(rint(W * s_w), -1, 1).
+ * W        : [N][K] fp32 or bf16 (w_dtype), finite values.
+ * pkW      : out, [N][K/4] bytes.  Codes are 2-bit two's complement (-1 = 0b11,
+ *            0 = 0b00, +1 = 0b01); in each little-endian 32-bit word holding
+ *            16 consecutive weights of a row, weight 4j+i sits at bits 8i+2j.
+ * s_w      : out, one fp32 on the device (the dequantisation uses 1/s_w).
+ * workspace: device scratch of at least bitnet_quantize_weights_workspace_size
+ *            bytes, 16-byte aligned, caller-owned; it is overwritten.
+ * Limits   : N >= 1, K >= 16, K % 16 == 0, N*K < 2^31.
+ */
+BITNET_API int bitnet_quantize_weights(const void* W, int w_dtype, int64_t N, int64_t K,
+                            uint8_t* pkW, float* s_w,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * BitLinear activation path: RMSNorm, then per-token absmax int8
+ * [P4 양자화 메커니즘; P5 absmax].  Per token (row of K values x):
+ *   ss = sum of x*x by the balanced pairwise tree over element indices
+ *        (zero padded to a power of two), fp32;
+ *   r  = 1 / sqrt(ss / K + eps);  y = (x * r) * gamma;
+ *   s_x = 127 / max(max|y|, 1e-5);  Xq = clamp(rint(y * s_x), -128, 127).
+ * X     : [M][K] fp32 or bf16 (x_dtype).
+ * gamma : [K] fp32, or NULL for all ones.
+ * Xq    : out, [M][K] int8.   s_x: out, [M] fp32 (the dequantisation uses 1/s_x).
+ * Limits: M >= 0 (M == 0 is a no-op), 16 <= K <= 16384, K % 16 == 0.
+ */
+BITNET_API int bitnet_quant_act(const void* X, int x_dtype, int64_t M, int64_t K,
+                     const float* gamma, float eps, int8_t* Xq, float* s_x, void* stream);
+
+/*
+ * H-BitLinear activation path: RMSNorm, Walsh-Hadamard transform, per-token
+ * absmax int4 [P1 방법론].  y as in bitnet_quant_act; then per block of
+ * b = 2^L consecutive features the Sylvester-order transform by radix-2 stages
+ * of stride 1, 2, ..., b/2 (pair (a, c) -> (a + c, a - c)), times
+ * fp32(1/sqrt(b)), giving t;  s_x = 7 / max(max|t|, 1e-5);
+ * codes = clamp(rint(t * s_x), -8, 7).
+ * had_block: b, a power of two in [32, 8192] dividing K, or 0 for the largest
+ *            power of two dividing K.
+ * Xq4  : out, [M][K/2] bytes; code 2j in the low nibble of byte j, code 2j+1
+ *        in the high nibble, two's complement.
+ * s_x  : out, [M] fp32.
+ * T_dbg: out, [M][K] fp32 transformed values t, or NULL (diagnostics only).
+ * Limits: M >= 0, 128 <= K <= 16384, K % 128 == 0.
+ */
+BITNET_API int bitnet_hadamard_quant_act(const void* X, int x_dtype, int64_t M, int64_t K,
+                              const float* gamma, float eps, int had_block,
+                              uint8_t* Xq4, float* s_x, float* T_dbg, void* stream);
+
+/*
+ * Ternary x int8 (act_bits = 8) or ternary x int4 (act_bits = 4) product with
+ * int32 accumulation and dequantisation [P4 계산 패러다임, 추론 최적화 및
+ * 커스텀 커널, 양자화 메커니즘 ("rescaled"); P5 (divide by the factor)]:
+ *   acc[m][n] = sum_k code_x[m][k] * w[n][k]      (exact int32)
+ *   Y[m][n]   = float(acc) * ((1 / s_x[m]) * (1 / s_w))   in fp32,
+ *   rounded to bf16 (nearest even) when y_dtype is BITNET_BF16.  No bias.
+ * Xq     : [M][K] int8 (act_bits 8) or [M][K/2] packed int4 (act_bits 4).
+ * s_x    : [M] fp32 from the matching quantiser.   s_w: one fp32 (device).
+ * pkW    : [N][K/4] packed ternary weights from bitnet_quantize_weights.
+ * Y      : out, [M][N] fp32 or bf16 (y_dtype).
+ * acc_dbg: out, [M][N] int32 accumulators, or NULL (diagnostics only).
+ * Limits : M >= 0, N >= 1, 128 <= K <= 65536, K % 128 == 0.
+ */
+BITNET_API int bitnet_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW,
+                  const float* s_w, int64_t M, int64_t N, int64_t K,
+                  void* Y, int y_dtype, int32_t* acc_dbg, void* stream);
+
+/*
+ * Diagnostics: selects the kernel family bitnet_linear uses in this process.
+ * 0 = automatic (default), 1 = CUDA-core dp4a kernel, 2 = tcgen05 tensor-core
+ * kernel.  Both compute the same bit-exact result.  Returns BITNET_ERR_SHAPE
+ * for any other value.
+ */
+BITNET_API int bitnet_set_linear_path(int path);
+
+/*
+ * Reads and clears the library's device-side error flag on the current
+ * device (synchronises the device).  A kernel that waited more than ~2 s on
+ * a pipeline barrier gives up, records a nonzero code here and returns; 0
+ * means no such event.  Returns BITNET_OK or BITNET_ERR_CUDA.
+ */
+BITNET_API int bitnet_device_error(int* code_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITNET_B200_H */

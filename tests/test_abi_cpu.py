@@ -1,0 +1,100 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/bitnet.h declares, and rejects bad arguments on the
+host before touching CUDA (no compute call is made here)."""
+import ctypes
+
+import pytest
+
+from bitlinear_bitnet_quant_b200 import api, build_lib
+
+ALIGNED = 0x10000          # fake device addresses: never dereferenced, validation fails first
+MISALIGNED = 0x10008
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_lib.build()
+    return api.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = api.header_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(api._SIGNATURES)
+
+
+def test_status_strings(L):
+    for code in range(8):
+        assert api.status_string(code)
+    assert api.status_string(0) == "ok"
+    assert api.status_string(99) == "unknown status"
+    assert L.bitnet_abi_version() == 1
+    assert L.bitnet_quantize_weights_workspace_size(4096, 4096) >= 80
+
+
+def _linear(L, **kw):
+    a = dict(Xq=ALIGNED, act_bits=8, s_x=ALIGNED, pkW=ALIGNED, s_w=ALIGNED, M=4, N=256, K=256,
+             Y=ALIGNED, y_dtype=0, acc=None)
+    a.update(kw)
+    return L.bitnet_linear(a["Xq"], a["act_bits"], a["s_x"], a["pkW"], a["s_w"], a["M"], a["N"], a["K"],
+                           a["Y"], a["y_dtype"], a["acc"], None)
+
+
+def test_linear_validation(L):
+    assert _linear(L, act_bits=5) == 4
+    assert _linear(L, y_dtype=7) == 4
+    assert _linear(L, K=100) == 2
+    assert _linear(L, K=64) == 2
+    assert _linear(L, K=65536 + 128) == 2
+    assert _linear(L, N=0) == 2
+    assert _linear(L, M=-1) == 2
+    assert _linear(L, M=0) == 0                 # empty batch: nothing to do
+    assert _linear(L, Xq=None) == 1
+    assert _linear(L, Y=None) == 1
+    assert _linear(L, Xq=MISALIGNED) == 3
+    assert _linear(L, pkW=MISALIGNED) == 3
+    assert _linear(L, acc=MISALIGNED) == 3
+    assert _linear(L, s_w=ALIGNED + 2) == 3
+
+
+def test_quant_act_validation(L):
+    q = lambda **kw: L.bitnet_quant_act(kw.get("X", ALIGNED), kw.get("dt", 1), kw.get("M", 4), kw.get("K", 256),
+                                        kw.get("gamma"), 1e-6, kw.get("Xq", ALIGNED), kw.get("s", ALIGNED), None)
+    assert q(dt=3) == 4
+    assert q(K=24) == 2 and q(K=0) == 2 and q(K=16384 + 16) == 2
+    assert q(M=0) == 0
+    assert q(X=None) == 1 and q(s=None) == 1
+    assert q(X=MISALIGNED) == 3 and q(gamma=MISALIGNED) == 3
+
+
+def test_hadamard_validation(L):
+    h = lambda **kw: L.bitnet_hadamard_quant_act(kw.get("X", ALIGNED), 1, kw.get("M", 4), kw.get("K", 1024), None,
+                                                 1e-6, kw.get("b", 0), kw.get("Xq", ALIGNED), ALIGNED,
+                                                 kw.get("T"), None)
+    assert h(K=1000) == 2
+    assert h(b=48) == 2            # not a power of two
+    assert h(b=16) == 2            # below the smallest block
+    assert h(b=2048) == 2          # does not divide K
+    assert h(K=128 * 3, b=256) == 2
+    assert h(M=0) == 0
+    assert h(Xq=None) == 1
+    assert h(T=MISALIGNED) == 3
+
+
+def test_weights_validation(L):
+    w = lambda **kw: L.bitnet_quantize_weights(kw.get("W", ALIGNED), kw.get("dt", 0), kw.get("N", 16),
+                                               kw.get("K", 64), kw.get("pk", ALIGNED), ALIGNED,
+                                               kw.get("ws", ALIGNED), kw.get("wsb", 128), None)
+    assert w(dt=2) == 4
+    assert w(K=24) == 2 and w(N=0) == 2 and w(N=1 << 20, K=1 << 12) == 2
+    assert w(ws=None) == 7 and w(wsb=8) == 7
+    assert w(W=None) == 1
+    assert w(pk=MISALIGNED) == 3
+
+
+def test_linear_path_selector(L):
+    assert L.bitnet_set_linear_path(3) == 2
+    assert L.bitnet_set_linear_path(-1) == 2
+    assert L.bitnet_set_linear_path(0) == 0

@@ -1,0 +1,279 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Bar: codes, packed weights, scales and int32 accumulators bit-exact; fp32
+outputs bit-exact to the oracle's fixed fp32 formula and within 1e-5 relative
+of its float64 rescale; bf16 outputs equal the round-to-nearest-even of the
+oracle's fp32 output.  Hadamard outputs bit-exact, and within 1e-5 of the
+largest magnitude of a float64 transform of the same normalised input.
+"""
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+from bitlinear_bitnet_quant_b200 import workloads as wl  # noqa: E402
+from oracle import bitnet_oracle as O  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+api = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    global api
+    from bitlinear_bitnet_quant_b200 import api as _api, build_lib
+    build_lib.build()
+    api = _api
+    api.lib()
+    yield
+    assert api.bitnet_device_error() == 0
+
+
+def dev(a: np.ndarray, dtype=None) -> "torch.Tensor":
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype == "bf16":
+        t = t.view(torch.int16).view(torch.bfloat16) if a.dtype == np.uint16 else t.to(torch.bfloat16)
+    return t.cuda()
+
+
+def x_inputs(x, dtype):
+    """(device tensor, fp32 values the oracle sees) for fp32 values or bf16 bits."""
+    if dtype == "bf16":
+        bits = x if x.dtype == np.uint16 else wl.f32_to_bf16_bits(x)
+        return dev(bits, "bf16"), O.bf16_bits_to_f32(bits)
+    return dev(x.astype(np.float32)), x.astype(np.float32)
+
+
+def host(t):
+    return t.cpu().numpy()
+
+
+# ------------------------------------------------------------------ weights --
+
+@pytest.mark.parametrize("N,K,dtype", [(256, 256, "f32"), (384, 1024, "f32"), (128, 2560, "bf16"),
+                                       (130, 48, "f32"), (6912, 2560, "f32")])
+def test_quantize_weights(N, K, dtype):
+    w = wl.weights(N, K, seed=N + K)
+    if dtype == "bf16":
+        bits = wl.f32_to_bf16_bits(w)
+        wd, w_or = dev(bits, "bf16"), O.bf16_bits_to_f32(bits)
+    else:
+        wd, w_or = dev(w), w
+    pk, s_w = api.bitnet_quantize_weights(wd)
+    pk_o, s_o, q_o = O.quantize_weights(w_or)
+    assert host(s_w)[0].view(np.uint32) == np.float32(s_o).view(np.uint32)
+    assert np.array_equal(host(pk), pk_o)
+
+
+def test_quantize_weights_edge_cases():
+    zero = np.zeros((128, 64), np.float32)
+    pk, s_w = api.bitnet_quantize_weights(dev(zero))
+    assert host(s_w)[0] == np.float32(1.0) / np.float32(1e-5) and not host(pk).any()
+    rng = np.random.default_rng(1)
+    wide = (rng.standard_normal((64, 256)) * np.exp2(rng.integers(-140, 120, (64, 256)))).astype(np.float32)
+    wide[0, :4] = [1e-45, -1e-44, 3e38, -2e-38]
+    pk, s_w = api.bitnet_quantize_weights(dev(wide))
+    pk_o, s_o, _ = O.quantize_weights(wide)
+    assert host(s_w)[0] == s_o and np.array_equal(host(pk), pk_o)
+    const = np.full((32, 32), -0.02, np.float32)
+    pk, s_w = api.bitnet_quantize_weights(dev(const))
+    pk_o, s_o, q_o = O.quantize_weights(const)
+    assert host(s_w)[0] == s_o and np.array_equal(host(pk), pk_o) and np.all(q_o == -1)
+
+
+# ------------------------------------------------------------------ int8 act --
+
+@pytest.mark.parametrize("M,K,dtype,use_gamma", [
+    (1, 16, "f32", False), (3, 48, "bf16", True), (17, 256, "f32", False), (8, 256, "f32", True),
+    (16, 2560, "bf16", False), (129, 4096, "bf16", False), (5, 2048, "bf16", True),
+    (7, 5632, "bf16", False), (2, 16384, "bf16", False), (3, 16384, "f32", True), (33, 1040, "f32", False)])
+def test_quant_act(M, K, dtype, use_gamma):
+    x = wl.add_entry_outliers(np.random.default_rng(M * K), wl.gaussian(np.random.default_rng(K), (M, K)),
+                              0.005, 30.0)
+    xd, x_or = x_inputs(x, dtype)
+    gamma = np.random.default_rng(7).uniform(0.5, 1.5, K).astype(np.float32) if use_gamma else None
+    q, s = api.bitnet_quant_act(xd, dev(gamma) if use_gamma else None, 1e-6)
+    q_o, s_o = O.quant_act(x_or, gamma, 1e-6)
+    assert np.array_equal(host(s).view(np.uint32), s_o.view(np.uint32))
+    assert np.array_equal(host(q), q_o)
+
+
+def test_quant_act_edge_rows():
+    K = 512
+    x = np.zeros((6, K), np.float32)
+    x[1, 100] = 3.5                            # single spike
+    x[2, :] = np.where(np.arange(K) % 2 == 0, 2.0, -2.0)   # every element at +-absmax
+    x[3, :] = 1e-30                            # tiny but nonzero
+    x[4, :] = np.linspace(-1, 1, K)
+    x[5, :7] = [6e4, -6e4, 1, 2, 3, 4, 5]      # large values
+    for dtype in ("f32", "bf16"):
+        xd, x_or = x_inputs(x, dtype)
+        q, s = api.bitnet_quant_act(xd, None, 1e-6)
+        q_o, s_o = O.quant_act(x_or, None, 1e-6)
+        assert np.array_equal(host(s), s_o) and np.array_equal(host(q), q_o)
+    assert np.all(q_o[0] == 0) and q_o[1, 100] == 127 and np.all(np.abs(q_o[2]) == 127)
+
+
+def test_quant_act_full_prefill():
+    c = wl.prefill(with_weights=False)
+    xd, x_or = x_inputs(c["x"], "bf16")
+    q, s = api.bitnet_quant_act(xd, None, 1e-6)
+    q_o, s_o = O.quant_act(x_or, None, 1e-6)
+    assert np.array_equal(host(s), s_o) and np.array_equal(host(q), q_o)
+
+
+# ------------------------------------------------------------------ Hadamard --
+
+def _check_hadamard(x, dtype, had_block, gamma=None):
+    xd, x_or = x_inputs(x, dtype)
+    q4, s, t = api.bitnet_hadamard_quant_act(xd, dev(gamma) if gamma is not None else None, 1e-6,
+                                             had_block, want_t=True)
+    pk_o, s_o, q_o, t_o = O.hadamard_quant_act(x_or, gamma, 1e-6, had_block)
+    assert np.array_equal(host(t).view(np.uint32), t_o.view(np.uint32))
+    assert np.array_equal(host(s), s_o)
+    assert np.array_equal(host(q4), pk_o)
+    # against a float64 transform of the same normalised input
+    b = had_block or O.default_had_block(x.shape[1])
+    y, _ = O.rms_norm(x_or, gamma, 1e-6)
+    y64 = y.astype(np.float64).reshape(y.shape[0], -1, b)
+    h = 1
+    while h < b:
+        v = y64.reshape(y.shape[0], -1, b // (2 * h), 2, h)
+        y64 = np.stack([v[..., 0, :] + v[..., 1, :], v[..., 0, :] - v[..., 1, :]], axis=-2).reshape(y64.shape)
+        h *= 2
+    t64 = y64.reshape(y.shape) / math.sqrt(b)
+    err = np.abs(host(t).astype(np.float64) - t64).max(axis=1)
+    assert np.all(err <= 1e-5 * np.abs(t64).max(axis=1) + 1e-30)
+
+
+@pytest.mark.parametrize("M,K,b,dtype", [
+    (1, 128, 0, "f32"), (5, 256, 32, "bf16"), (33, 1024, 64, "bf16"), (3, 1024, 256, "f32"),
+    (9, 2048, 0, "bf16"), (7, 5632, 0, "bf16"), (4, 8192, 0, "bf16"), (2, 8192, 1024, "f32"),
+    (130, 4096, 4096, "bf16"), (3, 16384, 8192, "bf16"), (17, 1536, 512, "f32")])
+def test_hadamard_quant(M, K, b, dtype):
+    rng = np.random.default_rng(M + K + b)
+    x = wl.add_channel_outliers(rng, wl.student_t(rng, (M, K)), 0.005, 50.0)
+    _check_hadamard(x, dtype, b)
+
+
+def test_hadamard_gamma_and_edges():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((6, 1024)).astype(np.float32)
+    x[0] = 0
+    x[1] = 0; x[1, 17] = 2.0
+    x[2] = 1.0
+    _check_hadamard(x, "f32", 0, rng.uniform(0.5, 2, 1024).astype(np.float32))
+
+
+def test_hadamard_full_config():
+    c = wl.hbitlinear(with_weights=False)
+    _check_hadamard(c["x"], "bf16", 0)
+
+
+# ------------------------------------------------------------------ linear ----
+
+def _random_codes(M, N, K, act_bits, seed):
+    rng = np.random.default_rng(seed)
+    lo, hi = (-128, 128) if act_bits == 8 else (-8, 8)
+    qx = rng.integers(lo, hi, size=(M, K)).astype(np.int8)
+    qw = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    s_x = rng.uniform(0.5, 200, size=M).astype(np.float32)
+    return qx, qw, s_x, np.float32(rng.uniform(5, 60))
+
+
+def _run_linear(qx, qw, s_x, s_w, act_bits, out, path):
+    api.bitnet_set_linear_path(path)
+    try:
+        xq_dev = dev(qx) if act_bits == 8 else dev(O.pack_int4(qx))
+        Y, acc = api.bitnet_linear(xq_dev, act_bits, dev(s_x), dev(O.pack_ternary(qw)),
+                                   dev(np.array([s_w], np.float32)),
+                                   out_dtype=torch.float32 if out == "f32" else torch.bfloat16, want_acc=True)
+        torch.cuda.synchronize()
+    finally:
+        api.bitnet_set_linear_path(0)
+    return Y, acc
+
+
+def _check_linear(qx, qw, s_x, s_w, act_bits, out, path, rows=None):
+    Y, acc = _run_linear(qx, qw, s_x, s_w, act_bits, out, path)
+    Y, acc = host(Y.float() if out == "bf16" else Y), host(acc)
+    if rows is not None:
+        Y, acc, qx, s_x = Y[rows], acc[rows], qx[rows], s_x[rows]
+    acc_o, y_o = O.linear(qx, s_x, qw, s_w)
+    assert np.array_equal(acc, acc_o)
+    if out == "f32":
+        assert np.array_equal(Y.view(np.uint32), y_o.view(np.uint32))
+        ref = O.dequantize_f64(acc_o, s_x, s_w)
+        nz = acc_o != 0
+        assert np.max(np.abs(Y[nz] - ref[nz]) / np.abs(ref[nz]), initial=0) <= 1e-5
+    else:
+        assert np.array_equal(O.bf16_round(Y), O.bf16_round(y_o))
+
+
+@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("M,N,K,act_bits,out", [
+    (1, 128, 128, 8, "f32"), (2, 256, 256, 8, "f32"), (3, 256, 256, 8, "bf16"), (16, 384, 1024, 8, "f32"),
+    (17, 400, 256, 8, "f32"), (100, 256, 2560, 8, "bf16"), (129, 256, 512, 8, "f32"),
+    (300, 272, 384, 8, "f32"), (257, 128, 1024, 8, "f32"),
+    (1, 128, 256, 4, "f32"), (5, 256, 1024, 4, "f32"), (33, 400, 512, 4, "bf16"), (200, 256, 2048, 4, "f32")])
+def test_linear_random_codes(M, N, K, act_bits, out, path):
+    qx, qw, s_x, s_w = _random_codes(M, N, K, act_bits, M * 7 + N + K)
+    _check_linear(qx, qw, s_x, s_w, act_bits, out, path)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_linear_decode_full(M):
+    c = wl.decode(M)
+    xd, x_or = x_inputs(c["x"], "bf16")
+    pk, s_w = api.bitnet_quantize_weights(dev(c["w"]))
+    q, s = api.bitnet_quant_act(xd, None, 1e-6)
+    Y, acc = api.bitnet_linear(q, 8, s, pk, s_w, want_acc=True)
+    pk_o, s_wo, qw_o = O.quantize_weights(c["w"])
+    q_o, s_o = O.quant_act(x_or, None, 1e-6)
+    acc_o, y_o = O.linear(q_o, s_o, qw_o, s_wo)
+    assert np.array_equal(host(acc), acc_o)
+    assert np.array_equal(host(Y).view(np.uint32), y_o.view(np.uint32))
+
+
+def test_linear_prefill_sampled():
+    c = wl.prefill()
+    xd, x_or = x_inputs(c["x"], "bf16")
+    pk, s_w = api.bitnet_quantize_weights(dev(c["w"]))
+    q, s = api.bitnet_quant_act(xd, None, 1e-6)
+    Y, acc = api.bitnet_linear(q, 8, s, pk, s_w, out_dtype=torch.bfloat16, want_acc=True)
+    rows = np.random.default_rng(0).choice(c["M"], size=12, replace=False)
+    rows = np.concatenate([rows, [0, c["M"] - 1]])
+    _, s_wo, qw_o = O.quantize_weights(c["w"])
+    q_o, s_o = O.quant_act(x_or[rows], None, 1e-6)
+    acc_o, y_o = O.linear(q_o, s_o, qw_o, s_wo)
+    assert np.array_equal(host(acc)[rows], acc_o)
+    assert np.array_equal(O.bf16_round(host(Y.float())[rows]), O.bf16_round(y_o))
+
+
+def test_hbitlinear_sampled():
+    c = wl.hbitlinear()
+    xd, x_or = x_inputs(c["x"], "bf16")
+    pk, s_w = api.bitnet_quantize_weights(dev(c["w"]))
+    q4, s, _ = api.bitnet_hadamard_quant_act(xd, None, 1e-6, 0)
+    Y, acc = api.bitnet_linear(q4, 4, s, pk, s_w, want_acc=True)
+    rows = np.concatenate([np.random.default_rng(1).choice(c["M"], size=14, replace=False), [0, c["M"] - 1]])
+    _, s_wo, qw_o = O.quantize_weights(c["w"])
+    _, s_o, q_o, _ = O.hadamard_quant_act(x_or[rows], None, 1e-6, 0)
+    acc_o, y_o = O.linear(q_o, s_o, qw_o, s_wo)
+    assert np.array_equal(host(acc)[rows], acc_o)
+    assert np.array_equal(host(Y)[rows].view(np.uint32), y_o.view(np.uint32))
+
+
+def test_tiny_bitlinear_forward():
+    c = wl.tiny()
+    pk, s_w = api.bitnet_quantize_weights(dev(c["w"]))
+    Y = api.bitlinear_forward(dev(c["x"]), pk, s_w)
+    _, s_wo, qw_o = O.quantize_weights(c["w"])
+    out = O.bitlinear(c["x"], qw_o, s_wo)
+    assert np.array_equal(host(Y), out["y"])
+    ref = O.fake_quant_matmul_f64(out["codes"], out["s_x"], qw_o, s_wo)
+    nz = out["acc"] != 0
+    assert np.max(np.abs(host(Y)[nz] - ref[nz]) / np.abs(ref[nz])) <= 1e-5
