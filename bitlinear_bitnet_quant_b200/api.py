@@ -31,6 +31,8 @@ _SIGNATURES = {
     "bitnet_quantize_weights_workspace_size": (ctypes.c_size_t, [_i64, _i64]),
     "bitnet_quantize_weights": (ctypes.c_int, [_c_void_p, ctypes.c_int, _i64, _i64, _c_void_p, _c_void_p,
                                                _c_void_p, ctypes.c_size_t, _c_void_p]),
+    "bitnet_quantize_weights_noalloc": (ctypes.c_int, [_c_void_p, ctypes.c_int, _i64, _i64, _c_void_p,
+                                                       _c_void_p, _c_void_p]),
     "bitnet_quant_act": (ctypes.c_int, [_c_void_p, ctypes.c_int, _i64, _i64, _c_void_p, ctypes.c_float,
                                         _c_void_p, _c_void_p, _c_void_p]),
     "bitnet_hadamard_quant_act": (ctypes.c_int, [_c_void_p, ctypes.c_int, _i64, _i64, _c_void_p, ctypes.c_float,
@@ -124,6 +126,17 @@ def bitnet_quantize_weights(W: torch.Tensor, pkW=None, s_w=None, workspace=None,
     _check("bitnet_quantize_weights", lib().bitnet_quantize_weights(
         _ptr(W), _dtype_code(W), N, K, _ptr(pkW), _ptr(s_w), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+    return pkW, s_w
+
+
+def bitnet_quantize_weights_noalloc(W: torch.Tensor, pkW: torch.Tensor, s_w: torch.Tensor, stream=None):
+    """Same as bitnet_quantize_weights, but the library allocates nothing: the
+    caller passes the outputs, and the scratch is a fixed array in the library."""
+    _require(W, "W")
+    _require(pkW, "pkW")
+    N, K = W.shape
+    _check("bitnet_quantize_weights_noalloc", lib().bitnet_quantize_weights_noalloc(
+        _ptr(W), _dtype_code(W), N, K, _ptr(pkW), _ptr(s_w), _stream(stream)))
     return pkW, s_w
 
 

@@ -90,6 +90,28 @@ BITNET_API int bitnet_quantize_weights(const void* W, int w_dtype, int64_t N, in
                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Variant of bitnet_quantize_weights for callers that cannot allocate device
+ * memory (no counterpart on the pages; this is a deployment convenience).
+ * Examples: a plugin inside an application that owns every device allocation,
+ * a runtime that reserves all of its memory up front, code that must avoid the
+ * implicit synchronisation of cudaMalloc/cudaFree.  Same arguments, result and
+ * bit-exact output as bitnet_quantize_weights, minus the workspace: the scratch
+ * is a fixed 256-byte array inside this library's device memory, held on every
+ * device that uses it until the library is unloaded.  The caller still owns W,
+ * pkW and s_w.  No cudaMalloc, cudaFree or allocating routine is called.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array and clears it before use; calls whose
+ *     kernels overlap on the GPU (e.g. on two streams) race on it.
+ *   - Limit: N*K <= BITNET_NOALLOC_MAX_WEIGHTS (what the fixed 64-bit counters
+ *     absorb without overflow); larger tensors return BITNET_ERR_SHAPE.
+ */
+#define BITNET_NOALLOC_MAX_WEIGHTS 2147483647LL
+BITNET_API int bitnet_quantize_weights_noalloc(const void* W, int w_dtype, int64_t N, int64_t K,
+                                               uint8_t* pkW, float* s_w, void* stream);
+
+/*
  * BitLinear activation path: RMSNorm, then per-token absmax int8
  * [P4 양자화 메커니즘; P5 absmax].  Per token (row of K values x):
  *   ss = sum of x*x by the balanced pairwise tree over element indices
