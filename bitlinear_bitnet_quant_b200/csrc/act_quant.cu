@@ -71,6 +71,8 @@ quant_act_i8_kernel(const TIn* __restrict__ X, int K, const float* __restrict__ 
   __shared__ float red[IT][NW];
   __shared__ float wmax[NW];
 
+  pdl_launch_dependents();
+  pdl_wait();                                // X may come from, and Xq may still be read by, the previous kernel
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int m = blockIdx.x;
   const int C = K / E;                       // chunks in the row
@@ -217,6 +219,8 @@ hadamard_quant_i4_kernel(const TIn* __restrict__ X, int M, int K, int GP,
                          uint8_t* __restrict__ Xq4, float* __restrict__ s_x,
                          float* __restrict__ T_dbg) {
   extern __shared__ float hsm[];
+  pdl_launch_dependents();
+  pdl_wait();                                // X may come from, and Xq4 may still be read by, the previous kernel
   const int G = K / HT_R;
   const int TPB = blockDim.x / GP;
   const int g = threadIdx.x / GP;                  // token slot in the CTA
@@ -359,8 +363,8 @@ hadamard_quant_i4_kernel(const TIn* __restrict__ X, int M, int K, int GP,
 template <typename TIn, int NT, int IT>
 static cudaError_t launch_q8(const void* X, int M, int K, const float* gamma, float eps,
                              int8_t* Xq, float* s_x, cudaStream_t st) {
-  quant_act_i8_kernel<TIn, NT, IT><<<M, NT, 0, st>>>(static_cast<const TIn*>(X), K, gamma, eps, Xq, s_x);
-  return cudaGetLastError();
+  return launch_pdl(quant_act_i8_kernel<TIn, NT, IT>, dim3(M), dim3(NT), 0, st, 1u,
+                    static_cast<const TIn*>(X), K, gamma, eps, Xq, s_x);
 }
 
 template <typename TIn>
@@ -405,8 +409,8 @@ static cudaError_t launch_h4(const void* X, int M, int K, const float* gamma, fl
   if (e != cudaSuccess) return e;
   const float cb = (float)(1.0 / sqrt((double)(1 << L)));
   const int grid = (M + TPB - 1) / TPB;
-  kern<<<grid, threads, smem, st>>>(static_cast<const TIn*>(X), M, K, GP, gamma, eps, cb, Xq4, s_x, T_dbg);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, 1u, static_cast<const TIn*>(X), M, K, GP, gamma,
+                    eps, cb, Xq4, s_x, T_dbg);
 }
 
 template <typename TIn>

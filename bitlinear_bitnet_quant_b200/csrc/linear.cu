@@ -44,7 +44,8 @@ BN_DEV void widen8(uint32_t p, uint32_t& lo4, uint32_t& hi4) {
 
 // ===========================================================================
 // SIMT kernel: one warp per output row n and block of 16 tokens; lanes split
-// K; dp4a accumulation.  Used for very small M and as a second GPU path.
+// K; dp4a accumulation.  A second, independent GPU implementation, selected
+// only through bitnet_set_linear_path (the tcgen05 kernel is faster at every M).
 // ===========================================================================
 template <int ACT_BITS, typename TOut>
 __global__ void __launch_bounds__(256)
@@ -52,6 +53,8 @@ linear_simt_kernel(const uint8_t* __restrict__ Xq, const float* __restrict__ s_x
                    const uint32_t* __restrict__ pkW, const float* __restrict__ s_w_ptr,
                    int M, int N, int K, TOut* __restrict__ Y, int32_t* __restrict__ acc_dbg) {
   constexpr int MT = 16;
+  pdl_launch_dependents();
+  pdl_wait();                                // Xq and s_x come from the previous kernel
   const int lane = threadIdx.x & 31;
   const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int m0 = blockIdx.y * MT;
@@ -106,11 +109,16 @@ linear_simt_kernel(const uint8_t* __restrict__ Xq, const float* __restrict__ s_x
 // operand B = the activation tile, brought by TMA into shared memory with the
 // 128-byte swizzle (int4 tiles are widened there by the converter warps);
 // D = int32 accumulators in tensor memory.
-//   warp 0   : TMA producer
-//   warp 1   : tensor-memory allocator and MMA issuer (one thread)
-//   warps 2-5: converters, then the epilogue (tensor-memory lanes 32*(w%4)..)
+//   warp 0    : TMA producer (and the per-token dequantisation scales)
+//   warp 1    : tensor-memory allocator and MMA issuer (one thread)
+//   warps 2-9 : converters, then the epilogue.  Warp w serves tensor-memory
+//               lanes 32*(w%4).. and half (w-2)/4 of the K bytes of a step
+//               (and of the token columns in the epilogue).
+// When the tiles alone leave SMs idle, K is split over a cluster of ksplit
+// CTAs (grid z); partial sums travel to the leader by one bulk copy each.
 // ===========================================================================
-constexpr int TC_THREADS = 192;
+constexpr int TC_THREADS = 320;
+constexpr int TC_CONV_THREADS = 256;
 constexpr int TC_BK = 128;
 constexpr int TC_WBYTES = 128 * TC_BK / 4;       // packed W tile: 128 rows x 32 B
 
@@ -119,26 +127,63 @@ struct TcCfg {
   static constexpr int XBYTES = BN * 128;                      // int8 operand tile
   static constexpr int XRAW = ACT_BITS == 4 ? BN * 64 : 0;     // packed int4 tile
   static constexpr int STAGE = XBYTES + XRAW + TC_WBYTES;
-  static constexpr int S_SMEM = (200 * 1024) / STAGE;
-  static constexpr int S_TMEM = (512 - BN) / 32;
+  // One accumulator: measured on B200, rotating tcgen05.mma over several
+  // accumulators costs ~3x more per instruction than chaining into one.
+  static constexpr int DCOLS = BN;                             // accumulator columns
+  // 256 columns: two CTAs share an SM, so one CTA's prologue and epilogue
+  // overlap the other's MMAs (a 256-token tile needs all 512 columns)
+  static constexpr int TMEM_BUDGET = BN <= 128 ? 256 : 512;
+  static constexpr int SMEM_BUDGET = TMEM_BUDGET == 256 ? 108 * 1024 : 200 * 1024;
+  static constexpr int S_SMEM = SMEM_BUDGET / STAGE;
+  static constexpr int S_TMEM = (TMEM_BUDGET - DCOLS) / 32;
   static constexpr int S0 = S_SMEM < S_TMEM ? S_SMEM : S_TMEM;
   static constexpr int S = S0 > 6 ? 6 : S0;
-  static constexpr int COLS_NEEDED = BN + 32 * S;
+  static constexpr int COLS_NEEDED = DCOLS + 32 * S;
   static constexpr int TMEM_COLS = COLS_NEEDED <= 32 ? 32 : COLS_NEEDED <= 64 ? 64 :
                                    COLS_NEEDED <= 128 ? 128 : COLS_NEEDED <= 256 ? 256 : 512;
   static constexpr size_t SMEM = (size_t)S * STAGE + 1024;
+  static constexpr int HALF = BN / 2;                          // token columns per epilogue warp
   static_assert(S >= 2, "pipeline needs two stages");
+  static_assert((size_t)BN * 128 * 4 <= (size_t)S * STAGE, "output staging fits in the operand stages");
 };
 
+// G chunks of NC (8 or 16) consecutive columns of this thread's TMEM lane,
+// starting at taddr, with a single wait for all of them.
+template <int NC, int G>
+BN_DEV void load_cols(uint32_t taddr, uint32_t (&v)[G][16]) {
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    if constexpr (NC == 8) {
+      uint32_t t[8];
+      tmem_ld8(taddr + (uint32_t)(g * NC), t);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[g][q] = t[q];
+    } else {
+      tmem_ld16(taddr + (uint32_t)(g * NC), v[g]);
+    }
+  }
+  tmem_wait_ld();
+}
+
 template <int BN, int ACT_BITS, typename TOut>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(TC_THREADS, BN <= 128 ? 2 : 1)
 linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                 const __grid_constant__ CUtensorMap tmY, int use_tma_store,
                  const float* __restrict__ s_x, const float* __restrict__ s_w_ptr,
-                 int M, int N, int K, TOut* __restrict__ Y, int32_t* __restrict__ acc_dbg) {
+                 int M, int N, int K, int ksplit, TOut* __restrict__ Y, int32_t* __restrict__ acc_dbg) {
   using C = TcCfg<BN, ACT_BITS>;
   constexpr int S = C::S;
+  constexpr uint32_t XTX = ACT_BITS == 8 ? BN * 128 : BN * 64;      // activation bytes per stage
+  constexpr uint32_t PART_BYTES = 128u * BN * 4u;                    // one split-K partial tile
+  constexpr int NC = C::HALF < 16 ? C::HALF : 16;                    // epilogue column chunk
+  constexpr int NCH = C::HALF / NC;                                  // chunks per epilogue warp
+  constexpr int G = NCH < 2 ? NCH : 2;                               // chunks per TMEM-load wait
   extern __shared__ uint8_t dsmem_raw[];
-  __shared__ __align__(8) uint64_t bar_full[S], bar_empty[S], bar_conv[S], bar_acc;
+  // wfull: weight tile landed; xfull: activation tile landed; conv: weights in TMEM (and, for
+  // int4, activations widened); empty: stage free; acc: all MMAs done; sdq: scales ready;
+  // red: split-K partials of the other ranks landed (leader only)
+  __shared__ __align__(8) uint64_t bar_wfull[S], bar_xfull[S], bar_empty[S], bar_conv[S];
+  __shared__ __align__(8) uint64_t bar_acc, bar_sdq, bar_red;
   __shared__ uint32_t tmem_base_sh;
   __shared__ float sdq[BN];
 
@@ -146,20 +191,32 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
   auto xs = [&](int s) { return base + (size_t)s * C::XBYTES; };                          // 1024-aligned
   auto xraw = [&](int s) { return base + (size_t)S * C::XBYTES + (size_t)s * C::XRAW; };
   auto ws = [&](int s) { return base + (size_t)S * (C::XBYTES + C::XRAW) + (size_t)s * TC_WBYTES; };
+  // split-K partial sums, [slot][column][row] int32: in the leader, slot r-1 receives rank r;
+  // in the other ranks, slot 0 stages the outgoing partial
+  int32_t* red = reinterpret_cast<int32_t*>(base + (size_t)S * C::STAGE);
+  // output staging for the TMA store, [token][128 features] (reuses the activation stages)
+  TOut* ostage = reinterpret_cast<TOut*>(base);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * 128;
   const int m0 = blockIdx.y * BN;
-  const int nk = K / TC_BK;
+  const int kr = blockIdx.z;                    // rank inside the cluster (cluster = 1 x 1 x ksplit)
+  const int nk_all = K / TC_BK;
+  const int kb = (int)((int64_t)nk_all * kr / ksplit);
+  const int nk = (int)((int64_t)nk_all * (kr + 1) / ksplit) - kb;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&bar_full[s], 1);
-      mbar_init(&bar_empty[s], 1 + 4);
-      mbar_init(&bar_conv[s], 4);
+      mbar_init(&bar_wfull[s], 1);
+      mbar_init(&bar_xfull[s], 1);
+      mbar_init(&bar_empty[s], 1 + 8);
+      mbar_init(&bar_conv[s], 8);
     }
     mbar_init(&bar_acc, 1);
+    mbar_init(&bar_sdq, 1);
+    mbar_init(&bar_red, 1);
     fence_barrier_init();
+    if (kr == 0 && ksplit > 1) mbar_arrive_expect_tx(&bar_red, (uint32_t)(ksplit - 1) * PART_BYTES);
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
   }
@@ -169,27 +226,60 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
   }
   tc_fence_before();
   __syncthreads();
+  if (ksplit > 1) cluster_arrive();            // matched by a cluster_wait before any remote access
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  // Only now, with this CTA's tensor memory held, may the next kernel in the
+  // stream be scheduled: a dependent CTA never takes tensor memory that a CTA
+  // of this grid still has to allocate (later grids only wait on earlier ones).
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    const int pre = nk < S ? nk : S;
     if (lane == 0) {
-      constexpr uint32_t XTX = ACT_BITS == 8 ? BN * 128 : BN * 64;
-      int issued = 0;
-      for (int i = 0; i < nk; ++i) {
+      // weights do not depend on the previous kernel: start streaming them now
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&bar_wfull[i], TC_WBYTES);
+        tma_load_2d(ws(i), &tmW, &bar_wfull[i], (kb + i) * (TC_BK / 4), n0);
+      }
+    }
+    __syncwarp();
+    pdl_wait();                                    // activations and s_x come from the previous kernel
+    auto load_x = [&](int i) {
+      const int s = i % S;
+      mbar_arrive_expect_tx(&bar_xfull[s], XTX);
+      if constexpr (ACT_BITS == 8) tma_load_2d(xs(s), &tmX, &bar_xfull[s], (kb + i) * TC_BK, m0);
+      else tma_load_2d(xraw(s), &tmX, &bar_xfull[s], (kb + i) * (TC_BK / 2), m0);
+    };
+    if (lane == 0)
+      for (int i = 0; i < pre; ++i) load_x(i);    // first: the activations are on the critical path
+    if (kr == 0) {
+      if (lane == 0 && use_tma_store) tma_prefetch_desc(&tmY);
+      const float sw = __ldg(s_w_ptr);
+      for (int j = lane; j < BN; j += 32) {
+        const int m = m0 + j;
+        sdq[j] = m < M ? dequant_scale(__ldg(s_x + m), sw) : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_sdq);
+    }
+    if (lane == 0) {
+      int issued = pre;
+      for (int i = pre; i < nk; ++i) {
         const int s = i % S, r = i / S;
-        if (r > 0 && !mbar_wait(&bar_empty[s], (r - 1) & 1, DEV_ERR_TIMEOUT_EMPTY)) break;
-        mbar_arrive_expect_tx(&bar_full[s], TC_WBYTES + XTX);
-        tma_load_2d(ws(s), &tmW, &bar_full[s], i * (TC_BK / 4), n0);
-        if constexpr (ACT_BITS == 8) tma_load_2d(xs(s), &tmX, &bar_full[s], i * TC_BK, m0);
-        else tma_load_2d(xraw(s), &tmX, &bar_full[s], i * (TC_BK / 2), m0);
+        if (!mbar_wait(&bar_empty[s], (r - 1) & 1, DEV_ERR_TIMEOUT_EMPTY)) break;
+        mbar_arrive_expect_tx(&bar_wfull[s], TC_WBYTES);
+        tma_load_2d(ws(s), &tmW, &bar_wfull[s], (kb + i) * (TC_BK / 4), n0);
+        load_x(i);
         issued = i + 1;
       }
       // every copy issued has landed before the CTA may exit (returns at once
       // on the normal path, where the consumers have already waited for them)
-      for (int i = issued - S < 0 ? 0 : issued - S; i < issued; ++i)
-        mbar_wait(&bar_full[i % S], (i / S) & 1, DEV_ERR_TIMEOUT_FULL, false);
+      for (int i = issued - S < 0 ? 0 : issued - S; i < issued; ++i) {
+        mbar_wait(&bar_wfull[i % S], (i / S) & 1, DEV_ERR_TIMEOUT_FULL, false);
+        mbar_wait(&bar_xfull[i % S], (i / S) & 1, DEV_ERR_TIMEOUT_FULL, false);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -197,17 +287,17 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       constexpr uint32_t IDESC = idesc_i8(128, BN);
       for (int i = 0; i < nk; ++i) {
         const int s = i % S, r = i / S;
-        if (!mbar_wait(&bar_full[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
+        if (!mbar_wait(&bar_xfull[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
         if (!mbar_wait(&bar_conv[s], r & 1, DEV_ERR_TIMEOUT_A)) break;
         tc_fence_after();
         const uint32_t xaddr = smem_u32(xs(s));
 #pragma unroll
         for (int kk = 0; kk < TC_BK / 32; ++kk) {
           const uint64_t bdesc = smem_desc_k_sw128(xaddr + kk * 32);
-          const uint32_t aaddr = tmem + (uint32_t)(BN + 32 * s + 8 * kk);
+          const uint32_t aaddr = tmem + (uint32_t)(C::DCOLS + 32 * s + 8 * kk);
           mma_i8_ts(tmem, aaddr, bdesc, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&bar_empty[s]);
+        if (i + S < nk) mma_commit(&bar_empty[s]);   // only stages that are refilled need releasing
       }
       mma_commit(&bar_acc);
       mbar_wait(&bar_acc, 0, DEV_ERR_TIMEOUT_ACC, false);   // no MMA in flight at teardown
@@ -215,36 +305,36 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
   } else {
     // ------------------------------------------------------------ converters
     const int q = warp & 3;                      // tensor-memory lane quarter
+    const int h = (warp - 2) >> 2;               // which half of the K bytes / token columns
     const int row = 32 * q + lane;               // output feature inside the tile
-    const int ct = threadIdx.x - 64;             // 0..127
-    const float sw = __ldg(s_w_ptr);
-    for (int j = ct; j < BN; j += 128) {
-      const int m = m0 + j;
-      sdq[j] = m < M ? dequant_scale(__ldg(s_x + m), sw) : 0.f;
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const int ct = threadIdx.x - 64;             // 0..255
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
 
+    int signalled = 0;                           // steps whose conv barrier has been arrived on
     for (int i = 0; i < nk; ++i) {
       const int s = i % S, r = i / S;
-      if (!mbar_wait_warp(&bar_full[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
+      if (!mbar_wait_warp(&bar_wfull[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
       tc_fence_after();
-      // weights: 128 values of this row -> 32 tensor-memory columns
-      const uint4* wp = reinterpret_cast<const uint4*>(ws(s) + 32 * row);
-      const uint4 w0 = wp[0], w1 = wp[1];
-      const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-      uint32_t a[32];
+      // 64 weights of this row -> 16 tensor-memory columns
+      const uint4 w = *reinterpret_cast<const uint4*>(ws(s) + 32 * row + 16 * h);
+      if constexpr (ACT_BITS == 8) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_empty[s]);   // packed tile consumed
+      }
+      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+      uint32_t a[16];
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
+      for (int g = 0; g < 4; ++g) {
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) a[4 * g + jj] = unpack4(wv[g], jj);
       }
-      tmem_st32(lane_base + (uint32_t)(BN + 32 * s), a);
+      tmem_st16(lane_base + (uint32_t)(C::DCOLS + 32 * s + 16 * h), a);
       if constexpr (ACT_BITS == 4) {
         // int4 activation tile: widen to int8 (16*x) in the 128-byte-swizzled layout
+        if (!mbar_wait_warp(&bar_xfull[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
         uint8_t* dst = xs(s);
         const uint8_t* src = xraw(s);
-        for (int idx = ct; idx < BN * 8; idx += 128) {
+        for (int idx = ct; idx < BN * 8; idx += TC_CONV_THREADS) {
           const int rr = idx >> 3, c = idx & 7;
           const uint2 p = *reinterpret_cast<const uint2*>(src + 64 * rr + 8 * c);
           uint32_t o0, o1, o2, o3;
@@ -253,36 +343,94 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
           *reinterpret_cast<uint4*>(dst + 128 * rr + 16 * (c ^ (rr & 7))) = make_uint4(o0, o1, o2, o3);
         }
         fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_empty[s]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bar_conv[s]);
-        mbar_arrive(&bar_empty[s]);
+      // Signal the MMA issuer in bursts: wait for the tensor-memory stores once
+      // for every run of steps whose weights had already landed.
+      const int nx = i + 1;
+      const bool more = nx < nk && __all_sync(0xffffffffu, mbar_test(&bar_wfull[nx % S], (nx / S) & 1));
+      if (!more) {
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+          for (int j = signalled; j <= i; ++j) mbar_arrive(&bar_conv[j % S]);
+        signalled = i + 1;
       }
     }
 
     // ------------------------------------------------------------ epilogue
-    if (mbar_wait_warp(&bar_acc, 0, DEV_ERR_TIMEOUT_ACC)) {
-      tc_fence_after();
-      const int n = n0 + row;
-      constexpr int SHIFT = ACT_BITS == 8 ? 6 : 10;
+    constexpr int SHIFT = ACT_BITS == 8 ? 6 : 10;
+    const int cbeg = h * C::HALF;                // this warp's token columns
+    const bool acc_ok = mbar_wait_warp(&bar_acc, 0, DEV_ERR_TIMEOUT_ACC);
+    tc_fence_after();
+    if (kr > 0) {
+      // split-K partner: stage the raw partial sums, then one bulk copy to the leader
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(lane_base + (uint32_t)c0, v);
-        tmem_wait_ld();
-        if (n < N) {
+      for (int g0 = 0; g0 < NCH; g0 += G) {
+        uint32_t v[G][16];
+        load_cols<NC, G>(lane_base + (uint32_t)(cbeg + g0 * NC), v);
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int m = m0 + c0 + jj;
-            if (m < M) {
-              const int acc = (int)v[jj] >> SHIFT;
-              if (acc_dbg) acc_dbg[(size_t)m * N + n] = acc;
-              store_out(Y + (size_t)m * N + n, __fmul_rn((float)acc, sdq[c0 + jj]));
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int jj = 0; jj < NC; ++jj)
+            red[(cbeg + (g0 + g) * NC + jj) * 128 + row] = acc_ok ? (int32_t)v[g][jj] : 0;
+      }
+      fence_proxy_async_smem();
+      cluster_wait();                              // the leader's barrier is initialised
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (ct == 0) {
+        const uint32_t dst = cluster_map(smem_u32(red), 0) + (uint32_t)(kr - 1) * PART_BYTES;
+        bulk_copy_to_cluster(dst, red, PART_BYTES, cluster_map(smem_u32(&bar_red), 0));
+        bulk_wait_read();                          // the source may be released after this
+      }
+    } else {
+      if (ksplit > 1) cluster_wait();
+      const bool sdq_ok = mbar_wait_warp(&bar_sdq, 0, DEV_ERR_TIMEOUT_ACC);
+      const bool red_ok = ksplit == 1 || mbar_wait_cluster(&bar_red, 0, DEV_ERR_TIMEOUT_CLUSTER);
+      const bool ok = acc_ok && red_ok && sdq_ok;
+      const int n = n0 + row;
+#pragma unroll 1
+      for (int g0 = 0; g0 < NCH; g0 += G) {
+        uint32_t v[G][16];
+        load_cols<NC, G>(lane_base + (uint32_t)(cbeg + g0 * NC), v);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const int c0 = cbeg + (g0 + g) * NC;
+          for (int pr = 1; pr < ksplit; ++pr) {
+#pragma unroll
+            for (int jj = 0; jj < NC; ++jj) v[g][jj] += (uint32_t)red[((pr - 1) * BN + c0 + jj) * 128 + row];
+          }
+          if (use_tma_store) {
+#pragma unroll
+            for (int jj = 0; jj < NC; ++jj) {
+              const int acc = (int)v[g][jj] >> SHIFT;
+              float y = __fmul_rn((float)acc, sdq[c0 + jj]);
+              if (!ok) y = 0.f;
+              store_out(ostage + (size_t)(c0 + jj) * 128 + row, y);
+            }
+          } else if (ok && n < N) {
+#pragma unroll
+            for (int jj = 0; jj < NC; ++jj) {
+              const int m = m0 + c0 + jj;
+              if (m < M) {
+                const int acc = (int)v[g][jj] >> SHIFT;
+                if (acc_dbg) acc_dbg[(size_t)m * N + n] = acc;
+                store_out(Y + (size_t)m * N + n, __fmul_rn((float)acc, sdq[c0 + jj]));
+              }
             }
           }
+        }
+      }
+      if (use_tma_store) {
+        // the staged tile leaves as one bulk tensor store (rows past M and
+        // columns past N are dropped by the copy engine)
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (ct == 0 && ok) {
+          tma_store_2d(&tmY, ostage, n0, m0);
+          bulk_wait_all();
         }
       }
     }
@@ -294,6 +442,7 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  if (ksplit > 1 && warp < 2) cluster_wait();     // pairs this warp's cluster_arrive
 }
 
 // ===========================================================================
@@ -317,36 +466,68 @@ static EncodeFn get_encode() {
   return fn;
 }
 
-static bool make_map_2d(CUtensorMap* map, const void* ptr, uint64_t inner_bytes, uint64_t rows,
-                        uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+static bool make_map_2d(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, uint64_t inner, uint64_t rows,
+                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
   EncodeFn enc = get_encode();
   if (!enc) return false;
-  cuuint64_t dims[2] = {inner_bytes, rows};
-  cuuint64_t strides[1] = {inner_bytes};
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+static bool make_map_bytes(CUtensorMap* map, const void* ptr, uint64_t inner_bytes, uint64_t rows,
+                           uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  return make_map_2d(map, ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, inner_bytes, rows, inner_bytes, box_inner, box_rows, sw);
+}
+
+template <typename T> struct MapType;
+template <> struct MapType<float> { static constexpr CUtensorMapDataType v = CU_TENSOR_MAP_DATA_TYPE_FLOAT32; };
+template <> struct MapType<__nv_bfloat16> { static constexpr CUtensorMapDataType v = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; };
 
 template <int BN, int ACT_BITS, typename TOut>
 static cudaError_t launch_tc(const void* Xq, const float* s_x, const uint8_t* pkW, const float* s_w,
                              int M, int N, int K, void* Y, int32_t* acc_dbg, cudaStream_t st) {
   using C = TcCfg<BN, ACT_BITS>;
-  CUtensorMap tmW, tmX;
-  if (!make_map_2d(&tmW, pkW, (uint64_t)K / 4, (uint64_t)N, TC_BK / 4, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+  CUtensorMap tmW, tmX, tmY;
+  if (!make_map_bytes(&tmW, pkW, (uint64_t)K / 4, (uint64_t)N, TC_BK / 4, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   const bool ok = ACT_BITS == 8
-      ? make_map_2d(&tmX, Xq, (uint64_t)K, (uint64_t)M, TC_BK, BN, CU_TENSOR_MAP_SWIZZLE_128B)
-      : make_map_2d(&tmX, Xq, (uint64_t)K / 2, (uint64_t)M, TC_BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
+      ? make_map_bytes(&tmX, Xq, (uint64_t)K, (uint64_t)M, TC_BK, BN, CU_TENSOR_MAP_SWIZZLE_128B)
+      : make_map_bytes(&tmX, Xq, (uint64_t)K / 2, (uint64_t)M, TC_BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
+  // The output leaves through one TMA store per tile when rows are 16-byte
+  // multiples; the diagnostics accumulators take the per-element path.
+  int use_tma_store = acc_dbg == nullptr && ((uint64_t)N * sizeof(TOut)) % 16 == 0;
+  if (use_tma_store && !make_map_2d(&tmY, Y, MapType<TOut>::v, (uint64_t)N, (uint64_t)M, (uint64_t)N * sizeof(TOut),
+                                     128, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    use_tma_store = 0;
+  if (!use_tma_store) tmY = tmX;                   // unused
+  // Split K across a cluster when the output tiles alone leave most SMs idle
+  // (decode): each rank streams a K range, partial sums meet in the leader.
+  const int tiles = ((N + 127) / 128) * ((M + BN - 1) / BN);
+  const int nk = K / TC_BK;
+  int ksplit = 1;
+  if (BN <= 32) {
+    int sms = 148, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    while (ksplit < 8 && tiles * ksplit * 2 <= 2 * sms && ksplit * 2 <= nk) ksplit *= 2;
+  }
+  size_t smem = C::SMEM + (size_t)(ksplit - 1) * 128 * BN * sizeof(int32_t);
+  // Never more CTAs per SM than tensor memory can serve at once (512 columns):
+  // a CTA blocked in tcgen05.alloc behind cluster peers waiting at the cluster
+  // barrier would never run.  Shared memory (228 KB per SM) enforces the bound.
+  const size_t min_smem = (size_t)(228 * 1024) / (512 / C::TMEM_COLS + 1) + 1024;
+  if (smem < min_smem) smem = min_smem;
   auto kern = linear_tc_kernel<BN, ACT_BITS, TOut>;
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), C::SMEM);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((N + 127) / 128, (M + BN - 1) / BN);
-  kern<<<grid, TC_THREADS, C::SMEM, st>>>(tmW, tmX, s_x, s_w, M, N, K, static_cast<TOut*>(Y), acc_dbg);
-  return cudaGetLastError();
+  dim3 grid((N + 127) / 128, (M + BN - 1) / BN, ksplit);
+  return launch_pdl(kern, grid, dim3(TC_THREADS), smem, st, (unsigned)ksplit, tmW, tmX, tmY, use_tma_store,
+                    s_x, s_w, M, N, K, ksplit, static_cast<TOut*>(Y), acc_dbg);
 }
 
 template <int ACT_BITS, typename TOut>
@@ -355,18 +536,16 @@ static cudaError_t dispatch_tc(const void* Xq, const float* s_x, const uint8_t* 
   if (M <= 16) return launch_tc<16, ACT_BITS, TOut>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st);
   if (M <= 32) return launch_tc<32, ACT_BITS, TOut>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st);
   if (M <= 64) return launch_tc<64, ACT_BITS, TOut>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st);
-  if (M <= 128) return launch_tc<128, ACT_BITS, TOut>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st);
-  return launch_tc<256, ACT_BITS, TOut>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st);
+  return launch_tc<128, ACT_BITS, TOut>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st);
 }
 
 template <int ACT_BITS, typename TOut>
 static cudaError_t launch_simt(const void* Xq, const float* s_x, const uint8_t* pkW, const float* s_w,
                                int M, int N, int K, void* Y, int32_t* acc_dbg, cudaStream_t st) {
   dim3 grid((N + 7) / 8, (M + 15) / 16);
-  linear_simt_kernel<ACT_BITS, TOut><<<grid, 256, 0, st>>>(
-      static_cast<const uint8_t*>(Xq), s_x, reinterpret_cast<const uint32_t*>(pkW), s_w, M, N, K,
-      static_cast<TOut*>(Y), acc_dbg);
-  return cudaGetLastError();
+  return launch_pdl(linear_simt_kernel<ACT_BITS, TOut>, grid, dim3(256), 0, st, 1u,
+                    static_cast<const uint8_t*>(Xq), s_x, reinterpret_cast<const uint32_t*>(pkW), s_w, M, N, K,
+                    static_cast<TOut*>(Y), acc_dbg);
 }
 
 bool tensor_map_encoder_available() { return get_encode() != nullptr; }
@@ -374,7 +553,7 @@ bool tensor_map_encoder_available() { return get_encode() != nullptr; }
 // path: 0 = automatic, 1 = SIMT, 2 = tcgen05
 cudaError_t run_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                        int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, int path, cudaStream_t st) {
-  const bool tc = path == 2 || (path == 0 && M > 2);
+  const bool tc = path != 1;          // the dp4a kernel is a diagnostics path (slower at every M)
 #define BN_LIN(BITS, T)                                                                  \
   return tc ? dispatch_tc<BITS, T>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st)           \
             : launch_simt<BITS, T>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st)

@@ -165,8 +165,8 @@ BITNET_API int bitnet_linear(const void* Xq, int act_bits, const float* s_x, con
 
 /*
  * Diagnostics: selects the kernel family bitnet_linear uses in this process.
- * 0 = automatic (default), 1 = CUDA-core dp4a kernel, 2 = tcgen05 tensor-core
- * kernel.  Both compute the same bit-exact result.  Returns BITNET_ERR_SHAPE
+ * 0 = automatic (default: the tcgen05 tensor-core kernel), 1 = CUDA-core dp4a
+ * kernel, 2 = tcgen05 kernel.  Both compute the same bit-exact result.  Returns BITNET_ERR_SHAPE
  * for any other value.
  */
 BITNET_API int bitnet_set_linear_path(int path);

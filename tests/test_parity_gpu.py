@@ -218,7 +218,8 @@ def _check_linear(qx, qw, s_x, s_w, act_bits, out, path, rows=None):
     (1, 128, 128, 8, "f32"), (2, 256, 256, 8, "f32"), (3, 256, 256, 8, "bf16"), (16, 384, 1024, 8, "f32"),
     (17, 400, 256, 8, "f32"), (100, 256, 2560, 8, "bf16"), (129, 256, 512, 8, "f32"),
     (300, 272, 384, 8, "f32"), (257, 128, 1024, 8, "f32"),
-    (1, 128, 256, 4, "f32"), (5, 256, 1024, 4, "f32"), (33, 400, 512, 4, "bf16"), (200, 256, 2048, 4, "f32")])
+    (1, 128, 256, 4, "f32"), (5, 256, 1024, 4, "f32"), (33, 400, 512, 4, "bf16"), (200, 256, 2048, 4, "f32"),
+    (16, 1024, 2560, 4, "f32"), (32, 1152, 2560, 8, "bf16"), (9, 128, 128, 8, "f32")])
 def test_linear_random_codes(M, N, K, act_bits, out, path):
     qx, qw, s_x, s_w = _random_codes(M, N, K, act_bits, M * 7 + N + K)
     _check_linear(qx, qw, s_x, s_w, act_bits, out, path)
