@@ -50,12 +50,13 @@ METRIC = "BitLinear tokens/sec and GB/s|TOPS vs HBM/int8 roofline, 1xB200"
 # ----------------------------------------------------------------------------
 
 WORKLOADS = {
-    # name: (builder, eps)
     "decode": lambda: wl.decode(16, with_weights=False),
     "prefill": lambda: wl.prefill(with_weights=False),
     "hbitlinear": lambda: wl.hbitlinear(with_weights=False),
     "tiny": lambda: wl.tiny(),
 }
+CHAIN_WORKLOADS = {"chain_decode": 32, "chain_prefill": 512}    # tokens per step
+CHAIN_LAYERS = 24
 
 
 def kernel_source_hash() -> str:
@@ -158,6 +159,37 @@ class ClockSampler:
 # our implementation
 # ----------------------------------------------------------------------------
 
+def max_over_ranks(ms: float, world: int, dev) -> float:
+    """The slowest rank's time (every rank takes this collective step)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed_replay(g, stream, world, dev) -> float:
+    """One warm replay, then a timed replay between CUDA events on the
+    launching stream, with a barrier and a device synchronise on both sides."""
+    import torch
+    import torch.distributed as dist
+    g.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    return max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -229,24 +261,7 @@ def run_ours(args, rank, world, local_rank):
         return g
 
     def timed(g):
-        g.replay()                      # untimed replay: warms the graph itself
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        g.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return timed_replay(g, stream, world, dev)
 
     steps = args.steps
     g_step = graph_of(step, steps)
@@ -286,12 +301,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_step(i)
     e1.record(stream)
     torch.cuda.synchronize()
-    t_e2e = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([t_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_e2e = float(t.item())
-        dist.barrier()
+    t_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
 
     if rank != 0:
         return None
@@ -341,6 +351,142 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
     }
     return line
+
+
+def run_chain(args, rank, world, local_rank):
+    """24 stacked layers (hidden 2048, FFN 5632) on M tokens per step."""
+    import torch
+    import torch.distributed as dist
+
+    from bitlinear_bitnet_quant_b200 import api, build_lib, chain
+
+    build_lib.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    M = CHAIN_WORKLOADS[args.workload]
+    H, F = wl.CHAIN_HIDDEN, wl.CHAIN_FFN
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + rank)
+    layers = []
+    for _ in range(CHAIN_LAYERS):          # N(0, 0.02) weights drawn on the device, quantised offline
+        w = {name: torch.randn((n, k), generator=g, device=dev) * 0.02 for name, n, k, _ in wl.CHAIN_PROJ}
+        layers.append(chain.quantize_layer(w))
+        del w
+    torch.cuda.synchronize()
+    ch = chain.BitLinearChain(layers, M, H, F, dev)
+    x = torch.from_numpy(wl.chain_input(M)).to(dev)
+
+    warmup = max(3, args.warmup)
+    for _ in range(warmup):
+        ch.forward(x, stream)
+    torch.cuda.synchronize()
+
+    def graph_of(fn):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for _ in range(args.steps):
+                fn()
+        return gr
+
+    def lin_only():                          # the chain's linear layers alone, same operands
+        for w in layers:
+            for name, Xq, sx, Y, bits in (("q", ch.xq, ch.sx, ch.q, 8), ("k", ch.xq, ch.sx, ch.k, 8),
+                                          ("v", ch.xq, ch.sx, ch.v, 8), ("o", ch.v4, ch.sv, ch.o, 4),
+                                          ("up", ch.hq, ch.sh, ch.up, 8), ("gate", ch.hq, ch.sh, ch.gate, 8),
+                                          ("down", ch.a4, ch.sa, ch.d, 4)):
+                api.bitnet_linear(Xq, bits, sx, *w[name], Y=Y, stream=stream)
+
+    g_step = graph_of(lambda: ch.forward(x, stream))
+    g_lin = graph_of(lin_only)
+    visible = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    clocks = ClockSampler(visible[local_rank] if local_rank < len(visible) else str(local_rank))
+    clocks.start()
+    t_step = timed_replay(g_step, stream, world, dev)
+    t_lin = timed_replay(g_lin, stream, world, dev)
+    clk = clocks.stop()
+
+    # e2e: host input in, host output back, through the Python API
+    x_pin = torch.empty((M, H), dtype=torch.float32).pin_memory()
+    x_pin.copy_(x.cpu())
+    y_pin = torch.empty((M, H), dtype=torch.float32).pin_memory()
+    for _ in range(warmup):
+        x.copy_(x_pin, non_blocking=True)
+        y_pin.copy_(ch.forward(x, stream), non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        x.copy_(x_pin, non_blocking=True)
+        y_pin.copy_(ch.forward(x, stream), non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    steps = args.steps
+    step_s = t_step / steps / 1e3
+    lin_s = t_lin / steps / 1e3                       # all 7 x 24 linear launches of one step
+    packed = ch.packed_bytes()
+    ops = 2.0 * M * sum(n * k for _, n, k, _ in wl.CHAIN_PROJ) * CHAIN_LAYERS
+    act_bytes = CHAIN_LAYERS * M * (4 * (5 * H + 3 * F) + 2 * H + H // 2 + F // 2 + 7 * 4)
+    if M <= 64:
+        roof = {"bound": "hbm", "achieved": (packed + act_bytes) / lin_s / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "kernel": "bitnet_linear, all 168 launches of a step",
+                "algorithmic_bytes_per_step": packed + act_bytes}
+    else:
+        roof = {"bound": "tensor", "achieved": ops / lin_s / 1e12, "peak": 2.0 * peaks["bf16_tflops"],
+                "unit": "TOPS", "kernel": "bitnet_linear, all 168 launches of a step",
+                "algorithmic_ops_per_step": ops, "peak_note": "2 x measured bf16 burst (nominal int8/bf16 ratio)"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = profiled_traffic(f"linear_{args.workload}")
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    tokens = M * world
+    return {
+        "metric": METRIC, "value": tokens * steps / (t_step / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": steps, "warmup": warmup, "ms_per_step": t_step / steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8/int4 x ternary -> int32, fp32 glue",
+        "data": "synthetic",
+        "config": {"workload": f"bitlinear_chain_{CHAIN_LAYERS}layers_m{M}_hidden{H}_ffn{F}", "M_tokens": M,
+                   "layers": CHAIN_LAYERS, "l2": f"{packed / 1e6:.0f} MB of packed weights per step (> 2x L2)",
+                   "timing": "CUDA graph of the K steps, CUDA events on the launching stream",
+                   "parallelism": f"dp{world} (independent batches per rank)"},
+        "roofline": roof,
+        "kernels_us": {"linear_all_per_step": lin_s * 1e6, "step": step_s * 1e6},
+        "e2e": {"value": tokens * steps / (t_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": M * H * 4, "d2h_bytes_per_step": M * H * 4},
+        "gpu_launches": ch.launches * steps,
+        "clocks": clk,
+    }
+
+
+def chain_cpu_baseline(M, budget_s=10.0):
+    """Oracle tokens/s through the chain: two layers, scaled to 24."""
+    from oracle import bitnet_oracle as O
+    layers = []
+    for l in range(2):
+        lw = {}
+        for name, w in wl.chain_weights(l).items():
+            _, s_w, q = O.quantize_weights(w)
+            lw[name] = (q, s_w)
+        layers.append(lw)
+    x = wl.chain_input(min(M, 4))
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        y = x
+        for lw in layers:
+            y = O.chain_layer(y, lw)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = (time.perf_counter() - t0) * CHAIN_LAYERS / 2
+    return {"value": n * len(x) / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} passes of {len(x)} tokens through 2 oracle layers, time scaled to {CHAIN_LAYERS} layers"}
 
 
 # ----------------------------------------------------------------------------
@@ -416,7 +562,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(CHAIN_WORKLOADS), default="decode")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -428,7 +574,15 @@ def main():
         world = max(world, 1)
 
     if args.impl == "reference":
-        line = run_reference(args, rank, world)
+        line = run_reference(args, rank, world) if args.workload in WORKLOADS else None
+        if args.workload in CHAIN_WORKLOADS and rank == 0:
+            cb = chain_cpu_baseline(CHAIN_WORKLOADS[args.workload], budget_s=2.0 * max(1, args.steps))
+            line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
+                    "n_gpus": world, "steps": args.steps, "warmup": 0, "higher_is_better": True,
+                    "scaling": "weak", "vs_baseline": None, "data": "synthetic",
+                    "config": {"workload": args.workload, "parallelism": "rank 0 only (CPU oracle)"},
+                    "cpu_baseline": cb, "e2e": {"value": cb["value"], "unit": "tokens/s",
+                                                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         if line is not None:
             print(json.dumps(line), flush=True)
         return
@@ -444,10 +598,15 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
         pg = True
     try:
-        line = run_ours(args, rank, world, local_rank)
-        if line is not None:
-            if world == 1 and not args.no_cpu_baseline:
+        if args.workload in CHAIN_WORKLOADS:
+            line = run_chain(args, rank, world, local_rank)
+            if line is not None and world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = chain_cpu_baseline(CHAIN_WORKLOADS[args.workload])
+        else:
+            line = run_ours(args, rank, world, local_rank)
+            if line is not None and world == 1 and not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline(WORKLOADS[args.workload]())
+        if line is not None:
             print(json.dumps(line), flush=True)
     finally:
         if pg:

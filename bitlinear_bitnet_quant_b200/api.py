@@ -39,6 +39,8 @@ _SIGNATURES = {
                                                  ctypes.c_int, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "bitnet_linear": (ctypes.c_int, [_c_void_p, ctypes.c_int, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64,
                                      _c_void_p, ctypes.c_int, _c_void_p, _c_void_p]),
+    "bitnet_add": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _i64, _c_void_p]),
+    "bitnet_relu2_glu": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _i64, _c_void_p]),
     "bitnet_set_linear_path": (ctypes.c_int, [ctypes.c_int]),
     "bitnet_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
 }
@@ -179,6 +181,21 @@ def bitnet_linear(Xq: torch.Tensor, act_bits: int, s_x: torch.Tensor, pkW: torch
         _ptr(Xq), int(act_bits), _ptr(s_x), _ptr(pkW), _ptr(s_w), M, N, K, _ptr(Y), _dtype_code(Y),
         _ptr(acc), _stream(stream)))
     return Y, acc
+
+
+def bitnet_add(a: torch.Tensor, b: torch.Tensor, out=None, stream=None):
+    """fp32 residual add: out = a + b."""
+    out = torch.empty_like(a) if out is None else out
+    _check("bitnet_add", lib().bitnet_add(_ptr(a), _ptr(b), _ptr(out), a.numel(), _stream(stream)))
+    return out
+
+
+def bitnet_relu2_glu(gate: torch.Tensor, up: torch.Tensor, out=None, stream=None):
+    """Squared-ReLU gated unit: out = relu(gate)^2 * up (fp32)."""
+    out = torch.empty_like(gate) if out is None else out
+    _check("bitnet_relu2_glu", lib().bitnet_relu2_glu(_ptr(gate), _ptr(up), _ptr(out), gate.numel(),
+                                                      _stream(stream)))
+    return out
 
 
 def bitnet_set_linear_path(path: int) -> None:

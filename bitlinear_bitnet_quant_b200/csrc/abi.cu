@@ -20,6 +20,8 @@ cudaError_t run_hadamard_quant_i4(const void* X, int bf16, int M, int K, int L, 
 cudaError_t run_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                        int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, int path, cudaStream_t st);
 bool tensor_map_encoder_available();
+cudaError_t run_add_f32(const float* a, const float* b, float* out, size_t n, cudaStream_t st);
+cudaError_t run_relu2_glu(const float* gate, const float* up, float* out, size_t n, cudaStream_t st);
 }  // namespace bitnet
 
 namespace {
@@ -147,6 +149,26 @@ int bitnet_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t*
   return cuda_status(bitnet::run_linear(Xq, act_bits, s_x, pkW, s_w, (int)M, (int)N, (int)K, Y,
                                         y_dtype == BITNET_BF16, acc_dbg, linear_path(),
                                         static_cast<cudaStream_t>(stream)));
+}
+
+static int elementwise_check(const float* a, const float* b, const float* out, int64_t n) {
+  if (n < 0 || n % 4 != 0) return BITNET_ERR_SHAPE;
+  if (n == 0) return -1;                                  // nothing to do
+  if (!a || !b || !out) return BITNET_ERR_NULL;
+  if (!aligned16(a) || !aligned16(b) || !aligned16(out)) return BITNET_ERR_ALIGN;
+  return check_device();
+}
+
+int bitnet_add(const float* a, const float* b, float* out, int64_t n, void* stream) {
+  const int c = elementwise_check(a, b, out, n);
+  if (c != BITNET_OK) return c < 0 ? BITNET_OK : c;
+  return cuda_status(bitnet::run_add_f32(a, b, out, (size_t)n, static_cast<cudaStream_t>(stream)));
+}
+
+int bitnet_relu2_glu(const float* gate, const float* up, float* out, int64_t n, void* stream) {
+  const int c = elementwise_check(gate, up, out, n);
+  if (c != BITNET_OK) return c < 0 ? BITNET_OK : c;
+  return cuda_status(bitnet::run_relu2_glu(gate, up, out, (size_t)n, static_cast<cudaStream_t>(stream)));
 }
 
 int bitnet_set_linear_path(int path) {

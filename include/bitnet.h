@@ -164,6 +164,17 @@ BITNET_API int bitnet_linear(const void* Xq, int act_bits, const float* s_x, con
                   void* Y, int y_dtype, int32_t* acc_dbg, void* stream);
 
 /*
+ * Element-wise glue of the stacked BitLinear chain (a transformer layer whose
+ * linear layers are BitLinear; P2 주요 아키텍처 혁신: squared ReLU, no bias).
+ * bitnet_add:        out[i] = a[i] + b[i]                      (fp32 residual)
+ * bitnet_relu2_glu:  out[i] = (r * r) * up[i],  r = max(gate[i], 0)
+ * fp32, round-to-nearest, no fused multiply-add; out may alias an input.
+ * Limits: n >= 0, n % 4 == 0; all pointers 16-byte aligned device pointers.
+ */
+BITNET_API int bitnet_add(const float* a, const float* b, float* out, int64_t n, void* stream);
+BITNET_API int bitnet_relu2_glu(const float* gate, const float* up, float* out, int64_t n, void* stream);
+
+/*
  * Diagnostics: selects the kernel family bitnet_linear uses in this process.
  * 0 = automatic (default: the tcgen05 tensor-core kernel), 1 = CUDA-core dp4a
  * kernel, 2 = tcgen05 kernel.  Both compute the same bit-exact result.  Returns BITNET_ERR_SHAPE

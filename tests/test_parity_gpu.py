@@ -278,3 +278,45 @@ def test_tiny_bitlinear_forward():
     ref = O.fake_quant_matmul_f64(out["codes"], out["s_x"], qw_o, s_wo)
     nz = out["acc"] != 0
     assert np.max(np.abs(host(Y)[nz] - ref[nz]) / np.abs(ref[nz])) <= 1e-5
+
+
+# ------------------------------------------------------------------ chain -----
+
+def _chain_weights(layers):
+    from bitlinear_bitnet_quant_b200 import chain
+    gpu, ora = [], []
+    for l in range(layers):
+        w = wl.chain_weights(l)
+        gpu.append(chain.quantize_layer({k: dev(v) for k, v in w.items()}))
+        oq = {}
+        for k, v in w.items():
+            _, s_w, q = O.quantize_weights(v)
+            oq[k] = (q, s_w)
+        ora.append(oq)
+    return gpu, ora
+
+
+@pytest.mark.parametrize("M,rows", [(32, None), (512, [0, 1, 77, 255, 256, 400, 510, 511])])
+def test_chain_two_layers(M, rows):
+    """Two stacked layers at full width (hidden 2048, FFN 5632); every op is per
+    token, so the oracle follows sampled token rows through both layers."""
+    from bitlinear_bitnet_quant_b200 import chain
+    gpu_w, ora_w = _chain_weights(2)
+    x = wl.chain_input(M)
+    ch = chain.BitLinearChain(gpu_w, M, wl.CHAIN_HIDDEN, wl.CHAIN_FFN, torch.device("cuda"))
+    out = host(ch.forward(dev(x)))
+    sel = np.arange(M) if rows is None else np.array(rows)
+    ref = x[sel]
+    for lw in ora_w:
+        ref = O.chain_layer(ref, lw)
+    assert np.array_equal(out[sel].view(np.uint32), ref.view(np.uint32))
+
+
+def test_elementwise_glue():
+    rng = np.random.default_rng(21)
+    a = rng.standard_normal(4096 * 3).astype(np.float32)
+    b = rng.standard_normal(4096 * 3).astype(np.float32)
+    s = host(api.bitnet_add(dev(a), dev(b)))
+    assert np.array_equal(s, a + b)
+    g = host(api.bitnet_relu2_glu(dev(a), dev(b)))
+    assert np.array_equal(g, O.squared_relu_glu(a, b))
