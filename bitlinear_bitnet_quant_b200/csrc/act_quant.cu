@@ -176,11 +176,15 @@ quant_act_i8_kernel(const TIn* __restrict__ X, int K, const float* __restrict__ 
 // tokens per CTA).  Stages of stride < 128 run in registers; the stages of
 // stride 128 .. b/2 run after one transpose through shared memory, in which
 // a thread holds the elements whose index bits [a, 7) and the block index are
-// fixed (a = 14 - L), i.e. in-thread bits [0, a) and [7, L).
+// fixed (a = 14 - L), i.e. in-thread bits [0, a) and [7, L).  Bit 0 stays in
+// the thread, so codes are packed two per byte there; the packed bytes (not
+// the fp32 values) go back through shared memory for coalesced stores.
 // ---------------------------------------------------------------------------
 constexpr int HT_R = 128;                          // elements per thread
 
-BN_DEV int hpidx(int e) { return e + (e >> 7); }   // one pad word per 128
+// fp32 slot of element e: two pad words per 128 keep 8-byte accesses of both
+// the transpose's writers and readers free of bank conflicts
+BN_DEV int hpidx(int e) { return e + 2 * (e >> 7); }
 
 // In-register radix-2 stages s = S0 .. S1-1 over v[c], where in-thread index
 // bit (s - SHIFT) is the element-index bit s.
@@ -188,7 +192,6 @@ template <int S0, int S1, int SHIFT>
 BN_DEV void fwht_reg(float (&v)[HT_R]) {
 #pragma unroll
   for (int s = S0; s < S1; ++s) {
-    constexpr int dummy = 0; (void)dummy;
     const int h = 1 << (s - SHIFT);
 #pragma unroll
     for (int c = 0; c < HT_R; ++c) {
@@ -212,8 +215,14 @@ BN_DEV int phase2_elem(int tprime, int c) {
   return (blk << L) | within;
 }
 
+BN_DEV uint32_t nib(float t, float s) {
+  int c = __float2int_rn(__fmul_rn(t, s));
+  c = max(-8, min(7, c));
+  return (uint32_t)(c & 0xF);
+}
+
 template <typename TIn, int L>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 3)
 hadamard_quant_i4_kernel(const TIn* __restrict__ X, int M, int K, int GP,
                          const float* __restrict__ gamma, float eps, float cb,
                          uint8_t* __restrict__ Xq4, float* __restrict__ s_x,
@@ -228,9 +237,10 @@ hadamard_quant_i4_kernel(const TIn* __restrict__ X, int M, int K, int GP,
   const int lane = threadIdx.x & 31;
   const int m = blockIdx.x * TPB + g;
   const bool active = (m < M) && (t < G);
-  const int rowpad = K + (K >> 7);
+  const int rowpad = (K + 2 * (K >> 7) + 3) & ~3;   // 16-byte aligned token rows
   float* tok = hsm + (size_t)g * rowpad;
   float* red = hsm + (size_t)TPB * rowpad;         // [TPB][4] partials
+  uint8_t* bytes = reinterpret_cast<uint8_t*>(tok);  // packed codes, K/2 bytes (after the transpose)
 
   float v[HT_R];
   if (active) {
@@ -248,13 +258,14 @@ hadamard_quant_i4_kernel(const TIn* __restrict__ X, int M, int K, int GP,
     for (int c = 0; c < HT_R; ++c) v[c] = 0.f;
   }
 
-  // ---- sum of squares: in-thread subtree of 128, then threads in order ----
+  // ---- sum of squares: in-thread subtree of 128 (first level fused), then threads in order ----
   float part;
   {
-    float sq[HT_R];
+    float sq[HT_R / 2];
 #pragma unroll
-    for (int c = 0; c < HT_R; ++c) sq[c] = __fmul_rn(v[c], v[c]);
-    part = tree_sum<HT_R>(sq);
+    for (int c = 0; c < HT_R / 2; ++c)
+      sq[c] = __fadd_rn(__fmul_rn(v[2 * c], v[2 * c]), __fmul_rn(v[2 * c + 1], v[2 * c + 1]));
+    part = tree_sum<HT_R / 2>(sq);
   }
   const int wl = GP < 32 ? GP : 32;                // lanes of one token inside a warp
 #pragma unroll
@@ -293,23 +304,19 @@ hadamard_quant_i4_kernel(const TIn* __restrict__ X, int M, int K, int GP,
     __syncthreads();                                // red[] reads above are done
     if (active) {
 #pragma unroll
-      for (int c = 0; c < HT_R; ++c) tok[hpidx(t * HT_R + c)] = v[c];
+      for (int c = 0; c < HT_R; c += 2)
+        *reinterpret_cast<float2*>(tok + hpidx(t * HT_R + c)) = make_float2(v[c], v[c + 1]);
     }
     __syncthreads();
     if (active) {
 #pragma unroll
-      for (int c = 0; c < HT_R; ++c) v[c] = tok[hpidx(phase2_elem<L>(t, c))];
+      for (int c = 0; c < HT_R; c += 2) {          // bit 0 of c is bit 0 of the element: pairs are adjacent
+        const float2 p = *reinterpret_cast<const float2*>(tok + hpidx(phase2_elem<L>(t, c)));
+        v[c] = p.x;
+        v[c + 1] = p.y;
+      }
     }
     fwht_reg<7, L, 7 - (14 - L)>(v);
-    if (active) {
-#pragma unroll
-      for (int c = 0; c < HT_R; ++c) tok[hpidx(phase2_elem<L>(t, c))] = v[c];
-    }
-    __syncthreads();
-    if (active) {
-#pragma unroll
-      for (int c = 0; c < HT_R; ++c) v[c] = tok[hpidx(t * HT_R + c)];
-    }
   }
 
   // ---- normalise, absmax over the token ----
@@ -331,30 +338,48 @@ hadamard_quant_i4_kernel(const TIn* __restrict__ X, int M, int K, int GP,
   }
   const float s = __fdiv_rn(7.0f, fmaxf(amax, 1e-5f));
 
-  if (!active) return;
-  if (T_dbg != nullptr) {
-    float* dst = T_dbg + (size_t)m * K + (size_t)t * HT_R;
+  if constexpr (L <= 7) {
+    // the thread's 128 elements are consecutive: 64 bytes straight out
+    if (!active) return;
+    if (T_dbg != nullptr) {
+      float* dst = T_dbg + (size_t)m * K + (size_t)t * HT_R;
 #pragma unroll
-    for (int c = 0; c < HT_R; c += 4)
-      *reinterpret_cast<float4*>(dst + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
-  }
-  // 128 codes -> 64 bytes: code 2j in the low nibble, 2j+1 in the high nibble
-  uint32_t w[16];
-#pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    uint32_t word = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      int c = __float2int_rn(__fmul_rn(v[8 * q + e], s));
-      c = max(-8, min(7, c));
-      word |= (uint32_t)(c & 0xF) << (4 * e);
+      for (int c = 0; c < HT_R; c += 4)
+        *reinterpret_cast<float4*>(dst + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
     }
-    w[q] = word;
-  }
-  uint4* dst = reinterpret_cast<uint4*>(Xq4 + (size_t)m * (K / 2) + (size_t)t * (HT_R / 2));
+    uint32_t w[16];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-  if (t == 0) s_x[m] = s;
+    for (int q = 0; q < 16; ++q) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) word |= nib(v[8 * q + e], s) << (4 * e);
+      w[q] = word;
+    }
+    uint4* dst = reinterpret_cast<uint4*>(Xq4 + (size_t)m * (K / 2) + (size_t)t * (HT_R / 2));
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    if (t == 0) s_x[m] = s;
+  } else {
+    // codes two per byte in the phase-2 mapping, staged as bytes, then coalesced stores
+    __syncthreads();                                // every thread has read its transposed values
+    if (active) {
+      if (T_dbg != nullptr) {
+        float* dst = T_dbg + (size_t)m * K;
+#pragma unroll
+        for (int c = 0; c < HT_R; ++c) dst[phase2_elem<L>(t, c)] = v[c];
+      }
+#pragma unroll
+      for (int c = 0; c < HT_R; c += 2)
+        bytes[phase2_elem<L>(t, c) >> 1] = (uint8_t)(nib(v[c], s) | (nib(v[c + 1], s) << 4));
+    }
+    __syncthreads();
+    if (m < M) {
+      const uint4* src = reinterpret_cast<const uint4*>(bytes);
+      uint4* dst = reinterpret_cast<uint4*>(Xq4 + (size_t)m * (K / 2));
+      for (int q = t; q < K / 32; q += GP) dst[q] = src[q];
+      if (t == 0) s_x[m] = s;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -403,7 +428,7 @@ static cudaError_t launch_h4(const void* X, int M, int K, const float* gamma, fl
   while (GP < G) GP <<= 1;
   const int TPB = GP >= 128 ? 1 : 128 / GP;
   const int threads = TPB * GP;
-  const size_t smem = (size_t)TPB * (K + (K >> 7)) * sizeof(float) + (size_t)TPB * 4 * sizeof(float);
+  const size_t smem = (size_t)TPB * ((K + 2 * (K >> 7) + 3) & ~3) * sizeof(float) + (size_t)TPB * 4 * sizeof(float);
   auto kern = hadamard_quant_i4_kernel<TIn, L>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;

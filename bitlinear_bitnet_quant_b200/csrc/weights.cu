@@ -22,16 +22,26 @@ namespace bitnet {
 
 constexpr int WQ_DIGITS = 10;           // 320 bits of 2^-149 units (max sum < 2^(277+31))
 
+// The counters live in registers: a switch on the digit index (weights of
+// one tensor share one or two exponent groups, so the branch hardly diverges).
+struct Digits {
+  uint64_t c[WQ_DIGITS];
+};
+
 // Adds |w| (given as its fp32 bit pattern) to the digit counters.
-BN_DEV void digits_add(uint64_t* acc, uint32_t bits) {
+BN_DEV void digits_add(Digits& acc, uint32_t bits) {
   bits &= 0x7FFFFFFFu;
   const uint32_t ex = bits >> 23;
   const uint32_t man = (bits & 0x7FFFFFu) | (ex ? 0x800000u : 0u);
   const uint32_t sh = ex ? ex - 1 : 0;             // value = man << sh (units of 2^-149)
   const uint64_t v = (uint64_t)man << (sh & 31);
-  const int d = (int)(sh >> 5);
-  acc[d] += (uint32_t)v;
-  acc[d + 1] += v >> 32;
+  const uint64_t lo = (uint32_t)v, hi = v >> 32;
+  switch (sh >> 5) {                               // 0 .. 7 (sh <= 254)
+#define BN_DIGIT_CASE(D) case D: acc.c[D] += lo; acc.c[D + 1] += hi; break;
+    BN_DIGIT_CASE(0) BN_DIGIT_CASE(1) BN_DIGIT_CASE(2) BN_DIGIT_CASE(3)
+    BN_DIGIT_CASE(4) BN_DIGIT_CASE(5) BN_DIGIT_CASE(6) BN_DIGIT_CASE(7)
+#undef BN_DIGIT_CASE
+  }
 }
 
 template <typename TIn>
@@ -40,9 +50,9 @@ absmean_digits_kernel(const TIn* __restrict__ W, size_t n16, uint64_t* __restric
   __shared__ unsigned long long sacc[WQ_DIGITS];
   if (threadIdx.x < WQ_DIGITS) sacc[threadIdx.x] = 0ull;
   __syncthreads();
-  uint64_t acc[WQ_DIGITS];
+  Digits acc;
 #pragma unroll
-  for (int i = 0; i < WQ_DIGITS; ++i) acc[i] = 0;
+  for (int i = 0; i < WQ_DIGITS; ++i) acc.c[i] = 0;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += stride) {
     uint4 u = ldg_nc_v4(reinterpret_cast<const uint8_t*>(W) + 16 * i);
@@ -56,8 +66,13 @@ absmean_digits_kernel(const TIn* __restrict__ W, size_t n16, uint64_t* __restric
     }
   }
 #pragma unroll
-  for (int i = 0; i < WQ_DIGITS; ++i)
-    if (acc[i]) atomicAdd(&sacc[i], (unsigned long long)acc[i]);
+  for (int i = 0; i < WQ_DIGITS; ++i) {
+    // warp-level sum first (integers: any order is exact), then one shared atomic per warp
+    unsigned long long x = acc.c[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if ((threadIdx.x & 31) == 0 && x) atomicAdd(&sacc[i], x);
+  }
   __syncthreads();
   if (threadIdx.x < WQ_DIGITS && sacc[threadIdx.x])
     atomicAdd(reinterpret_cast<unsigned long long*>(ws) + threadIdx.x, sacc[threadIdx.x]);
