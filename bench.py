@@ -51,6 +51,8 @@ METRIC = "BitLinear tokens/sec and GB/s|TOPS vs HBM/int8 roofline, 1xB200"
 
 WORKLOADS = {
     "decode": lambda: wl.decode(16, with_weights=False),
+    "decode_m4": lambda: wl.decode(4, with_weights=False),
+    "decode_m1": lambda: wl.decode(1, with_weights=False),
     "prefill": lambda: wl.prefill(with_weights=False),
     "hbitlinear": lambda: wl.hbitlinear(with_weights=False),
     "tiny": lambda: wl.tiny(),
@@ -314,10 +316,10 @@ def run_ours(args, rank, world, local_rank):
     q_s = t_q / steps / 1e3
     x_in_bytes = M * K * (2 if c["x_dtype"] == "bf16" else 4)
     xq_bytes = M * K if bits == 8 else M * K // 2
-    if args.workload in ("decode", "tiny"):
+    if args.workload.startswith("decode") or args.workload == "tiny":
         alg_bytes = packed_bytes + xq_bytes + 4 * M + 4 + M * N * out_bytes
         roof = {"bound": "hbm", "achieved": alg_bytes / lin_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "kernel": "bitnet_linear (tcgen05)" if M > 2 else "bitnet_linear (dp4a)",
+                "kernel": "bitnet_linear (warp-MMA decode)" if M <= 16 and K % 512 == 0 else "bitnet_linear (tcgen05)",
                 "algorithmic_bytes_per_launch": alg_bytes}
         tag = f"linear_{args.workload}"
     else:

@@ -20,6 +20,7 @@ cudaError_t run_hadamard_quant_i4(const void* X, int bf16, int M, int K, int L, 
 cudaError_t run_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                        int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, int path, cudaStream_t st);
 bool tensor_map_encoder_available();
+bool decode_path_applies(int M, int K);
 cudaError_t run_add_f32(const float* a, const float* b, float* out, size_t n, cudaStream_t st);
 cudaError_t run_relu2_glu(const float* gate, const float* up, float* out, size_t n, cudaStream_t st);
 }  // namespace bitnet
@@ -54,7 +55,7 @@ int cuda_status(cudaError_t e) {
   return BITNET_ERR_CUDA;
 }
 
-// 0 = automatic, 1 = SIMT, 2 = tcgen05 (set by bitnet_set_linear_path).
+// 0 = automatic, 1 = SIMT, 2 = tcgen05, 3 = warp-MMA decode (set by bitnet_set_linear_path).
 std::atomic<int> g_linear_path{0};
 int linear_path() { return g_linear_path.load(std::memory_order_relaxed); }
 
@@ -146,6 +147,7 @@ int bitnet_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t*
   int d = check_device();
   if (d != BITNET_OK) return d;
   if (!bitnet::tensor_map_encoder_available()) return BITNET_ERR_UNSUPPORTED;
+  if (linear_path() == 3 && !bitnet::decode_path_applies((int)M, (int)K)) return BITNET_ERR_SHAPE;
   return cuda_status(bitnet::run_linear(Xq, act_bits, s_x, pkW, s_w, (int)M, (int)N, (int)K, Y,
                                         y_dtype == BITNET_BF16, acc_dbg, linear_path(),
                                         static_cast<cudaStream_t>(stream)));
@@ -172,7 +174,7 @@ int bitnet_relu2_glu(const float* gate, const float* up, float* out, int64_t n, 
 }
 
 int bitnet_set_linear_path(int path) {
-  if (path < 0 || path > 2) return BITNET_ERR_SHAPE;
+  if (path < 0 || path > 3) return BITNET_ERR_SHAPE;
   g_linear_path.store(path, std::memory_order_relaxed);
   return BITNET_OK;
 }

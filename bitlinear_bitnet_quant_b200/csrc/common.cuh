@@ -185,6 +185,13 @@ BN_DEV void bulk_copy_to_cluster(uint32_t dst_cluster_addr, const void* src, uin
 }
 // Waits until the source reads of this thread's committed bulk copies are done.
 BN_DEV void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// 16-byte asynchronous global -> shared copy; src_bytes = 0 writes zeros.
+BN_DEV void cp_async_16(uint32_t dst_smem, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst_smem), "l"(src), "r"(src_bytes) : "memory");
+}
+BN_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+BN_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 BN_DEV void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }

@@ -550,9 +550,17 @@ static cudaError_t launch_simt(const void* Xq, const float* s_x, const uint8_t* 
 
 bool tensor_map_encoder_available() { return get_encode() != nullptr; }
 
-// path: 0 = automatic, 1 = SIMT, 2 = tcgen05
+bool decode_path_applies(int M, int K);
+cudaError_t run_linear_decode(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
+                              int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, cudaStream_t st);
+
+// path: 0 = automatic, 1 = SIMT, 2 = tcgen05, 3 = warp-MMA decode kernel
 cudaError_t run_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                        int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, int path, cudaStream_t st) {
+  // up to 16 tokens: one pass over the weights with warp-level MMA
+  if ((path == 0 || path == 3) && decode_path_applies(M, K))
+    return run_linear_decode(Xq, act_bits, s_x, pkW, s_w, M, N, K, Y, y_bf16, acc_dbg, st);
+  if (path == 3) return cudaErrorInvalidValue;
   const bool tc = path != 1;          // the dp4a kernel is a diagnostics path (slower at every M)
 #define BN_LIN(BITS, T)                                                                  \
   return tc ? dispatch_tc<BITS, T>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st)           \

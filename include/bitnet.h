@@ -158,6 +158,9 @@ BITNET_API int bitnet_hadamard_quant_act(const void* X, int x_dtype, int64_t M, 
  * Y      : out, [M][N] fp32 or bf16 (y_dtype).
  * acc_dbg: out, [M][N] int32 accumulators, or NULL (diagnostics only).
  * Limits : M >= 0, N >= 1, 128 <= K <= 65536, K % 128 == 0.
+ * Kernels: up to 32 tokens with K % 512 == 0 and K <= 16384, a one-pass
+ *          kernel on warp-level int8 MMA (each CTA streams a slice of whole
+ *          weight rows); otherwise the tcgen05 tensor-core kernel.
  */
 BITNET_API int bitnet_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW,
                   const float* s_w, int64_t M, int64_t N, int64_t K,
@@ -176,9 +179,11 @@ BITNET_API int bitnet_relu2_glu(const float* gate, const float* up, float* out, 
 
 /*
  * Diagnostics: selects the kernel family bitnet_linear uses in this process.
- * 0 = automatic (default: the tcgen05 tensor-core kernel), 1 = CUDA-core dp4a
- * kernel, 2 = tcgen05 kernel.  Both compute the same bit-exact result.  Returns BITNET_ERR_SHAPE
- * for any other value.
+ * 0 = automatic (default: warp-MMA decode kernel where it applies, else the
+ * tcgen05 tensor-core kernel), 1 = CUDA-core dp4a kernel, 2 = tcgen05 kernel,
+ * 3 = warp-MMA decode kernel (bitnet_linear then returns BITNET_ERR_SHAPE for
+ * shapes it does not cover: M > 32, K % 512 != 0 or K > 16384).  All compute
+ * the same bit-exact result.  Returns BITNET_ERR_SHAPE for any other value.
  */
 BITNET_API int bitnet_set_linear_path(int path);
 

@@ -225,6 +225,30 @@ def test_linear_random_codes(M, N, K, act_bits, out, path):
     _check_linear(qx, qw, s_x, s_w, act_bits, out, path)
 
 
+@pytest.mark.parametrize("M,N,K,act_bits,out", [
+    (1, 16, 512, 8, "f32"), (1, 1, 512, 8, "f32"), (3, 200, 1024, 8, "bf16"), (8, 1000, 1536, 8, "f32"),
+    (9, 4096, 512, 8, "f32"), (16, 6912, 2560, 8, "bf16"), (16, 300, 8192, 8, "f32"), (5, 64, 16384, 8, "f32"),
+    (1, 20000, 1024, 8, "f32"), (16, 2368, 4608, 8, "f32"),
+    (2, 512, 4608, 4, "f32"), (16, 2048, 5632, 4, "f32"), (7, 333, 2560, 4, "bf16"), (1, 48, 512, 4, "f32"),
+    (17, 1000, 2048, 8, "f32"), (32, 5632, 2048, 8, "bf16"), (32, 2048, 5632, 4, "f32"), (24, 333, 512, 4, "f32"),
+    (31, 100, 10240, 8, "f32")])
+def test_linear_decode_kernel(M, N, K, act_bits, out):
+    """The one-pass warp-MMA kernel (up to 32 tokens): ragged N, one, two and
+    four token groups, K of 1 to 32 segments (one and several activation
+    batches)."""
+    qx, qw, s_x, s_w = _random_codes(M, N, K, act_bits, M * 13 + N + K)
+    _check_linear(qx, qw, s_x, s_w, act_bits, out, path=3)
+
+
+def test_linear_decode_kernel_rejects_other_shapes():
+    qx, qw, s_x, s_w = _random_codes(33, 64, 512, 8, 1)
+    with pytest.raises(api.BitnetError):
+        _run_linear(qx, qw, s_x, s_w, 8, "f32", path=3)
+    qx, qw, s_x, s_w = _random_codes(4, 64, 384, 8, 2)
+    with pytest.raises(api.BitnetError):
+        _run_linear(qx, qw, s_x, s_w, 8, "f32", path=3)
+
+
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_linear_decode_full(M):
     c = wl.decode(M)
