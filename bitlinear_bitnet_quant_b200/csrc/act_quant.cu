@@ -29,7 +29,7 @@ template <typename TIn> struct InVec;
 template <> struct InVec<float> {
   static constexpr int E = 4;
   static BN_DEV void load(const float* p, float (&v)[4]) {
-    uint4 u = ldg_nc_v4(p);
+    uint4 u = ldg_v4(p);
     v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
     v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
   }
@@ -37,7 +37,7 @@ template <> struct InVec<float> {
 template <> struct InVec<uint16_t> {
   static constexpr int E = 8;
   static BN_DEV void load(const uint16_t* p, float (&v)[8]) {
-    uint4 u = ldg_nc_v4(p);
+    uint4 u = ldg_v4(p);
     v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
     v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
   }

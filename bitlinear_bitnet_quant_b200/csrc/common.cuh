@@ -36,10 +36,37 @@ enum DeviceError : int {
 BN_DEV float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
 BN_DEV float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
+// Read-only data of the whole call (weights, gamma): non-coherent path.
 BN_DEV uint4 ldg_nc_v4(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+BN_DEV float ldg_nc_f32(const float* p) {
+  float r;
+  asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(r) : "l"(p));
+  return r;
+}
+
+// Data written by the previous kernel in the stream (activations, s_x),
+// read after the programmatic-launch wait: plain coherent loads.  The asm is
+// volatile so that the loads are issued where they are written (all at once,
+// ahead of their first use) instead of being moved down to it.
+BN_DEV uint4 ldg_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+BN_DEV uint2 ldg_v2(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+BN_DEV float ldg_f32(const float* p) {
+  float r;
+  asm volatile("ld.global.f32 %0, [%1];" : "=f"(r) : "l"(p));
   return r;
 }
 

@@ -14,7 +14,9 @@ add_f32_kernel(const float4* __restrict__ a, const float4* __restrict__ b, float
   pdl_wait();                                   // inputs come from the previous kernels
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
-    const float4 x = a[i], y = b[i];
+    const uint4 ua = ldg_v4(a + i), ub = ldg_v4(b + i);
+    const float4 x = make_float4(__uint_as_float(ua.x), __uint_as_float(ua.y), __uint_as_float(ua.z), __uint_as_float(ua.w));
+    const float4 y = make_float4(__uint_as_float(ub.x), __uint_as_float(ub.y), __uint_as_float(ub.z), __uint_as_float(ub.w));
     out[i] = make_float4(__fadd_rn(x.x, y.x), __fadd_rn(x.y, y.y), __fadd_rn(x.z, y.z), __fadd_rn(x.w, y.w));
   }
 }
@@ -31,7 +33,9 @@ relu2_glu_kernel(const float4* __restrict__ gate, const float4* __restrict__ up,
   pdl_wait();
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
-    const float4 g = gate[i], u = up[i];
+    const uint4 ug = ldg_v4(gate + i), uu = ldg_v4(up + i);
+    const float4 g = make_float4(__uint_as_float(ug.x), __uint_as_float(ug.y), __uint_as_float(ug.z), __uint_as_float(ug.w));
+    const float4 u = make_float4(__uint_as_float(uu.x), __uint_as_float(uu.y), __uint_as_float(uu.z), __uint_as_float(uu.w));
     out[i] = make_float4(relu2_times(g.x, u.x), relu2_times(g.y, u.y), relu2_times(g.z, u.z), relu2_times(g.w, u.w));
   }
 }

@@ -75,10 +75,10 @@ linear_simt_kernel(const uint8_t* __restrict__ Xq, const float* __restrict__ s_x
       if (t < mcount) {
         uint32_t x4[4];
         if constexpr (ACT_BITS == 8) {
-          const uint4 u = ldg_nc_v4(Xq + (size_t)(m0 + t) * K + 16 * g);
+          const uint4 u = ldg_v4(Xq + (size_t)(m0 + t) * K + 16 * g);
           x4[0] = u.x; x4[1] = u.y; x4[2] = u.z; x4[3] = u.w;
         } else {
-          const uint2 u = __ldg(reinterpret_cast<const uint2*>(Xq + (size_t)(m0 + t) * (K / 2) + 8 * g));
+          const uint2 u = ldg_v2(Xq + (size_t)(m0 + t) * (K / 2) + 8 * g);
           widen8(u.x, x4[0], x4[1]);
           widen8(u.y, x4[2], x4[3]);
         }
@@ -97,7 +97,7 @@ linear_simt_kernel(const uint8_t* __restrict__ Xq, const float* __restrict__ s_x
       const int m = m0 + t;
       const int v = a >> (ACT_BITS == 8 ? 6 : 10);
       if (acc_dbg) acc_dbg[(size_t)m * N + n] = v;
-      store_out(Y + (size_t)m * N + n, __fmul_rn((float)v, dequant_scale(__ldg(s_x + m), sw)));
+      store_out(Y + (size_t)m * N + n, __fmul_rn((float)v, dequant_scale(ldg_f32(s_x + m), sw)));
     }
   }
 }
@@ -256,10 +256,10 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       for (int i = 0; i < pre; ++i) load_x(i);    // first: the activations are on the critical path
     if (kr == 0) {
       if (lane == 0 && use_tma_store) tma_prefetch_desc(&tmY);
-      const float sw = __ldg(s_w_ptr);
+      const float sw = ldg_nc_f32(s_w_ptr);
       for (int j = lane; j < BN; j += 32) {
         const int m = m0 + j;
-        sdq[j] = m < M ? dequant_scale(__ldg(s_x + m), sw) : 0.f;
+        sdq[j] = m < M ? dequant_scale(ldg_f32(s_x + m), sw) : 0.f;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_sdq);

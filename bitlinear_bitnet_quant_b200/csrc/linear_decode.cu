@@ -114,10 +114,10 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
     cp_async_commit();
   }
   // s_w belongs to the weights: read it before the wait as well
-  const float sw = threadIdx.x < TOK ? __ldg(s_w_ptr) : 0.0f;
+  const float sw = threadIdx.x < TOK ? ldg_nc_f32(s_w_ptr) : 0.0f;
   pdl_wait();                                  // activations and s_x come from the previous kernel
   // issued now, consumed only in the epilogue
-  const float sx = threadIdx.x < M && threadIdx.x < TOK ? s_x[threadIdx.x] : 1.0f;
+  const float sx = threadIdx.x < M && threadIdx.x < TOK ? ldg_f32(s_x + threadIdx.x) : 1.0f;
 
   int d[RG_MAX][TG][4];
 #pragma unroll
@@ -140,12 +140,19 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
         xv[u][tg] = make_uint4(0u, 0u, 0u, 0u);
         if (u0 + u < nseg && m < M) {
           if constexpr (ACT_BITS == 8) {
-            xv[u][tg] = *reinterpret_cast<const uint4*>(Xq + (size_t)m * xrow + k0);
+            xv[u][tg] = ldg_v4(Xq + (size_t)m * xrow + k0);
           } else {
-            xv[u][tg] = widen16(*reinterpret_cast<const uint2*>(Xq + (size_t)m * xrow + k0 / 2));
+            const uint2 p = ldg_v2(Xq + (size_t)m * xrow + k0 / 2);
+            xv[u][tg] = make_uint4(p.x, p.y, 0u, 0u);     // widened below, after every load is issued
           }
         }
       }
+    }
+    if constexpr (ACT_BITS == 4) {
+#pragma unroll
+      for (int u = 0; u < PB; ++u)
+#pragma unroll
+        for (int tg = 0; tg < TG; ++tg) xv[u][tg] = widen16(make_uint2(xv[u][tg].x, xv[u][tg].y));
     }
     if (u0 == 0) {
       cp_async_wait_all();                     // this thread's weight copies
