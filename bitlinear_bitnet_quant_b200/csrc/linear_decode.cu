@@ -75,15 +75,24 @@ BN_DEV uint4 widen16(uint2 p) {
   return r;
 }
 
-// TG = token groups of 8 (1: M <= 8, 2: M <= 16, 4: M <= 32).
-template <int ACT_BITS, int TG, typename TOut>
+// TG = token groups of 8 (1: M <= 8, 2: M <= 16, 4: M <= 32); RG = groups of
+// 16 weight rows per CTA (rows = 16 * RG).  Both are compile-time so that one
+// K segment is a single straight-line block: the next segment's weight words
+// are loaded while this one's MMAs issue, and consecutive MMAs never depend on
+// each other (with one token group, the two MMAs of a 64-wide slice go to two
+// accumulator sets, summed at the end).
+template <int ACT_BITS, int TG, int RG, typename TOut>
 __global__ void __launch_bounds__(DEC_THREADS, 2)
 linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict__ Xq,
                      const float* __restrict__ s_x, const float* __restrict__ s_w_ptr, int M, int N, int K,
-                     int rows, TOut* __restrict__ Y, int32_t* __restrict__ acc_dbg) {
+                     TOut* __restrict__ Y, int32_t* __restrict__ acc_dbg) {
   using C = DecCfg<TG>;
-  constexpr int RG_MAX = C::RG_MAX, TOK = C::TOK, PB = C::PASS_BATCH;
+  constexpr int TOK = C::TOK, PB = C::PASS_BATCH;
+  constexpr int ROWS = 16 * RG;
+  constexpr int NACC = TG == 1 ? 2 : 1;                      // accumulator sets
   constexpr int SHIFT = ACT_BITS == 8 ? 6 : 10;
+  constexpr uint32_t SEG_BYTES = ROWS * 128u;
+  static_assert(RG >= 1 && RG <= C::RG_MAX, "row groups");
   extern __shared__ uint8_t dec_smem_raw[];
   __shared__ float sdq[TOK];
 
@@ -91,25 +100,23 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int nseg = K / 512;
-  const int n0 = blockIdx.x * rows;
-  const int rg_count = rows / 16;
-  const uint32_t seg_bytes = (uint32_t)rows * 128u;
+  const int n0 = blockIdx.x * ROWS;
 
   // This kernel holds no tensor memory, so the next kernel in the stream may
   // be scheduled at once (it only waits for this grid to finish).
   pdl_launch_dependents();
   {
     // The weights do not depend on the previous kernel: stream them now.
-    // Chunk c (16 bytes): segment (c / 8) / rows, row (c / 8) % rows, chunk c % 8.
+    // Chunk c (16 bytes): segment (c / 8) / ROWS, row (c / 8) % ROWS, chunk c % 8.
     const size_t wrow = (size_t)K / 4;
-    const int nchunks = nseg * rows * 8;
+    const int nchunks = nseg * ROWS * 8;
     const uint32_t sbase = smem_u32(wsm);
     for (int c = threadIdx.x; c < nchunks; c += DEC_THREADS) {
       const int q = c & 7, line = c >> 3;
-      const int sg = line / rows, r = line - sg * rows;
+      const int sg = line / ROWS, r = line - sg * ROWS;
       const bool in = n0 + r < N;                         // rows past N read as zeros
       const uint8_t* src = pkW + (in ? (size_t)(n0 + r) * wrow + 128 * (size_t)sg + 16 * q : 0);
-      cp_async_16(sbase + sg * seg_bytes + (uint32_t)r * 128u + 16u * (uint32_t)(q ^ (r & 7)), src, in ? 16u : 0u);
+      cp_async_16(sbase + sg * SEG_BYTES + (uint32_t)r * 128u + 16u * (uint32_t)(q ^ (r & 7)), src, in ? 16u : 0u);
     }
     cp_async_commit();
   }
@@ -119,15 +126,30 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
   // issued now, consumed only in the epilogue
   const float sx = threadIdx.x < M && threadIdx.x < TOK ? ldg_f32(s_x + threadIdx.x) : 1.0f;
 
-  int d[RG_MAX][TG][4];
+  int d[NACC][RG][TG][4];
 #pragma unroll
-  for (int rg = 0; rg < RG_MAX; ++rg)
+  for (int h = 0; h < NACC; ++h)
 #pragma unroll
-    for (int tg = 0; tg < TG; ++tg)
+    for (int rg = 0; rg < RG; ++rg)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) d[rg][tg][j] = 0;
+      for (int tg = 0; tg < TG; ++tg)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) d[h][rg][tg][j] = 0;
+
+  // this thread's packed words of one segment: rows 16 rg + g and + 8, word t
+  // of 16-byte chunk `warp` (stored at chunk warp ^ (row & 7); (row & 7) = g)
+  const uint32_t woff = (uint32_t)g * 128u + 16u * (uint32_t)(warp ^ g) + 4u * (uint32_t)t;
+  auto load_w = [&](int sg, uint32_t (&w)[RG][2]) {
+    const uint8_t* base = wsm + (size_t)sg * SEG_BYTES + woff;
+#pragma unroll
+    for (int rg = 0; rg < RG; ++rg) {
+      w[rg][0] = *reinterpret_cast<const uint32_t*>(base + rg * 2048);
+      w[rg][1] = *reinterpret_cast<const uint32_t*>(base + rg * 2048 + 1024);
+    }
+  };
 
   const size_t xrow = ACT_BITS == 8 ? (size_t)K : (size_t)K / 2;
+  uint32_t wcur[RG][2];
   for (int u0 = 0; u0 < nseg; u0 += PB) {
     // activation bytes of this warp's K slices: 16 consecutive K per token and segment
     uint4 xv[PB][TG];
@@ -157,30 +179,37 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
     if (u0 == 0) {
       cp_async_wait_all();                     // this thread's weight copies
       __syncthreads();                         // and everyone else's
+      load_w(0, wcur);
     }
 #pragma unroll
     for (int u = 0; u < PB; ++u) {
       const int s = u0 + u;
       if (s < nseg) {
-        const uint8_t* seg = wsm + (size_t)s * seg_bytes;
+        uint32_t wnxt[RG][2];
+        load_w(s + 1 < nseg ? s + 1 : s, wnxt);            // next segment's words, ahead of use
+        // quarters 0,1 (first MMA) and 2,3 (second MMA) of each packed word,
+        // moved into the top two bits of every byte: int8 64 * w
+        uint32_t a[RG][2][4];
 #pragma unroll
-        for (int rg = 0; rg < RG_MAX; ++rg) {
-          if (rg < rg_count) {
-            const int r = 16 * rg + g;                          // rows r and r + 8 share (r & 7)
-            const uint32_t off = (uint32_t)r * 128u + 16u * (uint32_t)(warp ^ (r & 7)) + 4u * (uint32_t)t;
-            const uint32_t wl = *reinterpret_cast<const uint32_t*>(seg + off);
-            const uint32_t wh = *reinterpret_cast<const uint32_t*>(seg + off + 8 * 128);
-            const uint32_t a0 = (wl << 6) & 0xC0C0C0C0u, a1 = (wh << 6) & 0xC0C0C0C0u;
-            const uint32_t a2 = (wl << 4) & 0xC0C0C0C0u, a3 = (wh << 4) & 0xC0C0C0C0u;
-            const uint32_t c0 = (wl << 2) & 0xC0C0C0C0u, c1 = (wh << 2) & 0xC0C0C0C0u;
-            const uint32_t c2 = wl & 0xC0C0C0C0u, c3 = wh & 0xC0C0C0C0u;
-#pragma unroll
-            for (int tg = 0; tg < TG; ++tg) {
-              mma_s8_16832(d[rg][tg], a0, a1, a2, a3, xv[u][tg].x, xv[u][tg].y);
-              mma_s8_16832(d[rg][tg], c0, c1, c2, c3, xv[u][tg].z, xv[u][tg].w);
-            }
-          }
+        for (int rg = 0; rg < RG; ++rg) {
+          const uint32_t wl = wcur[rg][0], wh = wcur[rg][1];
+          a[rg][0][0] = (wl << 6) & 0xC0C0C0C0u;  a[rg][0][1] = (wh << 6) & 0xC0C0C0C0u;
+          a[rg][0][2] = (wl << 4) & 0xC0C0C0C0u;  a[rg][0][3] = (wh << 4) & 0xC0C0C0C0u;
+          a[rg][1][0] = (wl << 2) & 0xC0C0C0C0u;  a[rg][1][1] = (wh << 2) & 0xC0C0C0C0u;
+          a[rg][1][2] = wl & 0xC0C0C0C0u;         a[rg][1][3] = wh & 0xC0C0C0C0u;
         }
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int h = NACC == 2 ? q : 0;
+#pragma unroll
+          for (int rg = 0; rg < RG; ++rg)
+#pragma unroll
+            for (int tg = 0; tg < TG; ++tg)
+              mma_s8_16832(d[h][rg][tg], a[rg][q][0], a[rg][q][1], a[rg][q][2], a[rg][q][3],
+                           q == 0 ? xv[u][tg].x : xv[u][tg].z, q == 0 ? xv[u][tg].y : xv[u][tg].w);
+        }
+#pragma unroll
+        for (int rg = 0; rg < RG; ++rg) { wcur[rg][0] = wnxt[rg][0]; wcur[rg][1] = wnxt[rg][1]; }
       }
     }
   }
@@ -188,32 +217,33 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
   if (threadIdx.x < M && threadIdx.x < TOK) sdq[threadIdx.x] = __fmul_rn(__fdiv_rn(1.0f, sx), __fdiv_rn(1.0f, sw));
   __syncthreads();                             // all warps are done with the weight slice
 
-  // partial tiles [warp][token][row], row pitch rows + 4 (conflict-free stores)
-  const int rp = rows + 4;
+  // partial tiles [warp][token][row], row pitch ROWS + 4 (conflict-free stores)
+  constexpr int RP = ROWS + 4;
   int32_t* red = reinterpret_cast<int32_t*>(wsm);
-  int32_t* mine = red + (size_t)warp * TOK * rp;
+  int32_t* mine = red + (size_t)warp * TOK * RP;
 #pragma unroll
-  for (int rg = 0; rg < RG_MAX; ++rg) {
-    if (rg < rg_count) {
+  for (int rg = 0; rg < RG; ++rg) {
 #pragma unroll
-      for (int tg = 0; tg < TG; ++tg) {
-        const int tok = 8 * tg + 2 * t, r = 16 * rg + g;
-        mine[tok * rp + r] = d[rg][tg][0];
-        mine[(tok + 1) * rp + r] = d[rg][tg][1];
-        mine[tok * rp + r + 8] = d[rg][tg][2];
-        mine[(tok + 1) * rp + r + 8] = d[rg][tg][3];
-      }
+    for (int tg = 0; tg < TG; ++tg) {
+      int v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = NACC == 2 ? d[0][rg][tg][j] + d[NACC - 1][rg][tg][j] : d[0][rg][tg][j];
+      const int tok = 8 * tg + 2 * t, r = 16 * rg + g;
+      mine[tok * RP + r] = v[0];
+      mine[(tok + 1) * RP + r] = v[1];
+      mine[tok * RP + r + 8] = v[2];
+      mine[(tok + 1) * RP + r + 8] = v[3];
     }
   }
   __syncthreads();
   const int mcount = M < TOK ? M : TOK;
-  for (int idx = threadIdx.x; idx < mcount * rows; idx += DEC_THREADS) {
-    const int m = idx / rows, nn = idx - m * rows;
+  for (int idx = threadIdx.x; idx < mcount * ROWS; idx += DEC_THREADS) {
+    const int m = idx / ROWS, nn = idx - m * ROWS;
     const int n = n0 + nn;
     if (n < N) {
       int acc = 0;
 #pragma unroll
-      for (int w = 0; w < DEC_WARPS; ++w) acc += red[((size_t)w * TOK + m) * rp + nn];
+      for (int w = 0; w < DEC_WARPS; ++w) acc += red[((size_t)w * TOK + m) * RP + nn];
       acc >>= SHIFT;
       if (acc_dbg) acc_dbg[(size_t)m * N + n] = acc;
       dec_store(Y + (size_t)m * N + n, __fmul_rn((float)acc, sdq[m]));
@@ -237,23 +267,36 @@ static int decode_rows(int N, int K, int sms, int max_rows) {
   return rows;
 }
 
+template <int ACT_BITS, int TG, int RG, typename TOut>
+static cudaError_t launch_decode_rg(const void* Xq, const float* s_x, const uint8_t* pkW, const float* s_w, int M,
+                                    int N, int K, void* Y, int32_t* acc_dbg, cudaStream_t st) {
+  constexpr int ROWS = 16 * RG;
+  const size_t wbytes = (size_t)ROWS * (size_t)K / 4;
+  const size_t rbytes = (size_t)DEC_WARPS * DecCfg<TG>::TOK * (size_t)(ROWS + 4) * sizeof(int32_t);
+  const size_t smem = (wbytes > rbytes ? wbytes : rbytes) + 1024;
+  auto kern = linear_decode_kernel<ACT_BITS, TG, RG, TOut>;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((N + ROWS - 1) / ROWS));
+  return launch_pdl(kern, grid, dim3(DEC_THREADS), smem, st, 1u, pkW, static_cast<const uint8_t*>(Xq), s_x, s_w, M, N,
+                    K, static_cast<TOut*>(Y), acc_dbg);
+}
+
 template <int ACT_BITS, int TG, typename TOut>
 static cudaError_t launch_decode_t(const void* Xq, const float* s_x, const uint8_t* pkW, const float* s_w, int M,
                                    int N, int K, void* Y, int32_t* acc_dbg, cudaStream_t st) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  using C = DecCfg<TG>;
-  const int rows = decode_rows(N, K, sms, C::MAX_ROWS);
-  const size_t wbytes = (size_t)rows * (size_t)K / 4;
-  const size_t rbytes = (size_t)DEC_WARPS * C::TOK * (size_t)(rows + 4) * sizeof(int32_t);
-  const size_t smem = (wbytes > rbytes ? wbytes : rbytes) + 1024;
-  auto kern = linear_decode_kernel<ACT_BITS, TG, TOut>;
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
-  if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)((N + rows - 1) / rows));
-  return launch_pdl(kern, grid, dim3(DEC_THREADS), smem, st, 1u, pkW, static_cast<const uint8_t*>(Xq), s_x, s_w, M, N,
-                    K, rows, static_cast<TOut*>(Y), acc_dbg);
+  const int rg = decode_rows(N, K, sms, DecCfg<TG>::MAX_ROWS) / 16;
+#define BN_RG(R) launch_decode_rg<ACT_BITS, TG, (R <= DecCfg<TG>::RG_MAX ? R : 1), TOut>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st)
+  switch (rg) {
+    case 1: return BN_RG(1);
+    case 2: return BN_RG(2);
+    case 3: return BN_RG(3);
+    default: return BN_RG(4);
+  }
+#undef BN_RG
 }
 
 cudaError_t run_linear_decode(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
