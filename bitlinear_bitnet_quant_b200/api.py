@@ -39,6 +39,9 @@ _SIGNATURES = {
                                                  ctypes.c_int, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "bitnet_linear": (ctypes.c_int, [_c_void_p, ctypes.c_int, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64,
                                      _c_void_p, ctypes.c_int, _c_void_p, _c_void_p]),
+    "bitnet_bitlinear": (ctypes.c_int, [_c_void_p, ctypes.c_int, _i64, _i64, _c_void_p, ctypes.c_float,
+                                        _c_void_p, _c_void_p, _i64, _c_void_p, ctypes.c_int, _c_void_p, _c_void_p,
+                                        _c_void_p]),
     "bitnet_add": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _i64, _c_void_p]),
     "bitnet_relu2_glu": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _i64, _c_void_p]),
     "bitnet_set_linear_path": (ctypes.c_int, [ctypes.c_int]),
@@ -183,6 +186,24 @@ def bitnet_linear(Xq: torch.Tensor, act_bits: int, s_x: torch.Tensor, pkW: torch
     return Y, acc
 
 
+def bitnet_bitlinear(X: torch.Tensor, pkW: torch.Tensor, s_w: torch.Tensor, gamma=None, eps: float = 1e-6,
+                     out_dtype=torch.float32, Y=None, Xq=None, s_x=None, stream=None):
+    """Fused BitLinear forward with int8 activations (RMSNorm + absmax int8 +
+    ternary product + dequantisation).  Returns (Y [M, N], Xq [M, K], s_x [M])."""
+    _require(X, "X")
+    _require(pkW, "pkW")
+    M, K = X.shape
+    N = pkW.shape[0]
+    dev = X.device
+    Y = torch.empty((M, N), dtype=out_dtype, device=dev) if Y is None else Y
+    Xq = torch.empty((M, K), dtype=torch.int8, device=dev) if Xq is None else Xq
+    s_x = torch.empty((M,), dtype=torch.float32, device=dev) if s_x is None else s_x
+    _check("bitnet_bitlinear", lib().bitnet_bitlinear(
+        _ptr(X), _dtype_code(X), M, K, _ptr(gamma), float(eps), _ptr(pkW), _ptr(s_w), N, _ptr(Y), _dtype_code(Y),
+        _ptr(Xq), _ptr(s_x), _stream(stream)))
+    return Y, Xq, s_x
+
+
 def bitnet_add(a: torch.Tensor, b: torch.Tensor, out=None, stream=None):
     """fp32 residual add: out = a + b."""
     out = torch.empty_like(a) if out is None else out
@@ -210,9 +231,11 @@ def bitnet_device_error() -> int:
 
 def bitlinear_forward(X: torch.Tensor, pkW: torch.Tensor, s_w: torch.Tensor, act_bits: int = 8, gamma=None,
                       eps: float = 1e-6, had_block: int = 0, out_dtype=torch.float32, stream=None):
-    """One BitLinear forward: quantise the activations, then the ternary product."""
+    """One BitLinear forward: quantise the activations, then the ternary product
+    (int8: the fused entry point, one kernel for a few tokens)."""
     if act_bits == 8:
-        Xq, s_x = bitnet_quant_act(X, gamma, eps, stream=stream)
+        Y, _, _ = bitnet_bitlinear(X, pkW, s_w, gamma, eps, out_dtype=out_dtype, stream=stream)
+        return Y
     else:
         Xq, s_x, _ = bitnet_hadamard_quant_act(X, gamma, eps, had_block, stream=stream)
     Y, _ = bitnet_linear(Xq, act_bits, s_x, pkW, s_w, out_dtype=out_dtype, stream=stream)

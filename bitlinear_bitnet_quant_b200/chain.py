@@ -5,11 +5,13 @@ linear layers of attention and FFN are BitLinear (int8 activations), and in
 BitNet v2 the O and down projections are H-BitLinear (Hadamard + int4).
 Per layer, with fp32 residuals:
 
-    q, k, v = BitLinear(x)                      (one int8 quantisation of x)
+    q, k, v = BitLinear(x)                      (one int8 quantisation of x,
+                                                 fused into q's call)
     o = H-BitLinear(v)                          (attention over a one-token
                                                  context returns V)
     h = x + o
-    up, gate = BitLinear(h)                     (one int8 quantisation of h)
+    up, gate = BitLinear(h)                     (one int8 quantisation of h,
+                                                 fused into up's call)
     a = relu(gate)^2 * up                       (squared-ReLU gated unit)
     x' = h + H-BitLinear(a)                     (down projection)
 
@@ -53,14 +55,14 @@ class BitLinearChain:
 
     def layer(self, x: torch.Tensor, w: dict, out: torch.Tensor, stream=None) -> torch.Tensor:
         A, s = api, stream
-        A.bitnet_quant_act(x, None, self.eps, Xq=self.xq, s_x=self.sx, stream=s)
-        for name, Y in (("q", self.q), ("k", self.k), ("v", self.v)):
+        # q: the fused entry point quantises x (codes and scales kept for k, v)
+        A.bitnet_bitlinear(x, *w["q"], None, self.eps, Y=self.q, Xq=self.xq, s_x=self.sx, stream=s)
+        for name, Y in (("k", self.k), ("v", self.v)):
             A.bitnet_linear(self.xq, 8, self.sx, *w[name], Y=Y, stream=s)
         A.bitnet_hadamard_quant_act(self.v, None, self.eps, 0, Xq4=self.v4, s_x=self.sv, stream=s)
         A.bitnet_linear(self.v4, 4, self.sv, *w["o"], Y=self.o, stream=s)
         A.bitnet_add(x, self.o, out=self.h, stream=s)
-        A.bitnet_quant_act(self.h, None, self.eps, Xq=self.hq, s_x=self.sh, stream=s)
-        A.bitnet_linear(self.hq, 8, self.sh, *w["up"], Y=self.up, stream=s)
+        A.bitnet_bitlinear(self.h, *w["up"], None, self.eps, Y=self.up, Xq=self.hq, s_x=self.sh, stream=s)
         A.bitnet_linear(self.hq, 8, self.sh, *w["gate"], Y=self.gate, stream=s)
         A.bitnet_relu2_glu(self.gate, self.up, out=self.a, stream=s)
         A.bitnet_hadamard_quant_act(self.a, None, self.eps, 0, Xq4=self.a4, s_x=self.sa, stream=s)
@@ -76,11 +78,13 @@ class BitLinearChain:
             cur = self.layer(cur, w, self.x[i % 2], stream)
         return cur
 
-    # kernels launched per forward: per layer 2 int8 quantisers, 2 Hadamard
-    # quantisers, 7 linear layers, 2 adds and 1 gated unit
+    # kernels launched per forward: per layer 2 fused BitLinear calls (one
+    # kernel each for a few tokens, else a quantiser and a linear layer),
+    # 5 further linear layers, 2 Hadamard quantisers, 2 adds, 1 gated unit
     @property
     def launches(self) -> int:
-        return 14 * len(self.layers)
+        fused = self.M <= 32 and self.hidden % 512 == 0 and self.hidden <= 8192
+        return (12 if fused else 14) * len(self.layers)
 
     def packed_bytes(self) -> int:
         return sum(pk.numel() for w in self.layers for pk, _ in w.values())

@@ -20,6 +20,9 @@ cudaError_t run_hadamard_quant_i4(const void* X, int bf16, int M, int K, int L, 
 cudaError_t run_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                        int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, int path, cudaStream_t st);
 bool tensor_map_encoder_available();
+cudaError_t run_bitlinear(const void* X, int x_bf16, int M, int K, const float* gamma, float eps, const uint8_t* pkW,
+                          const float* s_w, int N, void* Y, int y_bf16, int8_t* Xq, float* s_x, int path,
+                          cudaStream_t st);
 bool decode_path_applies(int M, int K);
 cudaError_t run_add_f32(const float* a, const float* b, float* out, size_t n, cudaStream_t st);
 cudaError_t run_relu2_glu(const float* gate, const float* up, float* out, size_t n, cudaStream_t st);
@@ -159,6 +162,29 @@ static int elementwise_check(const float* a, const float* b, const float* out, i
   if (!a || !b || !out) return BITNET_ERR_NULL;
   if (!aligned16(a) || !aligned16(b) || !aligned16(out)) return BITNET_ERR_ALIGN;
   return check_device();
+}
+
+int bitnet_bitlinear(const void* X, int x_dtype, int64_t M, int64_t K, const float* gamma, float eps,
+                     const uint8_t* pkW, const float* s_w, int64_t N, void* Y, int y_dtype, int8_t* Xq, float* s_x,
+                     void* stream) {
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (M < 0 || M > (int64_t(1) << 30) || N < 1 || N > (int64_t(1) << 30) || K < 128 || K > 16384 ||
+      K % 128 != 0 || M * N >= (int64_t(1) << 40))
+    return BITNET_ERR_SHAPE;
+  if (M == 0) return BITNET_OK;
+  if (!X || !pkW || !s_w || !Y || !Xq || !s_x) return BITNET_ERR_NULL;
+  if (!aligned16(X) || !aligned16(pkW) || !aligned16(Y) || !aligned16(Xq) || (gamma && !aligned16(gamma)) ||
+      (reinterpret_cast<uintptr_t>(s_x) & 3u) || (reinterpret_cast<uintptr_t>(s_w) & 3u))
+    return BITNET_ERR_ALIGN;
+  int d = check_device();
+  if (d != BITNET_OK) return d;
+  if (!bitnet::tensor_map_encoder_available()) return BITNET_ERR_UNSUPPORTED;
+  const int path = linear_path();
+  if (path == 3 && !bitnet::decode_path_applies((int)M, (int)K)) return BITNET_ERR_SHAPE;
+  return cuda_status(bitnet::run_bitlinear(X, x_dtype == BITNET_BF16, (int)M, (int)K, gamma, eps, pkW, s_w, (int)N,
+                                           Y, y_dtype == BITNET_BF16, Xq, s_x, path,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 int bitnet_add(const float* a, const float* b, float* out, int64_t n, void* stream) {

@@ -526,7 +526,7 @@ static cudaError_t launch_tc(const void* Xq, const float* s_x, const uint8_t* pk
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   dim3 grid((N + 127) / 128, (M + BN - 1) / BN, ksplit);
-  return launch_pdl(kern, grid, dim3(TC_THREADS), smem, st, (unsigned)ksplit, tmW, tmX, tmY, use_tma_store,
+  return launch_pdl(kern, grid, dim3(TC_THREADS), smem, st, dim3(1, 1, ksplit), tmW, tmX, tmY, use_tma_store,
                     s_x, s_w, M, N, K, ksplit, static_cast<TOut*>(Y), acc_dbg);
 }
 

@@ -27,53 +27,9 @@
 //   tiles meet in shared memory and one pass sums, shifts (>> 6, or >> 10 for
 //   int4 activations held as 16*x) and dequantises:
 //   y = float(acc) * ((1/s_x) * (1/s_w)) in fp32 round-to-nearest.
-#include <cuda_bf16.h>
-
-#include "common.cuh"
+#include "decode_common.cuh"
 
 namespace bitnet {
-
-constexpr int DEC_WARPS = 8;
-constexpr int DEC_THREADS = 32 * DEC_WARPS;
-constexpr int DEC_MAX_TOKENS = 32;
-constexpr int DEC_MAX_SEGS = 32;                 // K <= 16384
-constexpr size_t DEC_W_SMEM_MAX = 96 * 1024;
-
-// Per token-group count TG (groups of 8 tokens): weight rows per CTA and K
-// segments whose activations are held in registers at once (the register
-// budget is 128 per thread for two CTAs per SM).
-template <int TG> struct DecCfg {
-  static constexpr int TOK = 8 * TG;
-  static constexpr int RG_MAX = TG == 4 ? 2 : 4;            // groups of 16 weight rows
-  static constexpr int MAX_ROWS = 16 * RG_MAX;
-  static constexpr int PASS_BATCH = TG == 4 ? 4 : 8;
-};
-
-template <typename T> BN_DEV void dec_store(T* p, float v);
-template <> BN_DEV void dec_store<float>(float* p, float v) { *p = v; }
-template <> BN_DEV void dec_store<__nv_bfloat16>(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
-
-// D[16 x 8] += A[16 x 32] * B[32 x 8], s8 inputs, s32 accumulators.
-BN_DEV void mma_s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                         uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// 16 int4 codes (8 bytes, code 2j in the low nibble of byte j) -> 16 int8
-// values 16*x in K order.
-BN_DEV uint4 widen16(uint2 p) {
-  uint4 r;
-  const uint32_t e0 = (p.x << 4) & 0xF0F0F0F0u, o0 = p.x & 0xF0F0F0F0u;
-  const uint32_t e1 = (p.y << 4) & 0xF0F0F0F0u, o1 = p.y & 0xF0F0F0F0u;
-  r.x = __byte_perm(e0, o0, 0x5140);
-  r.y = __byte_perm(e0, o0, 0x7362);
-  r.z = __byte_perm(e1, o1, 0x5140);
-  r.w = __byte_perm(e1, o1, 0x7362);
-  return r;
-}
 
 // TG = token groups of 8 (1: M <= 8, 2: M <= 16, 4: M <= 32); RG = groups of
 // 16 weight rows per CTA (rows = 16 * RG).  Both are compile-time so that one
@@ -89,9 +45,8 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
   using C = DecCfg<TG>;
   constexpr int TOK = C::TOK, PB = C::PASS_BATCH;
   constexpr int ROWS = 16 * RG;
-  constexpr int NACC = TG == 1 ? 2 : 1;                      // accumulator sets
+  constexpr int NACC = C::NACC;
   constexpr int SHIFT = ACT_BITS == 8 ? 6 : 10;
-  constexpr uint32_t SEG_BYTES = ROWS * 128u;
   static_assert(RG >= 1 && RG <= C::RG_MAX, "row groups");
   extern __shared__ uint8_t dec_smem_raw[];
   __shared__ float sdq[TOK];
@@ -105,21 +60,8 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
   // This kernel holds no tensor memory, so the next kernel in the stream may
   // be scheduled at once (it only waits for this grid to finish).
   pdl_launch_dependents();
-  {
-    // The weights do not depend on the previous kernel: stream them now.
-    // Chunk c (16 bytes): segment (c / 8) / ROWS, row (c / 8) % ROWS, chunk c % 8.
-    const size_t wrow = (size_t)K / 4;
-    const int nchunks = nseg * ROWS * 8;
-    const uint32_t sbase = smem_u32(wsm);
-    for (int c = threadIdx.x; c < nchunks; c += DEC_THREADS) {
-      const int q = c & 7, line = c >> 3;
-      const int sg = line / ROWS, r = line - sg * ROWS;
-      const bool in = n0 + r < N;                         // rows past N read as zeros
-      const uint8_t* src = pkW + (in ? (size_t)(n0 + r) * wrow + 128 * (size_t)sg + 16 * q : 0);
-      cp_async_16(sbase + sg * SEG_BYTES + (uint32_t)r * 128u + 16u * (uint32_t)(q ^ (r & 7)), src, in ? 16u : 0u);
-    }
-    cp_async_commit();
-  }
+  // the weights do not depend on the previous kernel: stream them now
+  dec_copy_weights<ROWS>(pkW, N, K, n0, wsm);
   // s_w belongs to the weights: read it before the wait as well
   const float sw = threadIdx.x < TOK ? ldg_nc_f32(s_w_ptr) : 0.0f;
   pdl_wait();                                  // activations and s_x come from the previous kernel
@@ -135,18 +77,6 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
       for (int tg = 0; tg < TG; ++tg)
 #pragma unroll
         for (int j = 0; j < 4; ++j) d[h][rg][tg][j] = 0;
-
-  // this thread's packed words of one segment: rows 16 rg + g and + 8, word t
-  // of 16-byte chunk `warp` (stored at chunk warp ^ (row & 7); (row & 7) = g)
-  const uint32_t woff = (uint32_t)g * 128u + 16u * (uint32_t)(warp ^ g) + 4u * (uint32_t)t;
-  auto load_w = [&](int sg, uint32_t (&w)[RG][2]) {
-    const uint8_t* base = wsm + (size_t)sg * SEG_BYTES + woff;
-#pragma unroll
-    for (int rg = 0; rg < RG; ++rg) {
-      w[rg][0] = *reinterpret_cast<const uint32_t*>(base + rg * 2048);
-      w[rg][1] = *reinterpret_cast<const uint32_t*>(base + rg * 2048 + 1024);
-    }
-  };
 
   const size_t xrow = ACT_BITS == 8 ? (size_t)K : (size_t)K / 2;
   uint32_t wcur[RG][2];
@@ -179,35 +109,15 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
     if (u0 == 0) {
       cp_async_wait_all();                     // this thread's weight copies
       __syncthreads();                         // and everyone else's
-      load_w(0, wcur);
+      dec_load_w<RG>(wsm, 0, warp, g, t, wcur);
     }
 #pragma unroll
     for (int u = 0; u < PB; ++u) {
       const int s = u0 + u;
       if (s < nseg) {
         uint32_t wnxt[RG][2];
-        load_w(s + 1 < nseg ? s + 1 : s, wnxt);            // next segment's words, ahead of use
-        // quarters 0,1 (first MMA) and 2,3 (second MMA) of each packed word,
-        // moved into the top two bits of every byte: int8 64 * w
-        uint32_t a[RG][2][4];
-#pragma unroll
-        for (int rg = 0; rg < RG; ++rg) {
-          const uint32_t wl = wcur[rg][0], wh = wcur[rg][1];
-          a[rg][0][0] = (wl << 6) & 0xC0C0C0C0u;  a[rg][0][1] = (wh << 6) & 0xC0C0C0C0u;
-          a[rg][0][2] = (wl << 4) & 0xC0C0C0C0u;  a[rg][0][3] = (wh << 4) & 0xC0C0C0C0u;
-          a[rg][1][0] = (wl << 2) & 0xC0C0C0C0u;  a[rg][1][1] = (wh << 2) & 0xC0C0C0C0u;
-          a[rg][1][2] = wl & 0xC0C0C0C0u;         a[rg][1][3] = wh & 0xC0C0C0C0u;
-        }
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int h = NACC == 2 ? q : 0;
-#pragma unroll
-          for (int rg = 0; rg < RG; ++rg)
-#pragma unroll
-            for (int tg = 0; tg < TG; ++tg)
-              mma_s8_16832(d[h][rg][tg], a[rg][q][0], a[rg][q][1], a[rg][q][2], a[rg][q][3],
-                           q == 0 ? xv[u][tg].x : xv[u][tg].z, q == 0 ? xv[u][tg].y : xv[u][tg].w);
-        }
+        dec_load_w<RG>(wsm, s + 1 < nseg ? s + 1 : s, warp, g, t, wnxt);   // next segment, ahead of use
+        dec_segment_mma<TG, RG, NACC>(d, wcur, xv[u]);
 #pragma unroll
         for (int rg = 0; rg < RG; ++rg) { wcur[rg][0] = wnxt[rg][0]; wcur[rg][1] = wnxt[rg][1]; }
       }
@@ -215,40 +125,8 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
   }
 
   if (threadIdx.x < M && threadIdx.x < TOK) sdq[threadIdx.x] = __fmul_rn(__fdiv_rn(1.0f, sx), __fdiv_rn(1.0f, sw));
-  __syncthreads();                             // all warps are done with the weight slice
-
-  // partial tiles [warp][token][row], row pitch ROWS + 4 (conflict-free stores)
-  constexpr int RP = ROWS + 4;
-  int32_t* red = reinterpret_cast<int32_t*>(wsm);
-  int32_t* mine = red + (size_t)warp * TOK * RP;
-#pragma unroll
-  for (int rg = 0; rg < RG; ++rg) {
-#pragma unroll
-    for (int tg = 0; tg < TG; ++tg) {
-      int v[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = NACC == 2 ? d[0][rg][tg][j] + d[NACC - 1][rg][tg][j] : d[0][rg][tg][j];
-      const int tok = 8 * tg + 2 * t, r = 16 * rg + g;
-      mine[tok * RP + r] = v[0];
-      mine[(tok + 1) * RP + r] = v[1];
-      mine[tok * RP + r + 8] = v[2];
-      mine[(tok + 1) * RP + r + 8] = v[3];
-    }
-  }
-  __syncthreads();
-  const int mcount = M < TOK ? M : TOK;
-  for (int idx = threadIdx.x; idx < mcount * ROWS; idx += DEC_THREADS) {
-    const int m = idx / ROWS, nn = idx - m * ROWS;
-    const int n = n0 + nn;
-    if (n < N) {
-      int acc = 0;
-#pragma unroll
-      for (int w = 0; w < DEC_WARPS; ++w) acc += red[((size_t)w * TOK + m) * RP + nn];
-      acc >>= SHIFT;
-      if (acc_dbg) acc_dbg[(size_t)m * N + n] = acc;
-      dec_store(Y + (size_t)m * N + n, __fmul_rn((float)acc, sdq[m]));
-    }
-  }
+  // the partial tiles reuse the weight slice's memory (after the epilogue's barrier)
+  dec_epilogue<TG, RG, NACC, SHIFT>(d, reinterpret_cast<int32_t*>(wsm), sdq, M, N, n0, Y, acc_dbg);
 }
 
 // ---------------------------------------------------------------------------
@@ -258,21 +136,12 @@ bool decode_path_applies(int M, int K) {
   return M >= 1 && M <= DEC_MAX_TOKENS && K % 512 == 0 && K / 512 <= DEC_MAX_SEGS;
 }
 
-// Weight rows per CTA: spread N over the SMs in multiples of 16, at most
-// max_rows, with the weight slice within the shared-memory budget.
-static int decode_rows(int N, int K, int sms, int max_rows) {
-  int rows = 16 * ((N + 16 * sms - 1) / (16 * sms));
-  if (rows > max_rows) rows = max_rows;
-  while (rows > 16 && (size_t)rows * (size_t)K / 4 > DEC_W_SMEM_MAX) rows -= 16;
-  return rows;
-}
-
 template <int ACT_BITS, int TG, int RG, typename TOut>
 static cudaError_t launch_decode_rg(const void* Xq, const float* s_x, const uint8_t* pkW, const float* s_w, int M,
                                     int N, int K, void* Y, int32_t* acc_dbg, cudaStream_t st) {
   constexpr int ROWS = 16 * RG;
   const size_t wbytes = (size_t)ROWS * (size_t)K / 4;
-  const size_t rbytes = (size_t)DEC_WARPS * DecCfg<TG>::TOK * (size_t)(ROWS + 4) * sizeof(int32_t);
+  const size_t rbytes = dec_red_bytes<TG, RG>();
   const size_t smem = (wbytes > rbytes ? wbytes : rbytes) + 1024;
   auto kern = linear_decode_kernel<ACT_BITS, TG, RG, TOut>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);

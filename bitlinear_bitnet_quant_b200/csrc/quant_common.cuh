@@ -1,0 +1,49 @@
+// Pieces of the RMSNorm + absmax quantisers shared by act_quant.cu and the
+// fused decode kernel (bitlinear_fused.cu): 16-byte input chunks and the
+// fixed pairwise-tree reductions.
+#pragma once
+
+#include "common.cuh"
+
+namespace bitnet {
+
+// One 16-byte chunk of activations (E elements), read with a coherent load
+// (the activations come from the previous kernel).
+template <typename TIn> struct InVec;
+template <> struct InVec<float> {
+  static constexpr int E = 4;
+  static BN_DEV void load(const float* p, float (&v)[4]) {
+    uint4 u = ldg_v4(p);
+    v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+    v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+  }
+};
+template <> struct InVec<uint16_t> {
+  static constexpr int E = 8;
+  static BN_DEV void load(const uint16_t* p, float (&v)[8]) {
+    uint4 u = ldg_v4(p);
+    v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+    v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+  }
+};
+
+// Balanced tree over N (power of two) register values, in index order.
+template <int N>
+BN_DEV float tree_sum(float (&a)[N]) {
+#pragma unroll
+  for (int s = 1; s < N; s <<= 1) {
+#pragma unroll
+    for (int i = 0; i < N; i += 2 * s) a[i] = __fadd_rn(a[i], a[i + s]);
+  }
+  return a[0];
+}
+
+// Tree over the 32 lanes: after offsets 1, 2, 4, 8, 16 every lane holds the
+// sum in which lane pairs (2u, 2u+1), then quads, ... were combined in order.
+BN_DEV float warp_tree_sum(float v) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+}  // namespace bitnet

@@ -167,6 +167,28 @@ BITNET_API int bitnet_linear(const void* Xq, int act_bits, const float* s_x, con
                   void* Y, int y_dtype, int32_t* acc_dbg, void* stream);
 
 /*
+ * Fused BitLinear forward with int8 activations: bitnet_quant_act followed by
+ * bitnet_linear (act_bits = 8) in one call, with bit-identical results
+ * [P4 양자화 메커니즘, 계산 패러다임, 추론 최적화 및 커스텀 커널].
+ * X      : [M][K] fp32 or bf16 (x_dtype).   gamma: [K] fp32 or NULL (= 1).
+ * pkW    : [N][K/4] packed ternary weights.  s_w: one fp32 (device).
+ * Y      : out, [M][N] fp32 or bf16 (y_dtype).
+ * Xq, s_x: out, [M][K] int8 codes and [M] fp32 scales (always written).
+ * Kernels: up to 32 tokens with K % 512 == 0 and K <= 8192 (and the codes of
+ *          all tokens within shared memory), one kernel: thread-block
+ *          clusters of 8 CTAs share the quantisation (each CTA quantises
+ *          every eighth token and copies codes and scale into the shared
+ *          memory of the other seven), then the one-pass decode product.
+ *          Otherwise the two kernels of bitnet_quant_act and bitnet_linear.
+ *          With bitnet_set_linear_path(p != 0) always the two kernels.
+ * Limits : M >= 0, N >= 1, 128 <= K <= 16384, K % 128 == 0; gamma, X, Xq,
+ *          pkW and Y 16-byte aligned.
+ */
+BITNET_API int bitnet_bitlinear(const void* X, int x_dtype, int64_t M, int64_t K, const float* gamma, float eps,
+                     const uint8_t* pkW, const float* s_w, int64_t N, void* Y, int y_dtype,
+                     int8_t* Xq, float* s_x, void* stream);
+
+/*
  * Element-wise glue of the stacked BitLinear chain (a transformer layer whose
  * linear layers are BitLinear; P2 주요 아키텍처 혁신: squared ReLU, no bias).
  * bitnet_add:        out[i] = a[i] + b[i]                      (fp32 residual)

@@ -94,6 +94,21 @@ def test_weights_validation(L):
     assert w(pk=MISALIGNED) == 3
 
 
+def test_bitlinear_validation(L):
+    def b(**kw):
+        a = dict(X=ALIGNED, dt=1, M=4, K=512, gamma=None, pkW=ALIGNED, s_w=ALIGNED, N=256, Y=ALIGNED, yt=0,
+                 Xq=ALIGNED, s_x=ALIGNED)
+        a.update(kw)
+        return L.bitnet_bitlinear(a["X"], a["dt"], a["M"], a["K"], a["gamma"], 1e-6, a["pkW"], a["s_w"], a["N"],
+                                  a["Y"], a["yt"], a["Xq"], a["s_x"], None)
+    assert b(dt=2) == 4 and b(yt=3) == 4
+    assert b(K=100) == 2 and b(K=64) == 2 and b(K=16384 + 128) == 2 and b(N=0) == 2 and b(M=-1) == 2
+    assert b(M=0) == 0
+    assert b(X=None) == 1 and b(Xq=None) == 1 and b(s_x=None) == 1 and b(Y=None) == 1 and b(pkW=None) == 1
+    assert b(X=MISALIGNED) == 3 and b(Xq=MISALIGNED) == 3 and b(gamma=MISALIGNED) == 3
+    assert b(s_x=ALIGNED + 2) == 3
+
+
 def test_linear_path_selector(L):
     assert L.bitnet_set_linear_path(4) == 2
     assert L.bitnet_set_linear_path(3) == 0

@@ -263,6 +263,55 @@ def test_linear_decode_full(M):
     assert np.array_equal(host(Y).view(np.uint32), y_o.view(np.uint32))
 
 
+# ------------------------------------------------------- fused BitLinear ----
+
+def _check_bitlinear(M, N, K, dtype, use_gamma, out, path=0, seed=0):
+    rng = np.random.default_rng(seed + M * 31 + K)
+    x = wl.add_entry_outliers(rng, wl.gaussian(rng, (M, K)), 0.005, 30.0)
+    xd, x_or = x_inputs(x, dtype)
+    gamma = rng.uniform(0.5, 1.5, K).astype(np.float32) if use_gamma else None
+    w = wl.weights(N, K, seed=seed + N)
+    pk, s_w = api.bitnet_quantize_weights(dev(w))
+    api.bitnet_set_linear_path(path)
+    try:
+        Y, q, s = api.bitnet_bitlinear(xd, pk, s_w, dev(gamma) if use_gamma else None, 1e-6,
+                                       out_dtype=torch.float32 if out == "f32" else torch.bfloat16)
+        torch.cuda.synchronize()
+    finally:
+        api.bitnet_set_linear_path(0)
+    assert api.bitnet_device_error() == 0
+    _, s_wo, qw_o = O.quantize_weights(w)
+    q_o, s_o = O.quant_act(x_or, gamma, 1e-6)
+    assert np.array_equal(host(s).view(np.uint32), s_o.view(np.uint32))
+    assert np.array_equal(host(q), q_o)
+    acc_o, y_o = O.linear(q_o, s_o, qw_o, s_wo)
+    if out == "f32":
+        assert np.array_equal(host(Y).view(np.uint32), y_o.view(np.uint32))
+    else:
+        assert np.array_equal(O.bf16_round(host(Y.float())), O.bf16_round(y_o))
+
+
+@pytest.mark.parametrize("M,N,K,dtype,use_gamma,out", [
+    (1, 6912, 2560, "bf16", False, "f32"), (4, 6912, 2560, "bf16", False, "f32"),
+    (16, 6912, 2560, "bf16", False, "bf16"), (3, 200, 512, "f32", True, "f32"), (8, 1000, 1536, "bf16", True, "f32"),
+    (9, 2048, 2048, "f32", False, "f32"), (17, 5632, 2048, "f32", True, "f32"), (32, 2048, 2048, "f32", False, "bf16"),
+    (32, 300, 8192, "bf16", False, "f32"), (12, 16, 4608, "f32", False, "f32"), (1, 1, 512, "bf16", False, "f32")])
+def test_bitlinear_fused(M, N, K, dtype, use_gamma, out):
+    """One kernel: clusters of 8 CTAs quantise every eighth token each and
+    share the codes through distributed shared memory; the codes, scales and
+    outputs match the oracle bit for bit (ragged N, 1 to 4 token groups, K of
+    1 to 16 segments, grids padded to whole clusters)."""
+    _check_bitlinear(M, N, K, dtype, use_gamma, out)
+
+
+@pytest.mark.parametrize("M,N,K,path", [(40, 512, 1024, 0), (4, 256, 384, 0), (16, 6912, 2560, 2),
+                                        (5, 300, 1024, 3), (2, 128, 16384, 0)])
+def test_bitlinear_two_kernel_paths(M, N, K, path):
+    """Shapes the fused kernel does not cover, and forced kernel families:
+    the quantiser and the selected linear kernel in sequence."""
+    _check_bitlinear(M, N, K, "bf16", False, "f32", path=path)
+
+
 def test_linear_prefill_sampled():
     c = wl.prefill()
     xd, x_or = x_inputs(c["x"], "bf16")
