@@ -246,16 +246,11 @@ def run_ours(args, rank, world, local_rank):
         pk, s_w = ring[i % copies]
         api.bitnet_linear(xq, bits, s_x, pk, s_w, Y=Y, stream=stream)
 
-    # a few tokens with int8 activations: the fused entry point (one kernel per step)
-    fused = bits == 8 and M <= 32 and K % 512 == 0 and K <= 8192
-
+    # the step is the quantiser and the linear kernel (the single-kernel path
+    # of bitnet_bitlinear is slower on B200; the decode sweep reports it)
     def step(i):
-        if fused:
-            pk, s_w = ring[i % copies]
-            api.bitnet_bitlinear(x, pk, s_w, None, eps, Y=Y, Xq=xq, s_x=s_x, stream=stream)
-        else:
-            quant()
-            linear(i)
+        quant()
+        linear(i)
 
     warmup = max(3, args.warmup)
     for i in range(warmup):
@@ -331,17 +326,26 @@ def run_ours(args, rank, world, local_rank):
                 pk, s_w = ring[i % copies]
                 api.bitnet_bitlinear(xs, pk, s_w, None, eps, Y=Ys, Xq=xqs, s_x=sxs, stream=stream)
 
+            def step_s(i, xs=xs, xqs=xqs, sxs=sxs, Ys=Ys):
+                api.bitnet_quant_act(xs, None, eps, Xq=xqs, s_x=sxs, stream=stream)
+                lin_s(i)
+
+            api.bitnet_set_linear_path(4)
+            for i in range(warmup):
+                fused_s(i)
+            t_f = timed(graph_of(fused_s, steps)) / steps / 1e3
+            api.bitnet_set_linear_path(0)
             for i in range(warmup):
                 lin_s(i)
-                fused_s(i)
+                step_s(i)
             t_s = timed(graph_of(lin_s, steps)) / steps / 1e3
-            t_f = timed(graph_of(fused_s, steps)) / steps / 1e3
+            t_st = timed(graph_of(step_s, steps)) / steps / 1e3
             hbm = load_peaks()[0]["hbm_gbs"]
             b = packed_bytes + Ms * K + 4 * Ms + 4 + Ms * N * out_bytes
             bf = packed_bytes + 2 * Ms * K + Ms * K + 4 * Ms + 4 + Ms * N * out_bytes
             sweep.append({"M": Ms, "linear_us": t_s * 1e6, "linear_GBs": b / t_s / 1e9,
-                          "linear_frac": b / t_s / 1e9 / hbm, "fused_us": t_f * 1e6, "fused_GBs": bf / t_f / 1e9,
-                          "fused_frac": bf / t_f / 1e9 / hbm, "tokens_per_s_fused": Ms / t_f})
+                          "linear_frac": b / t_s / 1e9 / hbm, "step_us": t_st * 1e6, "tokens_per_s": Ms / t_st,
+                          "fused_kernel_us": t_f * 1e6, "fused_kernel_frac": bf / t_f / 1e9 / hbm})
 
     if rank != 0:
         return None
@@ -354,18 +358,7 @@ def run_ours(args, rank, world, local_rank):
     q_s = t_q / steps / 1e3
     x_in_bytes = M * K * (2 if c["x_dtype"] == "bf16" else 4)
     xq_bytes = M * K if bits == 8 else M * K // 2
-    if fused:
-        # the step is one kernel: RMSNorm + int8 codes + product + dequant
-        alg_bytes = packed_bytes + x_in_bytes + xq_bytes + 4 * M + 4 + M * N * out_bytes
-        step_s = t_step / steps / 1e3
-        roof = {"bound": "hbm", "achieved": alg_bytes / step_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "kernel": "bitnet_bitlinear (fused decode, clusters of 8)", "algorithmic_bytes_per_launch": alg_bytes}
-        tag = f"bitlinear_{args.workload}"
-        lin_bytes = packed_bytes + xq_bytes + 4 * M + 4 + M * N * out_bytes
-        linear_roof = {"kernel": "bitnet_linear (warp-MMA decode), separately", "achieved": lin_bytes / lin_s / 1e9,
-                       "unit": "GB/s", "frac": lin_bytes / lin_s / 1e9 / peaks["hbm_gbs"],
-                       "algorithmic_bytes_per_launch": lin_bytes}
-    elif args.workload.startswith("decode") or args.workload == "tiny":
+    if args.workload.startswith("decode") or args.workload == "tiny":
         alg_bytes = packed_bytes + xq_bytes + 4 * M + 4 + M * N * out_bytes
         roof = {"bound": "hbm", "achieved": alg_bytes / lin_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "kernel": "bitnet_linear (warp-MMA decode)" if M <= 32 and K % 512 == 0 else "bitnet_linear (tcgen05)",
@@ -393,18 +386,16 @@ def run_ours(args, rank, world, local_rank):
                    "timing": "CUDA graph of the K steps, CUDA events on the launching stream",
                    "parallelism": f"dp{world} (independent batches per rank)"},
         "roofline": roof,
-        "kernels_us": {"quant": q_s * 1e6, "linear": lin_s * 1e6, **({"fused": t_step / steps * 1e3} if fused else {})},
+        "kernels_us": {"quant": q_s * 1e6, "linear": lin_s * 1e6},
         "quant_roofline": {"bound": "hbm", "achieved": quant_bytes / q_s / 1e9, "peak": peaks["hbm_gbs"],
                            "unit": "GB/s", "frac": quant_bytes / q_s / 1e9 / peaks["hbm_gbs"]},
         "e2e": {"value": tokens_per_step * steps / (t_e2e / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": (1 if fused else 2) * steps,
+        "gpu_launches": 2 * steps,
         "clocks": clk,
     }
     if sweep:
         line["decode_sweep"] = sweep
-    if fused:
-        line["linear_roofline"] = linear_roof
     return line
 
 

@@ -6,12 +6,12 @@ BitNet v2 the O and down projections are H-BitLinear (Hadamard + int4).
 Per layer, with fp32 residuals:
 
     q, k, v = BitLinear(x)                      (one int8 quantisation of x,
-                                                 fused into q's call)
+                                                 in q's call; k, v reuse it)
     o = H-BitLinear(v)                          (attention over a one-token
                                                  context returns V)
     h = x + o
     up, gate = BitLinear(h)                     (one int8 quantisation of h,
-                                                 fused into up's call)
+                                                 in up's call; gate reuses it)
     a = relu(gate)^2 * up                       (squared-ReLU gated unit)
     x' = h + H-BitLinear(a)                     (down projection)
 
@@ -55,7 +55,7 @@ class BitLinearChain:
 
     def layer(self, x: torch.Tensor, w: dict, out: torch.Tensor, stream=None) -> torch.Tensor:
         A, s = api, stream
-        # q: the fused entry point quantises x (codes and scales kept for k, v)
+        # q: bitnet_bitlinear quantises x (codes and scales kept for k, v)
         A.bitnet_bitlinear(x, *w["q"], None, self.eps, Y=self.q, Xq=self.xq, s_x=self.sx, stream=s)
         for name, Y in (("k", self.k), ("v", self.v)):
             A.bitnet_linear(self.xq, 8, self.sx, *w[name], Y=Y, stream=s)
@@ -78,13 +78,12 @@ class BitLinearChain:
             cur = self.layer(cur, w, self.x[i % 2], stream)
         return cur
 
-    # kernels launched per forward: per layer 2 fused BitLinear calls (one
-    # kernel each for a few tokens, else a quantiser and a linear layer),
-    # 5 further linear layers, 2 Hadamard quantisers, 2 adds, 1 gated unit
+    # kernels launched per forward: per layer 2 BitLinear calls (a quantiser
+    # and a linear layer each), 5 further linear layers, 2 Hadamard
+    # quantisers, 2 adds, 1 gated unit
     @property
     def launches(self) -> int:
-        fused = self.M <= 32 and self.hidden % 512 == 0 and self.hidden <= 8192
-        return (12 if fused else 14) * len(self.layers)
+        return 14 * len(self.layers)
 
     def packed_bytes(self) -> int:
         return sum(pk.numel() for w in self.layers for pk, _ in w.values())

@@ -24,6 +24,7 @@ cudaError_t run_bitlinear(const void* X, int x_bf16, int M, int K, const float* 
                           const float* s_w, int N, void* Y, int y_bf16, int8_t* Xq, float* s_x, int path,
                           cudaStream_t st);
 bool decode_path_applies(int M, int K);
+bool fused_path_applies(int M, int K, int x_bf16);
 cudaError_t run_add_f32(const float* a, const float* b, float* out, size_t n, cudaStream_t st);
 cudaError_t run_relu2_glu(const float* gate, const float* up, float* out, size_t n, cudaStream_t st);
 }  // namespace bitnet
@@ -58,7 +59,8 @@ int cuda_status(cudaError_t e) {
   return BITNET_ERR_CUDA;
 }
 
-// 0 = automatic, 1 = SIMT, 2 = tcgen05, 3 = warp-MMA decode (set by bitnet_set_linear_path).
+// 0 = automatic, 1 = SIMT, 2 = tcgen05, 3 = warp-MMA decode, 4 = fused BitLinear kernel
+// (set by bitnet_set_linear_path).
 std::atomic<int> g_linear_path{0};
 int linear_path() { return g_linear_path.load(std::memory_order_relaxed); }
 
@@ -182,6 +184,7 @@ int bitnet_bitlinear(const void* X, int x_dtype, int64_t M, int64_t K, const flo
   if (!bitnet::tensor_map_encoder_available()) return BITNET_ERR_UNSUPPORTED;
   const int path = linear_path();
   if (path == 3 && !bitnet::decode_path_applies((int)M, (int)K)) return BITNET_ERR_SHAPE;
+  if (path == 4 && !bitnet::fused_path_applies((int)M, (int)K, x_dtype == BITNET_BF16)) return BITNET_ERR_SHAPE;
   return cuda_status(bitnet::run_bitlinear(X, x_dtype == BITNET_BF16, (int)M, (int)K, gamma, eps, pkW, s_w, (int)N,
                                            Y, y_dtype == BITNET_BF16, Xq, s_x, path,
                                            static_cast<cudaStream_t>(stream)));
@@ -200,7 +203,7 @@ int bitnet_relu2_glu(const float* gate, const float* up, float* out, int64_t n, 
 }
 
 int bitnet_set_linear_path(int path) {
-  if (path < 0 || path > 3) return BITNET_ERR_SHAPE;
+  if (path < 0 || path > 4) return BITNET_ERR_SHAPE;
   g_linear_path.store(path, std::memory_order_relaxed);
   return BITNET_OK;
 }

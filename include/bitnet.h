@@ -174,13 +174,15 @@ BITNET_API int bitnet_linear(const void* Xq, int act_bits, const float* s_x, con
  * pkW    : [N][K/4] packed ternary weights.  s_w: one fp32 (device).
  * Y      : out, [M][N] fp32 or bf16 (y_dtype).
  * Xq, s_x: out, [M][K] int8 codes and [M] fp32 scales (always written).
- * Kernels: up to 32 tokens with K % 512 == 0 and K <= 8192 (and the codes of
- *          all tokens within shared memory), one kernel: thread-block
- *          clusters of 8 CTAs share the quantisation (each CTA quantises
- *          every eighth token and copies codes and scale into the shared
- *          memory of the other seven), then the one-pass decode product.
- *          Otherwise the two kernels of bitnet_quant_act and bitnet_linear.
- *          With bitnet_set_linear_path(p != 0) always the two kernels.
+ * Kernels: by default the two kernels of bitnet_quant_act and bitnet_linear
+ *          (on B200 the faster choice for every decode shape measured: the
+ *          quantiser overlaps the linear kernel's weight stream).  After
+ *          bitnet_set_linear_path(4), one fused kernel: thread-block clusters
+ *          of 8 CTAs share the quantisation (each CTA quantises every eighth
+ *          token and copies codes and scale into the shared memory of the
+ *          other seven), then the one-pass decode product; it covers up to
+ *          32 tokens with K % 512 == 0 and K <= 8192 (else BITNET_ERR_SHAPE).
+ *          Paths 1-3 select the linear kernel family as for bitnet_linear.
  * Limits : M >= 0, N >= 1, 128 <= K <= 16384, K % 128 == 0; gamma, X, Xq,
  *          pkW and Y 16-byte aligned.
  */
@@ -204,8 +206,9 @@ BITNET_API int bitnet_relu2_glu(const float* gate, const float* up, float* out, 
  * 0 = automatic (default: warp-MMA decode kernel where it applies, else the
  * tcgen05 tensor-core kernel), 1 = CUDA-core dp4a kernel, 2 = tcgen05 kernel,
  * 3 = warp-MMA decode kernel (bitnet_linear then returns BITNET_ERR_SHAPE for
- * shapes it does not cover: M > 32, K % 512 != 0 or K > 16384).  All compute
- * the same bit-exact result.  Returns BITNET_ERR_SHAPE for any other value.
+ * shapes it does not cover: M > 32, K % 512 != 0 or K > 16384), 4 = the fused
+ * kernel of bitnet_bitlinear (bitnet_linear as with 0).  All compute the same
+ * bit-exact result.  Returns BITNET_ERR_SHAPE for any other value.
  */
 BITNET_API int bitnet_set_linear_path(int path);
 

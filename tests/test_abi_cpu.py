@@ -110,7 +110,8 @@ def test_bitlinear_validation(L):
 
 
 def test_linear_path_selector(L):
-    assert L.bitnet_set_linear_path(4) == 2
+    assert L.bitnet_set_linear_path(5) == 2
+    assert L.bitnet_set_linear_path(4) == 0
     assert L.bitnet_set_linear_path(3) == 0
     assert L.bitnet_set_linear_path(-1) == 2
     assert L.bitnet_set_linear_path(0) == 0

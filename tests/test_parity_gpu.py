@@ -301,15 +301,21 @@ def test_bitlinear_fused(M, N, K, dtype, use_gamma, out):
     share the codes through distributed shared memory; the codes, scales and
     outputs match the oracle bit for bit (ragged N, 1 to 4 token groups, K of
     1 to 16 segments, grids padded to whole clusters)."""
-    _check_bitlinear(M, N, K, dtype, use_gamma, out)
+    _check_bitlinear(M, N, K, dtype, use_gamma, out, path=4)
+    _check_bitlinear(M, N, K, dtype, use_gamma, out, path=0)     # the two-kernel default
 
 
 @pytest.mark.parametrize("M,N,K,path", [(40, 512, 1024, 0), (4, 256, 384, 0), (16, 6912, 2560, 2),
-                                        (5, 300, 1024, 3), (2, 128, 16384, 0)])
+                                        (5, 300, 1024, 3), (2, 128, 16384, 0), (3, 100, 1024, 1)])
 def test_bitlinear_two_kernel_paths(M, N, K, path):
-    """Shapes the fused kernel does not cover, and forced kernel families:
-    the quantiser and the selected linear kernel in sequence."""
+    """The quantiser and the selected linear kernel in sequence."""
     _check_bitlinear(M, N, K, "bf16", False, "f32", path=path)
+
+
+def test_bitlinear_fused_rejects_other_shapes():
+    for M, K in ((33, 512), (4, 384), (40, 1024)):
+        with pytest.raises(api.BitnetError):
+            _check_bitlinear(M, 64, K, "bf16", False, "f32", path=4)
 
 
 def test_linear_prefill_sampled():
