@@ -295,7 +295,8 @@ def _check_bitlinear(M, N, K, dtype, use_gamma, out, path=0, seed=0):
     (1, 6912, 2560, "bf16", False, "f32"), (4, 6912, 2560, "bf16", False, "f32"),
     (16, 6912, 2560, "bf16", False, "bf16"), (3, 200, 512, "f32", True, "f32"), (8, 1000, 1536, "bf16", True, "f32"),
     (9, 2048, 2048, "f32", False, "f32"), (17, 5632, 2048, "f32", True, "f32"), (32, 2048, 2048, "f32", False, "bf16"),
-    (32, 300, 8192, "bf16", False, "f32"), (12, 16, 4608, "f32", False, "f32"), (1, 1, 512, "bf16", False, "f32")])
+    (32, 300, 4096, "bf16", False, "f32"), (16, 300, 8192, "bf16", False, "f32"), (12, 16, 4608, "f32", False, "f32"),
+    (1, 1, 512, "bf16", False, "f32")])
 def test_bitlinear_fused(M, N, K, dtype, use_gamma, out):
     """One kernel: clusters of 8 CTAs quantise every eighth token each and
     share the codes through distributed shared memory; the codes, scales and
@@ -313,7 +314,7 @@ def test_bitlinear_two_kernel_paths(M, N, K, path):
 
 
 def test_bitlinear_fused_rejects_other_shapes():
-    for M, K in ((33, 512), (4, 384), (40, 1024)):
+    for M, K in ((33, 512), (4, 384), (40, 1024), (32, 8192)):
         with pytest.raises(api.BitnetError):
             _check_bitlinear(M, 64, K, "bf16", False, "f32", path=4)
 
