@@ -42,6 +42,10 @@ _SIGNATURES = {
     "bitnet_bitlinear": (ctypes.c_int, [_c_void_p, ctypes.c_int, _i64, _i64, _c_void_p, ctypes.c_float,
                                         _c_void_p, _c_void_p, _i64, _c_void_p, ctypes.c_int, _c_void_p, _c_void_p,
                                         _c_void_p]),
+    "bitnet_add_quant_act": (ctypes.c_int, [_c_void_p, _c_void_p, _i64, _i64, _c_void_p, ctypes.c_float, _c_void_p,
+                                            _c_void_p, _c_void_p, _c_void_p]),
+    "bitnet_glu_hadamard_quant_act": (ctypes.c_int, [_c_void_p, _c_void_p, _i64, _i64, _c_void_p, ctypes.c_float,
+                                                     ctypes.c_int, _c_void_p, _c_void_p, _c_void_p]),
     "bitnet_add": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _i64, _c_void_p]),
     "bitnet_relu2_glu": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _i64, _c_void_p]),
     "bitnet_set_linear_path": (ctypes.c_int, [ctypes.c_int]),
@@ -168,6 +172,33 @@ def bitnet_hadamard_quant_act(X: torch.Tensor, gamma=None, eps: float = 1e-6, ha
         _ptr(X), _dtype_code(X), M, K, _ptr(gamma), float(eps), int(had_block), _ptr(Xq4), _ptr(s_x),
         _ptr(T), _stream(stream)))
     return Xq4, s_x, T
+
+
+def bitnet_add_quant_act(A: torch.Tensor, B: torch.Tensor, gamma=None, eps: float = 1e-6, H=None, Xq=None, s_x=None,
+                         stream=None):
+    """H = A + B (fp32), then the int8 quantiser of H.  Returns (H, Xq, s_x)."""
+    _require(A, "A")
+    _require(B, "B")
+    M, K = A.shape
+    H = torch.empty_like(A) if H is None else H
+    Xq = torch.empty((M, K), dtype=torch.int8, device=A.device) if Xq is None else Xq
+    s_x = torch.empty((M,), dtype=torch.float32, device=A.device) if s_x is None else s_x
+    _check("bitnet_add_quant_act", lib().bitnet_add_quant_act(
+        _ptr(A), _ptr(B), M, K, _ptr(gamma), float(eps), _ptr(H), _ptr(Xq), _ptr(s_x), _stream(stream)))
+    return H, Xq, s_x
+
+
+def bitnet_glu_hadamard_quant_act(gate: torch.Tensor, up: torch.Tensor, gamma=None, eps: float = 1e-6,
+                                  had_block: int = 0, Xq4=None, s_x=None, stream=None):
+    """x = relu(gate)^2 * up (fp32), then the Hadamard int4 quantiser of x.  Returns (Xq4, s_x)."""
+    _require(gate, "gate")
+    _require(up, "up")
+    M, K = gate.shape
+    Xq4 = torch.empty((M, K // 2), dtype=torch.uint8, device=gate.device) if Xq4 is None else Xq4
+    s_x = torch.empty((M,), dtype=torch.float32, device=gate.device) if s_x is None else s_x
+    _check("bitnet_glu_hadamard_quant_act", lib().bitnet_glu_hadamard_quant_act(
+        _ptr(gate), _ptr(up), M, K, _ptr(gamma), float(eps), int(had_block), _ptr(Xq4), _ptr(s_x), _stream(stream)))
+    return Xq4, s_x
 
 
 def bitnet_linear(Xq: torch.Tensor, act_bits: int, s_x: torch.Tensor, pkW: torch.Tensor, s_w: torch.Tensor,

@@ -5,18 +5,19 @@ linear layers of attention and FFN are BitLinear (int8 activations), and in
 BitNet v2 the O and down projections are H-BitLinear (Hadamard + int4).
 Per layer, with fp32 residuals:
 
-    q, k, v = BitLinear(x)                      (one int8 quantisation of x,
-                                                 in q's call; k, v reuse it)
+    q, k, v = BitLinear(x)                      (one int8 quantisation of x)
     o = H-BitLinear(v)                          (attention over a one-token
                                                  context returns V)
     h = x + o
-    up, gate = BitLinear(h)                     (one int8 quantisation of h,
-                                                 in up's call; gate reuses it)
+    up, gate = BitLinear(h)                     (one int8 quantisation of h)
     a = relu(gate)^2 * up                       (squared-ReLU gated unit)
     x' = h + H-BitLinear(a)                     (down projection)
 
 Every step is a kernel of libbitnet.so; this module only sequences the calls
-and owns the activation buffers (allocated once per batch size).
+and owns the activation buffers (allocated once per batch size).  The
+element-wise steps run inside the quantiser that consumes them: h = x + o in
+the quantisation of h, a in the Hadamard quantisation of a, and x' = h + d
+in the next layer's first quantisation (a final add after the last layer).
 """
 from __future__ import annotations
 
@@ -41,7 +42,7 @@ class BitLinearChain:
         self.M, self.hidden, self.ffn, self.eps = M, hidden, ffn, eps
         f32 = dict(dtype=torch.float32, device=device)
         e = lambda *shape: torch.empty(shape, **f32)
-        self.x = [e(M, hidden), e(M, hidden)]          # ping-pong layer inputs
+        self.x = [e(M, hidden), e(M, hidden)]          # layer input, chain output
         self.xq = torch.empty((M, hidden), dtype=torch.int8, device=device)
         self.sx = e(M)
         self.q, self.k, self.v, self.o, self.h, self.d = (e(M, hidden) for _ in range(6))
@@ -49,41 +50,49 @@ class BitLinearChain:
         self.sv = e(M)
         self.hq = torch.empty((M, hidden), dtype=torch.int8, device=device)
         self.sh = e(M)
-        self.up, self.gate, self.a = e(M, ffn), e(M, ffn), e(M, ffn)
+        self.up, self.gate = e(M, ffn), e(M, ffn)
         self.a4 = torch.empty((M, ffn // 2), dtype=torch.uint8, device=device)
         self.sa = e(M)
 
-    def layer(self, x: torch.Tensor, w: dict, out: torch.Tensor, stream=None) -> torch.Tensor:
+    def layer(self, x_parts, w: dict, stream=None):
+        """One layer.  x_parts: (x,) or (h_prev, d_prev), whose sum is the
+        layer input.  Returns (h, d), whose sum is the layer output.  Buffers
+        are reused from layer to layer: every kernel waits for the one before
+        it, so a buffer is rewritten only after its last reader has finished."""
         A, s = api, stream
-        # q: bitnet_bitlinear quantises x (codes and scales kept for k, v)
-        A.bitnet_bitlinear(x, *w["q"], None, self.eps, Y=self.q, Xq=self.xq, s_x=self.sx, stream=s)
-        for name, Y in (("k", self.k), ("v", self.v)):
+        if len(x_parts) == 1:
+            x = x_parts[0]
+            A.bitnet_quant_act(x, None, self.eps, Xq=self.xq, s_x=self.sx, stream=s)
+        else:
+            x = self.x[0]
+            A.bitnet_add_quant_act(x_parts[0], x_parts[1], None, self.eps, H=x, Xq=self.xq, s_x=self.sx, stream=s)
+        for name, Y in (("q", self.q), ("k", self.k), ("v", self.v)):
             A.bitnet_linear(self.xq, 8, self.sx, *w[name], Y=Y, stream=s)
         A.bitnet_hadamard_quant_act(self.v, None, self.eps, 0, Xq4=self.v4, s_x=self.sv, stream=s)
         A.bitnet_linear(self.v4, 4, self.sv, *w["o"], Y=self.o, stream=s)
-        A.bitnet_add(x, self.o, out=self.h, stream=s)
-        A.bitnet_bitlinear(self.h, *w["up"], None, self.eps, Y=self.up, Xq=self.hq, s_x=self.sh, stream=s)
+        A.bitnet_add_quant_act(x, self.o, None, self.eps, H=self.h, Xq=self.hq, s_x=self.sh, stream=s)
+        A.bitnet_linear(self.hq, 8, self.sh, *w["up"], Y=self.up, stream=s)
         A.bitnet_linear(self.hq, 8, self.sh, *w["gate"], Y=self.gate, stream=s)
-        A.bitnet_relu2_glu(self.gate, self.up, out=self.a, stream=s)
-        A.bitnet_hadamard_quant_act(self.a, None, self.eps, 0, Xq4=self.a4, s_x=self.sa, stream=s)
+        A.bitnet_glu_hadamard_quant_act(self.gate, self.up, None, self.eps, 0, Xq4=self.a4, s_x=self.sa, stream=s)
         A.bitnet_linear(self.a4, 4, self.sa, *w["down"], Y=self.d, stream=s)
-        A.bitnet_add(self.h, self.d, out=out, stream=s)
-        return out
+        return self.h, self.d
 
     def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
         """x: [M, hidden] fp32 on the device; returns the last layer's output
         (one of the chain's own buffers)."""
-        cur = x
-        for i, w in enumerate(self.layers):
-            cur = self.layer(cur, w, self.x[i % 2], stream)
-        return cur
+        parts = (x,)
+        for w in self.layers:
+            parts = self.layer(parts, w, stream)
+        api.bitnet_add(parts[0], parts[1], out=self.x[1], stream=stream)
+        return self.x[1]
 
-    # kernels launched per forward: per layer 2 BitLinear calls (a quantiser
-    # and a linear layer each), 5 further linear layers, 2 Hadamard
-    # quantisers, 2 adds, 1 gated unit
+    # kernels launched per forward: per layer 2 int8 quantisers (the second, and
+    # from the second layer on the first, with the residual add folded in), 7
+    # linear layers, 2 Hadamard quantisers (one with the gated unit folded in);
+    # one residual add after the last layer
     @property
     def launches(self) -> int:
-        return 14 * len(self.layers)
+        return 11 * len(self.layers) + 1
 
     def packed_bytes(self) -> int:
         return sum(pk.numel() for w in self.layers for pk, _ in w.values())

@@ -20,11 +20,15 @@ cudaError_t run_hadamard_quant_i4(const void* X, int bf16, int M, int K, int L, 
 cudaError_t run_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                        int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, int path, cudaStream_t st);
 bool tensor_map_encoder_available();
+cudaError_t run_add_quant_act_i8(const float* A, const float* B, int M, int K, const float* gamma, float eps,
+                                 float* H, int8_t* Xq, float* s_x, cudaStream_t st);
+cudaError_t run_glu_hadamard_quant_i4(const float* gate, const float* up, int M, int K, int L, const float* gamma,
+                                      float eps, uint8_t* Xq4, float* s_x, cudaStream_t st);
 cudaError_t run_bitlinear(const void* X, int x_bf16, int M, int K, const float* gamma, float eps, const uint8_t* pkW,
                           const float* s_w, int N, void* Y, int y_bf16, int8_t* Xq, float* s_x, int path,
                           cudaStream_t st);
 bool decode_path_applies(int M, int K);
-bool fused_path_applies(int M, int K, int x_bf16);
+bool fused_path_applies(int M, int N, int K, int x_bf16);
 cudaError_t run_add_f32(const float* a, const float* b, float* out, size_t n, cudaStream_t st);
 cudaError_t run_relu2_glu(const float* gate, const float* up, float* out, size_t n, cudaStream_t st);
 }  // namespace bitnet
@@ -117,6 +121,39 @@ int bitnet_quant_act(const void* X, int x_dtype, int64_t M, int64_t K, const flo
                                               static_cast<cudaStream_t>(stream)));
 }
 
+int bitnet_add_quant_act(const float* A, const float* B, int64_t M, int64_t K, const float* gamma, float eps,
+                         float* H, int8_t* Xq, float* s_x, void* stream) {
+  if (M < 0 || M > (int64_t(1) << 30) || K < 16 || K > 16384 || K % 16 != 0) return BITNET_ERR_SHAPE;
+  if (M == 0) return BITNET_OK;
+  if (!A || !B || !H || !Xq || !s_x) return BITNET_ERR_NULL;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(H) || !aligned16(Xq) || (gamma && !aligned16(gamma)) ||
+      (reinterpret_cast<uintptr_t>(s_x) & 3u))
+    return BITNET_ERR_ALIGN;
+  int d = check_device();
+  if (d != BITNET_OK) return d;
+  return cuda_status(bitnet::run_add_quant_act_i8(A, B, (int)M, (int)K, gamma, eps, H, Xq, s_x,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
+int bitnet_glu_hadamard_quant_act(const float* gate, const float* up, int64_t M, int64_t K, const float* gamma,
+                                  float eps, int had_block, uint8_t* Xq4, float* s_x, void* stream) {
+  if (M < 0 || M > (int64_t(1) << 30) || K < 128 || K > 16384 || K % 128 != 0) return BITNET_ERR_SHAPE;
+  int64_t b = had_block;
+  if (b == 0) b = K & (-K);                    // the largest power of two dividing K
+  if (b < 32 || b > 8192 || (b & (b - 1)) != 0 || K % b != 0) return BITNET_ERR_SHAPE;
+  if (M == 0) return BITNET_OK;
+  if (!gate || !up || !Xq4 || !s_x) return BITNET_ERR_NULL;
+  if (!aligned16(gate) || !aligned16(up) || !aligned16(Xq4) || (gamma && !aligned16(gamma)) ||
+      (reinterpret_cast<uintptr_t>(s_x) & 3u))
+    return BITNET_ERR_ALIGN;
+  int d = check_device();
+  if (d != BITNET_OK) return d;
+  int L = 0;
+  while ((int64_t(1) << L) < b) ++L;
+  return cuda_status(bitnet::run_glu_hadamard_quant_i4(gate, up, (int)M, (int)K, L, gamma, eps, Xq4, s_x,
+                                                       static_cast<cudaStream_t>(stream)));
+}
+
 int bitnet_hadamard_quant_act(const void* X, int x_dtype, int64_t M, int64_t K, const float* gamma, float eps,
                               int had_block, uint8_t* Xq4, float* s_x, float* T_dbg, void* stream) {
   if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
@@ -184,7 +221,7 @@ int bitnet_bitlinear(const void* X, int x_dtype, int64_t M, int64_t K, const flo
   if (!bitnet::tensor_map_encoder_available()) return BITNET_ERR_UNSUPPORTED;
   const int path = linear_path();
   if (path == 3 && !bitnet::decode_path_applies((int)M, (int)K)) return BITNET_ERR_SHAPE;
-  if (path == 4 && !bitnet::fused_path_applies((int)M, (int)K, x_dtype == BITNET_BF16)) return BITNET_ERR_SHAPE;
+  if (path == 4 && !bitnet::fused_path_applies((int)M, (int)N, (int)K, x_dtype == BITNET_BF16)) return BITNET_ERR_SHAPE;
   return cuda_status(bitnet::run_bitlinear(X, x_dtype == BITNET_BF16, (int)M, (int)K, gamma, eps, pkW, s_w, (int)N,
                                            Y, y_dtype == BITNET_BF16, Xq, s_x, path,
                                            static_cast<cudaStream_t>(stream)));

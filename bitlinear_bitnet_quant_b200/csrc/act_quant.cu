@@ -19,16 +19,37 @@
 
 namespace bitnet {
 
+// Element-wise prologues of the stacked layer, applied to each fp32 input
+// chunk before the quantiser sees it (bit-identical to running bitnet_add or
+// bitnet_relu2_glu first):
+//   PRE_ADD: x = a + b, and x is written out (the residual stream);
+//   PRE_GLU: x = (r * r) * up with r = max(gate, 0).
+enum Prologue : int { PRE_NONE = 0, PRE_ADD = 1, PRE_GLU = 2 };
+
+template <int PRE, typename TIn, int E>
+BN_DEV void load_chunk(const TIn* x, const float* b, float* h, float (&v)[E]) {
+  InVec<TIn>::load(x, v);
+  if constexpr (PRE == PRE_ADD || PRE == PRE_GLU) {
+    static_assert(sizeof(TIn) == 4, "prologues take fp32 inputs");
+    float u[E];
+    InVec<float>::load(b, u);
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] = PRE == PRE_ADD ? __fadd_rn(v[e], u[e]) : relu2_times(v[e], u[e]);
+    if constexpr (PRE == PRE_ADD)
+      *reinterpret_cast<float4*>(h) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // RMSNorm + int8: one CTA of NT threads per token.  Chunk j (16 bytes of
 // input: E elements) goes to thread j % NT in iteration j / NT, so the loads
 // are coalesced; the pairwise tree is then: E elements inside a chunk, the
 // NT threads (warp xor-shuffles, then warps in order), the IT iterations.
 // ---------------------------------------------------------------------------
-template <typename TIn, int NT, int IT>
+template <typename TIn, int NT, int IT, int PRE>
 __global__ void __launch_bounds__(NT)
-quant_act_i8_kernel(const TIn* __restrict__ X, int K, const float* __restrict__ gamma, float eps,
-                    int8_t* __restrict__ Xq, float* __restrict__ s_x) {
+quant_act_i8_kernel(const TIn* __restrict__ X, const float* __restrict__ B, float* __restrict__ H, int K,
+                    const float* __restrict__ gamma, float eps, int8_t* __restrict__ Xq, float* __restrict__ s_x) {
   constexpr int E = InVec<TIn>::E;
   constexpr int NW = NT / 32;
   __shared__ float red[IT][NW];
@@ -46,7 +67,8 @@ quant_act_i8_kernel(const TIn* __restrict__ X, int K, const float* __restrict__ 
   for (int it = 0; it < IT; ++it) {
     const int j = it * NT + tid;
     if (j < C) {
-      InVec<TIn>::load(xrow + (size_t)j * E, v[it]);
+      const size_t off = (size_t)m * K + (size_t)j * E;
+      load_chunk<PRE, TIn, E>(xrow + (size_t)j * E, B + off, H + off, v[it]);
     } else {
 #pragma unroll
       for (int e = 0; e < E; ++e) v[it][e] = 0.f;
@@ -184,9 +206,9 @@ BN_DEV uint32_t nib(float t, float s) {
   return (uint32_t)(c & 0xF);
 }
 
-template <typename TIn, int L>
+template <typename TIn, int L, int PRE>
 __global__ void __launch_bounds__(128, 3)
-hadamard_quant_i4_kernel(const TIn* __restrict__ X, int M, int K, int GP,
+hadamard_quant_i4_kernel(const TIn* __restrict__ X, const float* __restrict__ B, int M, int K, int GP,
                          const float* __restrict__ gamma, float eps, float cb,
                          uint8_t* __restrict__ Xq4, float* __restrict__ s_x,
                          float* __restrict__ T_dbg) {
@@ -207,12 +229,13 @@ hadamard_quant_i4_kernel(const TIn* __restrict__ X, int M, int K, int GP,
 
   float v[HT_R];
   if (active) {
-    const TIn* src = X + (size_t)m * K + (size_t)t * HT_R;
+    const size_t off = (size_t)m * K + (size_t)t * HT_R;
+    const TIn* src = X + off;
     constexpr int E = InVec<TIn>::E;
 #pragma unroll
     for (int q = 0; q < HT_R / E; ++q) {
       float tmp[E];
-      InVec<TIn>::load(src + q * E, tmp);
+      load_chunk<PRE, TIn, E>(src + q * E, B + off + q * E, nullptr, tmp);
 #pragma unroll
       for (int e = 0; e < E; ++e) v[q * E + e] = tmp[e];
     }
@@ -348,43 +371,50 @@ hadamard_quant_i4_kernel(const TIn* __restrict__ X, int M, int K, int GP,
 // ---------------------------------------------------------------------------
 // host launchers (called from abi.cu after validation)
 // ---------------------------------------------------------------------------
-template <typename TIn, int NT, int IT>
-static cudaError_t launch_q8(const void* X, int M, int K, const float* gamma, float eps,
+template <typename TIn, int NT, int IT, int PRE>
+static cudaError_t launch_q8(const void* X, const float* B, float* H, int M, int K, const float* gamma, float eps,
                              int8_t* Xq, float* s_x, cudaStream_t st) {
-  return launch_pdl(quant_act_i8_kernel<TIn, NT, IT>, dim3(M), dim3(NT), 0, st, 1u,
-                    static_cast<const TIn*>(X), K, gamma, eps, Xq, s_x);
+  return launch_pdl(quant_act_i8_kernel<TIn, NT, IT, PRE>, dim3(M), dim3(NT), 0, st, 1u,
+                    static_cast<const TIn*>(X), B, H, K, gamma, eps, Xq, s_x);
 }
 
-template <typename TIn>
-static cudaError_t dispatch_q8(const void* X, int M, int K, const float* gamma, float eps,
+template <typename TIn, int PRE>
+static cudaError_t dispatch_q8(const void* X, const float* B, float* H, int M, int K, const float* gamma, float eps,
                                int8_t* Xq, float* s_x, cudaStream_t st) {
   constexpr int E = InVec<TIn>::E;
   int C = K / E, PC = 1;
   while (PC < C) PC <<= 1;
+#define BN_Q8(NT, IT) launch_q8<TIn, NT, IT, PRE>(X, B, H, M, K, gamma, eps, Xq, s_x, st)
   if (PC <= 1024) {
     switch (PC <= 128 ? 1 : PC / 128) {
-      case 1: return launch_q8<TIn, 128, 1>(X, M, K, gamma, eps, Xq, s_x, st);
-      case 2: return launch_q8<TIn, 128, 2>(X, M, K, gamma, eps, Xq, s_x, st);
-      case 4: return launch_q8<TIn, 128, 4>(X, M, K, gamma, eps, Xq, s_x, st);
-      case 8: return launch_q8<TIn, 128, 8>(X, M, K, gamma, eps, Xq, s_x, st);
+      case 1: return BN_Q8(128, 1);
+      case 2: return BN_Q8(128, 2);
+      case 4: return BN_Q8(128, 4);
+      case 8: return BN_Q8(128, 8);
     }
   } else {
     switch (PC / 256) {
-      case 8: return launch_q8<TIn, 256, 8>(X, M, K, gamma, eps, Xq, s_x, st);
-      case 16: return launch_q8<TIn, 256, 16>(X, M, K, gamma, eps, Xq, s_x, st);
+      case 8: return BN_Q8(256, 8);
+      case 16: return BN_Q8(256, 16);
     }
   }
+#undef BN_Q8
   return cudaErrorInvalidValue;
 }
 
 cudaError_t run_quant_act_i8(const void* X, int bf16, int M, int K, const float* gamma, float eps,
                              int8_t* Xq, float* s_x, cudaStream_t st) {
-  return bf16 ? dispatch_q8<uint16_t>(X, M, K, gamma, eps, Xq, s_x, st)
-              : dispatch_q8<float>(X, M, K, gamma, eps, Xq, s_x, st);
+  return bf16 ? dispatch_q8<uint16_t, PRE_NONE>(X, nullptr, nullptr, M, K, gamma, eps, Xq, s_x, st)
+              : dispatch_q8<float, PRE_NONE>(X, nullptr, nullptr, M, K, gamma, eps, Xq, s_x, st);
 }
 
-template <typename TIn, int L>
-static cudaError_t launch_h4(const void* X, int M, int K, const float* gamma, float eps,
+cudaError_t run_add_quant_act_i8(const float* A, const float* B, int M, int K, const float* gamma, float eps,
+                                 float* H, int8_t* Xq, float* s_x, cudaStream_t st) {
+  return dispatch_q8<float, PRE_ADD>(A, B, H, M, K, gamma, eps, Xq, s_x, st);
+}
+
+template <typename TIn, int L, int PRE>
+static cudaError_t launch_h4(const void* X, const float* B, int M, int K, const float* gamma, float eps,
                              uint8_t* Xq4, float* s_x, float* T_dbg, cudaStream_t st) {
   const int G = K / HT_R;
   int GP = 1;
@@ -392,36 +422,43 @@ static cudaError_t launch_h4(const void* X, int M, int K, const float* gamma, fl
   const int TPB = GP >= 128 ? 1 : 128 / GP;
   const int threads = TPB * GP;
   const size_t smem = (size_t)TPB * ((K + 2 * (K >> 7) + 3) & ~3) * sizeof(float) + (size_t)TPB * 4 * sizeof(float);
-  auto kern = hadamard_quant_i4_kernel<TIn, L>;
+  auto kern = hadamard_quant_i4_kernel<TIn, L, PRE>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const float cb = (float)(1.0 / sqrt((double)(1 << L)));
   const int grid = (M + TPB - 1) / TPB;
-  return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, 1u, static_cast<const TIn*>(X), M, K, GP, gamma,
+  return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, 1u, static_cast<const TIn*>(X), B, M, K, GP, gamma,
                     eps, cb, Xq4, s_x, T_dbg);
 }
 
-template <typename TIn>
-static cudaError_t dispatch_h4(const void* X, int M, int K, int L, const float* gamma, float eps,
+template <typename TIn, int PRE>
+static cudaError_t dispatch_h4(const void* X, const float* B, int M, int K, int L, const float* gamma, float eps,
                                uint8_t* Xq4, float* s_x, float* T_dbg, cudaStream_t st) {
+#define BN_H4(LL) launch_h4<TIn, LL, PRE>(X, B, M, K, gamma, eps, Xq4, s_x, T_dbg, st)
   switch (L) {
-    case 5: return launch_h4<TIn, 5>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
-    case 6: return launch_h4<TIn, 6>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
-    case 7: return launch_h4<TIn, 7>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
-    case 8: return launch_h4<TIn, 8>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
-    case 9: return launch_h4<TIn, 9>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
-    case 10: return launch_h4<TIn, 10>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
-    case 11: return launch_h4<TIn, 11>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
-    case 12: return launch_h4<TIn, 12>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
-    case 13: return launch_h4<TIn, 13>(X, M, K, gamma, eps, Xq4, s_x, T_dbg, st);
+    case 5: return BN_H4(5);
+    case 6: return BN_H4(6);
+    case 7: return BN_H4(7);
+    case 8: return BN_H4(8);
+    case 9: return BN_H4(9);
+    case 10: return BN_H4(10);
+    case 11: return BN_H4(11);
+    case 12: return BN_H4(12);
+    case 13: return BN_H4(13);
   }
+#undef BN_H4
   return cudaErrorInvalidValue;
 }
 
 cudaError_t run_hadamard_quant_i4(const void* X, int bf16, int M, int K, int L, const float* gamma,
                                   float eps, uint8_t* Xq4, float* s_x, float* T_dbg, cudaStream_t st) {
-  return bf16 ? dispatch_h4<uint16_t>(X, M, K, L, gamma, eps, Xq4, s_x, T_dbg, st)
-              : dispatch_h4<float>(X, M, K, L, gamma, eps, Xq4, s_x, T_dbg, st);
+  return bf16 ? dispatch_h4<uint16_t, PRE_NONE>(X, nullptr, M, K, L, gamma, eps, Xq4, s_x, T_dbg, st)
+              : dispatch_h4<float, PRE_NONE>(X, nullptr, M, K, L, gamma, eps, Xq4, s_x, T_dbg, st);
+}
+
+cudaError_t run_glu_hadamard_quant_i4(const float* gate, const float* up, int M, int K, int L, const float* gamma,
+                                      float eps, uint8_t* Xq4, float* s_x, cudaStream_t st) {
+  return dispatch_h4<float, PRE_GLU>(gate, up, M, K, L, gamma, eps, Xq4, s_x, nullptr, st);
 }
 
 }  // namespace bitnet

@@ -333,17 +333,26 @@ static int fused_rg(int M, int N, int K) {
 }
 
 // True when one fused kernel covers the shape (else two kernels run).
-// (largest row-group count of each token-group count: an upper bound of the
-// shared memory any of its kernels takes)
-bool fused_path_applies(int M, int K, int x_bf16) {
-  if (M < 1 || M > DEC_MAX_TOKENS || K % 512 != 0 || K > 8192) return false;
+// Shared memory of the launch that would run (its row-group count), and the
+// register budget of the quantising groups.
+bool fused_path_applies(int M, int N, int K, int x_bf16) {
+  if (M < 1 || M > DEC_MAX_TOKENS || N < 1 || K % 512 != 0 || K > 8192) return false;
   // every thread of a token's group holds at most FUSE_QIT chunks
   const int C = K / (x_bf16 ? 8 : 4);
   int PC = 1;
   while (PC < C) PC <<= 1;
   if (PC > FUSE_QIT * 32 * fused_wpt(M)) return false;
-  const size_t smem = M <= 8 ? fused_smem_bytes<1, 4>(M, K) : M <= 16 ? fused_smem_bytes<2, 4>(M, K)
-                                                                       : fused_smem_bytes<4, 2>(M, K);
+  const int rg = fused_rg(M, N, K);
+  size_t smem;
+  if (M <= 8) {
+    smem = rg == 1 ? fused_smem_bytes<1, 1>(M, K) : rg == 2 ? fused_smem_bytes<1, 2>(M, K)
+         : rg == 3 ? fused_smem_bytes<1, 3>(M, K) : fused_smem_bytes<1, 4>(M, K);
+  } else if (M <= 16) {
+    smem = rg == 1 ? fused_smem_bytes<2, 1>(M, K) : rg == 2 ? fused_smem_bytes<2, 2>(M, K)
+         : rg == 3 ? fused_smem_bytes<2, 3>(M, K) : fused_smem_bytes<2, 4>(M, K);
+  } else {
+    smem = rg == 1 ? fused_smem_bytes<4, 1>(M, K) : fused_smem_bytes<4, 2>(M, K);
+  }
   return smem <= FUSE_SMEM_MAX;
 }
 

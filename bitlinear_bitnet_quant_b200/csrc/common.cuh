@@ -70,6 +70,12 @@ BN_DEV float ldg_f32(const float* p) {
   return r;
 }
 
+// Squared-ReLU gated unit, fp32 round-to-nearest: (r * r) * u, r = max(g, 0).
+BN_DEV float relu2_times(float g, float u) {
+  const float r = fmaxf(g, 0.0f);
+  return __fmul_rn(__fmul_rn(r, r), u);
+}
+
 BN_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

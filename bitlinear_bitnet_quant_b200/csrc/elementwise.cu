@@ -21,11 +21,6 @@ add_f32_kernel(const float4* __restrict__ a, const float4* __restrict__ b, float
   }
 }
 
-BN_DEV float relu2_times(float g, float u) {
-  const float r = fmaxf(g, 0.0f);
-  return __fmul_rn(__fmul_rn(r, r), u);
-}
-
 __global__ void __launch_bounds__(256)
 relu2_glu_kernel(const float4* __restrict__ gate, const float4* __restrict__ up, float4* __restrict__ out,
                  size_t n4) {

@@ -146,6 +146,24 @@ BITNET_API int bitnet_hadamard_quant_act(const void* X, int x_dtype, int64_t M, 
                               uint8_t* Xq4, float* s_x, float* T_dbg, void* stream);
 
 /*
+ * The quantisers with the stacked layer's element-wise producer folded in
+ * (one kernel instead of two; results bit-identical to calling bitnet_add or
+ * bitnet_relu2_glu first) [P2 주요 아키텍처 혁신: squared ReLU; residuals]:
+ * bitnet_add_quant_act:          H = A + B (fp32, written out), then
+ *                                bitnet_quant_act of H (fp32 input).
+ * bitnet_glu_hadamard_quant_act: x = (r * r) * up with r = max(gate, 0),
+ *                                then bitnet_hadamard_quant_act of x
+ *                                (fp32 input; x is not written out).
+ * A, B, H, gate, up: [M][K] fp32, 16-byte aligned.  Other arguments and
+ * limits as for the plain quantisers.
+ */
+BITNET_API int bitnet_add_quant_act(const float* A, const float* B, int64_t M, int64_t K, const float* gamma,
+                         float eps, float* H, int8_t* Xq, float* s_x, void* stream);
+BITNET_API int bitnet_glu_hadamard_quant_act(const float* gate, const float* up, int64_t M, int64_t K,
+                                  const float* gamma, float eps, int had_block, uint8_t* Xq4, float* s_x,
+                                  void* stream);
+
+/*
  * Ternary x int8 (act_bits = 8) or ternary x int4 (act_bits = 4) product with
  * int32 accumulation and dequantisation [P4 계산 패러다임, 추론 최적화 및
  * 커스텀 커널, 양자화 메커니즘 ("rescaled"); P5 (divide by the factor)]:

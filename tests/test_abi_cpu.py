@@ -109,6 +109,20 @@ def test_bitlinear_validation(L):
     assert b(s_x=ALIGNED + 2) == 3
 
 
+def test_fused_quantiser_validation(L):
+    aq = lambda **kw: L.bitnet_add_quant_act(kw.get("A", ALIGNED), kw.get("B", ALIGNED), kw.get("M", 4),
+                                             kw.get("K", 256), None, 1e-6, kw.get("H", ALIGNED), ALIGNED, ALIGNED,
+                                             None)
+    assert aq(K=24) == 2 and aq(M=-1) == 2 and aq(M=0) == 0
+    assert aq(B=None) == 1 and aq(H=None) == 1
+    assert aq(A=MISALIGNED) == 3 and aq(H=MISALIGNED) == 3
+    gh = lambda **kw: L.bitnet_glu_hadamard_quant_act(kw.get("g", ALIGNED), kw.get("u", ALIGNED), kw.get("M", 4),
+                                                      kw.get("K", 1024), None, 1e-6, kw.get("b", 0), ALIGNED,
+                                                      ALIGNED, None)
+    assert gh(K=1000) == 2 and gh(b=48) == 2 and gh(K=16384, b=0) == 2 and gh(M=0) == 0
+    assert gh(u=None) == 1 and gh(g=MISALIGNED) == 3
+
+
 def test_linear_path_selector(L):
     assert L.bitnet_set_linear_path(5) == 2
     assert L.bitnet_set_linear_path(4) == 0

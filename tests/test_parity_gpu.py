@@ -295,7 +295,7 @@ def _check_bitlinear(M, N, K, dtype, use_gamma, out, path=0, seed=0):
     (1, 6912, 2560, "bf16", False, "f32"), (4, 6912, 2560, "bf16", False, "f32"),
     (16, 6912, 2560, "bf16", False, "bf16"), (3, 200, 512, "f32", True, "f32"), (8, 1000, 1536, "bf16", True, "f32"),
     (9, 2048, 2048, "f32", False, "f32"), (17, 5632, 2048, "f32", True, "f32"), (32, 2048, 2048, "f32", False, "bf16"),
-    (32, 300, 4096, "bf16", False, "f32"), (16, 300, 8192, "bf16", False, "f32"), (12, 16, 4608, "f32", False, "f32"),
+    (32, 300, 4096, "bf16", False, "f32"), (16, 300, 8192, "bf16", False, "f32"), (12, 16, 4608, "bf16", False, "f32"),
     (1, 1, 512, "bf16", False, "f32")])
 def test_bitlinear_fused(M, N, K, dtype, use_gamma, out):
     """One kernel: clusters of 8 CTAs quantise every eighth token each and
@@ -390,6 +390,36 @@ def test_chain_two_layers(M, rows):
     for lw in ora_w:
         ref = O.chain_layer(ref, lw)
     assert np.array_equal(out[sel].view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("M,K,use_gamma", [(3, 2048, False), (32, 2048, True), (5, 16, False), (17, 5632, False),
+                                             (2, 16384, True)])
+def test_add_quant_act(M, K, use_gamma):
+    """Residual add folded into the int8 quantiser: H, codes and scales equal
+    bitnet_add followed by bitnet_quant_act, bit for bit."""
+    rng = np.random.default_rng(M * 3 + K)
+    a = wl.gaussian(rng, (M, K))
+    b = wl.gaussian(rng, (M, K), 0.5)
+    gamma = rng.uniform(0.5, 1.5, K).astype(np.float32) if use_gamma else None
+    H, q, s = api.bitnet_add_quant_act(dev(a), dev(b), dev(gamma) if use_gamma else None, 1e-6)
+    h_o = a + b
+    q_o, s_o = O.quant_act(h_o, gamma, 1e-6)
+    assert np.array_equal(host(H).view(np.uint32), h_o.view(np.uint32))
+    assert np.array_equal(host(s).view(np.uint32), s_o.view(np.uint32))
+    assert np.array_equal(host(q), q_o)
+
+
+@pytest.mark.parametrize("M,K,b", [(3, 5632, 0), (32, 5632, 0), (4, 2048, 0), (7, 8192, 1024), (2, 1024, 32)])
+def test_glu_hadamard_quant_act(M, K, b):
+    """Squared-ReLU gated unit folded into the Hadamard int4 quantiser: codes
+    and scales equal bitnet_relu2_glu followed by bitnet_hadamard_quant_act."""
+    rng = np.random.default_rng(M * 5 + K)
+    gate = wl.gaussian(rng, (M, K))
+    up = wl.gaussian(rng, (M, K))
+    q4, s = api.bitnet_glu_hadamard_quant_act(dev(gate), dev(up), None, 1e-6, b)
+    pk_o, s_o, _, _ = O.hadamard_quant_act(O.squared_relu_glu(gate, up), None, 1e-6, b)
+    assert np.array_equal(host(s).view(np.uint32), s_o.view(np.uint32))
+    assert np.array_equal(host(q4), pk_o)
 
 
 def test_elementwise_glue():
