@@ -369,6 +369,131 @@ hadamard_quant_i4_kernel(const TIn* __restrict__ X, const float* __restrict__ B,
 }
 
 // ---------------------------------------------------------------------------
+// RMSNorm + Hadamard + int4 for a few tokens: one CTA of 256 threads per token.
+// The sum of squares uses the fixed tree (E elements of a chunk, 32 lanes, the
+// 8 warps in order, then the iterations, padded with zero subtrees); the
+// normalised row is kept in shared memory and each radix-2 stage (stride 1, 2,
+// ..., b/2, pairs (a, c) -> (a + c, a - c)) runs over it between barriers, so
+// every value is the one the register kernel produces.
+// ---------------------------------------------------------------------------
+constexpr int HR_THREADS = 256;
+constexpr int HR_MAX_IT = 16;                        // K <= 16384 (fp32: 4 elements per chunk)
+
+template <typename TIn, int L, int PRE>
+__global__ void __launch_bounds__(HR_THREADS)
+hadamard_quant_i4_row_kernel(const TIn* __restrict__ X, const float* __restrict__ B, int K,
+                             const float* __restrict__ gamma, float eps, float cb, uint8_t* __restrict__ Xq4,
+                             float* __restrict__ s_x, float* __restrict__ T_dbg) {
+  constexpr int E = InVec<TIn>::E, NW = HR_THREADS / 32;
+  extern __shared__ float hrow[];                    // K floats
+  __shared__ float red[HR_MAX_IT][NW];
+  __shared__ float bcast[2];
+  pdl_launch_dependents();
+  pdl_wait();                                        // X may come from, and Xq4 may still be read by, the previous kernel
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int m = blockIdx.x;
+  const int C = K / E;
+  int P = 1;
+  while (P < C) P <<= 1;
+  const int IT = P > HR_THREADS ? P / HR_THREADS : 1;  // iterations covering the padded row
+
+  // ---- load (with the prologue), squares by the fixed tree ----
+  for (int it = 0; it < IT; ++it) {
+    const int j = it * HR_THREADS + tid;
+    float v[E];
+    if (j < C) {
+      const size_t off = (size_t)m * K + (size_t)j * E;
+      load_chunk<PRE, TIn, E>(X + off, B + off, nullptr, v);
+#pragma unroll
+      for (int q = 0; q < E; q += 4)
+        *reinterpret_cast<float4*>(hrow + (size_t)j * E + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[e] = 0.f;
+    }
+    float sq[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) sq[e] = __fmul_rn(v[e], v[e]);
+    const float w = warp_tree_sum(tree_sum<E>(sq));
+    if (lane == 0) red[it][warp] = w;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float cs[HR_MAX_IT];
+#pragma unroll
+    for (int it = 0; it < HR_MAX_IT; ++it) {
+      cs[it] = 0.f;                                  // past the padded row: zero subtrees, exact
+      if (it < IT) {
+        float p[NW];
+#pragma unroll
+        for (int w = 0; w < NW; ++w) p[w] = red[it][w];
+        cs[it] = tree_sum<NW>(p);
+      }
+    }
+    const float ss = tree_sum<HR_MAX_IT>(cs);
+    bcast[0] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)K), eps)));
+  }
+  __syncthreads();
+  const float r = bcast[0];
+  for (int i = tid; i < K; i += HR_THREADS)
+    hrow[i] = gamma != nullptr ? __fmul_rn(__fmul_rn(hrow[i], r), __ldg(gamma + i)) : __fmul_rn(hrow[i], r);
+  __syncthreads();
+
+  // ---- radix-2 stages over the row (blocks of 2^L; pairs never cross a block) ----
+#pragma unroll 1
+  for (int st = 0; st < L; ++st) {
+    const int h = 1 << st;
+    for (int q = tid; q < K / 2; q += HR_THREADS) {
+      const int i = ((q >> st) << (st + 1)) | (q & (h - 1));
+      const float a = hrow[i], c = hrow[i + h];
+      hrow[i] = __fadd_rn(a, c);
+      hrow[i + h] = __fsub_rn(a, c);
+    }
+    __syncthreads();
+  }
+
+  // ---- normalise, absmax ----
+  float amax = 0.f;
+  for (int i = tid; i < K; i += HR_THREADS) {
+    const float tv = __fmul_rn(hrow[i], cb);
+    hrow[i] = tv;
+    amax = fmaxf(amax, fabsf(tv));
+  }
+  amax = warp_max(amax);
+  if (lane == 0) red[0][warp] = amax;
+  __syncthreads();
+  if (tid == 0) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) a = fmaxf(a, red[0][w]);
+    bcast[1] = __fdiv_rn(7.0f, fmaxf(a, 1e-5f));
+  }
+  __syncthreads();
+  const float s = bcast[1];
+
+  // ---- codes: 32 elements (16 bytes) per step, two per byte ----
+  for (int c32 = tid; c32 < K / 32; c32 += HR_THREADS) {
+    const float* src = hrow + 32 * c32;
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) word |= nib(src[8 * q + e], s) << (4 * e);
+      w[q] = word;
+    }
+    *reinterpret_cast<uint4*>(Xq4 + (size_t)m * (K / 2) + 16 * (size_t)c32) = make_uint4(w[0], w[1], w[2], w[3]);
+    if (T_dbg != nullptr) {
+#pragma unroll
+      for (int q = 0; q < 32; q += 4)
+        *reinterpret_cast<float4*>(T_dbg + (size_t)m * K + 32 * (size_t)c32 + q) =
+            make_float4(src[q], src[q + 1], src[q + 2], src[q + 3]);
+    }
+  }
+  if (tid == 0) s_x[m] = s;
+}
+
+// ---------------------------------------------------------------------------
 // host launchers (called from abi.cu after validation)
 // ---------------------------------------------------------------------------
 template <typename TIn, int NT, int IT, int PRE>
@@ -421,11 +546,23 @@ static cudaError_t launch_h4(const void* X, const float* B, int M, int K, const 
   while (GP < G) GP <<= 1;
   const int TPB = GP >= 128 ? 1 : 128 / GP;
   const int threads = TPB * GP;
+  const float cb = (float)(1.0 / sqrt((double)(1 << L)));
+  // Few tokens: the register kernel would leave most SMs idle; one CTA per token instead.
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if ((M + TPB - 1) / TPB < 2 * sms) {
+    auto rk = hadamard_quant_i4_row_kernel<TIn, L, PRE>;
+    const size_t rsmem = (size_t)K * sizeof(float);
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(rk), rsmem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(rk, dim3(M), dim3(HR_THREADS), rsmem, st, 1u, static_cast<const TIn*>(X), B, K, gamma, eps, cb,
+                      Xq4, s_x, T_dbg);
+  }
   const size_t smem = (size_t)TPB * ((K + 2 * (K >> 7) + 3) & ~3) * sizeof(float) + (size_t)TPB * 4 * sizeof(float);
   auto kern = hadamard_quant_i4_kernel<TIn, L, PRE>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  const float cb = (float)(1.0 / sqrt((double)(1 << L)));
   const int grid = (M + TPB - 1) / TPB;
   return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, 1u, static_cast<const TIn*>(X), B, M, K, GP, gamma,
                     eps, cb, Xq4, s_x, T_dbg);

@@ -159,6 +159,14 @@ def test_hadamard_quant(M, K, b, dtype):
     _check_hadamard(x, dtype, b)
 
 
+@pytest.mark.parametrize("M,K,b,dtype", [(2400, 2048, 0, "bf16"), (700, 5632, 0, "f32"), (4800, 256, 32, "f32")])
+def test_hadamard_quant_many_tokens(M, K, b, dtype):
+    """Enough tokens for the register kernel (few tokens take the one-CTA-per-
+    token kernel): both must give the same bits as the oracle."""
+    x = wl.student_t(np.random.default_rng(M + K), (M, K))
+    _check_hadamard(x, dtype, b)
+
+
 def test_hadamard_gamma_and_edges():
     rng = np.random.default_rng(3)
     x = rng.standard_normal((6, 1024)).astype(np.float32)
