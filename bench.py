@@ -291,7 +291,7 @@ def run_ours(args, rank, world, local_rank):
         x.copy_(x_pin, non_blocking=True)
         pk, s_w = ring[i % copies]
         Yo = api.bitlinear_forward(x, pk, s_w, act_bits=bits, eps=eps, had_block=c.get("had_block", 0),
-                                   out_dtype=out_dtype, stream=stream)
+                                   out_dtype=out_dtype, Y=Y, Xq=xq, s_x=s_x, stream=stream)
         y_pin.copy_(Yo, non_blocking=True)
 
     for i in range(warmup):

@@ -261,13 +261,15 @@ def bitnet_device_error() -> int:
 
 
 def bitlinear_forward(X: torch.Tensor, pkW: torch.Tensor, s_w: torch.Tensor, act_bits: int = 8, gamma=None,
-                      eps: float = 1e-6, had_block: int = 0, out_dtype=torch.float32, stream=None):
-    """One BitLinear forward: quantise the activations, then the ternary product
-    (int8: the fused entry point, one kernel for a few tokens)."""
+                      eps: float = 1e-6, had_block: int = 0, out_dtype=torch.float32, Y=None, Xq=None, s_x=None,
+                      stream=None):
+    """One BitLinear forward: quantise the activations, then the ternary
+    product.  Y, Xq and s_x may be passed in to reuse buffers across calls
+    (Xq: [M, K] int8 for act_bits 8, [M, K/2] uint8 packed int4 for 4)."""
     if act_bits == 8:
-        Y, _, _ = bitnet_bitlinear(X, pkW, s_w, gamma, eps, out_dtype=out_dtype, stream=stream)
+        Y, _, _ = bitnet_bitlinear(X, pkW, s_w, gamma, eps, out_dtype=out_dtype, Y=Y, Xq=Xq, s_x=s_x,
+                                   stream=stream)
         return Y
-    else:
-        Xq, s_x, _ = bitnet_hadamard_quant_act(X, gamma, eps, had_block, stream=stream)
-    Y, _ = bitnet_linear(Xq, act_bits, s_x, pkW, s_w, out_dtype=out_dtype, stream=stream)
+    Xq, s_x, _ = bitnet_hadamard_quant_act(X, gamma, eps, had_block, Xq4=Xq, s_x=s_x, stream=stream)
+    Y, _ = bitnet_linear(Xq, act_bits, s_x, pkW, s_w, out_dtype=out_dtype, Y=Y, stream=stream)
     return Y
