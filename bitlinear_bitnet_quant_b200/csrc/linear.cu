@@ -316,7 +316,10 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       if (!mbar_wait_warp(&bar_wfull[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
       tc_fence_after();
       // 64 weights of this row -> 16 tensor-memory columns
-      const uint4 w = *reinterpret_cast<const uint4*>(ws(s) + 32 * row + 16 * h);
+      // the tile arrives with the 32-byte swizzle: the two 16-byte halves of
+      // row r are swapped when bit 2 of r is set, so the eight rows a
+      // quarter-warp reads fall on distinct banks
+      const uint4 w = *reinterpret_cast<const uint4*>(ws(s) + 32 * row + 16 * (h ^ ((row >> 2) & 1)));
       if constexpr (ACT_BITS == 8) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_empty[s]);   // packed tile consumed
@@ -492,7 +495,7 @@ static cudaError_t launch_tc(const void* Xq, const float* s_x, const uint8_t* pk
                              int M, int N, int K, void* Y, int32_t* acc_dbg, cudaStream_t st) {
   using C = TcCfg<BN, ACT_BITS>;
   CUtensorMap tmW, tmX, tmY;
-  if (!make_map_bytes(&tmW, pkW, (uint64_t)K / 4, (uint64_t)N, TC_BK / 4, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (!make_map_bytes(&tmW, pkW, (uint64_t)K / 4, (uint64_t)N, TC_BK / 4, 128, CU_TENSOR_MAP_SWIZZLE_32B))
     return cudaErrorInvalidValue;
   const bool ok = ACT_BITS == 8
       ? make_map_bytes(&tmX, Xq, (uint64_t)K, (uint64_t)M, TC_BK, BN, CU_TENSOR_MAP_SWIZZLE_128B)
