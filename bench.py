@@ -307,6 +307,24 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     t_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
 
+    # the offline weight path (absmean ternarisation + packing) on fp32 weights of this layer's
+    # shape, timed on its own: it is not part of a forward step
+    wq = None
+    if args.workload in ("decode", "prefill", "hbitlinear"):
+        w32 = torch.from_numpy(wl.weights(N, K, seed=rank + 7)).to(dev)
+        pk_o = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
+        sw_o = torch.empty((1,), dtype=torch.float32, device=dev)
+        ws_o = torch.empty((api.bitnet_quantize_weights_workspace_size(N, K),), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            api.bitnet_quantize_weights(w32, pkW=pk_o, s_w=sw_o, workspace=ws_o, stream=stream)
+        reps = 10
+        t_wq = timed(graph_of(lambda i: api.bitnet_quantize_weights(w32, pkW=pk_o, s_w=sw_o, workspace=ws_o,
+                                                                    stream=stream), reps)) / reps / 1e3
+        wbytes = N * K * 4 * 2 + N * K // 4 + 4          # fp32 weights read twice (mean, codes), packed written
+        wq = {"us": t_wq * 1e6, "achieved_GBs": wbytes / t_wq / 1e9, "frac": wbytes / t_wq / 1e9 /
+              load_peaks()[0]["hbm_gbs"], "algorithmic_bytes": wbytes, "weights": N * K, "input": "fp32"}
+        del w32
+
     # decode: the same weight ring at the other decode batch sizes (linear launches only)
     sweep = []
     if args.workload == "decode":
@@ -396,6 +414,8 @@ def run_ours(args, rank, world, local_rank):
     }
     if sweep:
         line["decode_sweep"] = sweep
+    if wq is not None:
+        line["weights_quant"] = wq
     return line
 
 
