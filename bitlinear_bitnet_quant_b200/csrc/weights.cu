@@ -53,16 +53,27 @@ absmean_digits_kernel(const TIn* __restrict__ W, size_t n16, uint64_t* __restric
   Digits acc;
 #pragma unroll
   for (int i = 0; i < WQ_DIGITS; ++i) acc.c[i] = 0;
+  // four independent 16-byte loads in flight per thread (integer sums: any
+  // grouping gives the same counters; padding chunks add zero)
+  constexpr int U = 4;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += stride) {
-    uint4 u = ldg_nc_v4(reinterpret_cast<const uint8_t*>(W) + 16 * i);
-    if constexpr (sizeof(TIn) == 4) {
-      digits_add(acc, u.x); digits_add(acc, u.y); digits_add(acc, u.z); digits_add(acc, u.w);
-    } else {
-      digits_add(acc, u.x << 16); digits_add(acc, u.x & 0xFFFF0000u);
-      digits_add(acc, u.y << 16); digits_add(acc, u.y & 0xFFFF0000u);
-      digits_add(acc, u.z << 16); digits_add(acc, u.z & 0xFFFF0000u);
-      digits_add(acc, u.w << 16); digits_add(acc, u.w & 0xFFFF0000u);
+  for (size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < n16; i0 += U * stride) {
+    uint4 u[U];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const size_t i = i0 + k * stride;
+      u[k] = i < n16 ? ldg_nc_v4(reinterpret_cast<const uint8_t*>(W) + 16 * i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      if constexpr (sizeof(TIn) == 4) {
+        digits_add(acc, u[k].x); digits_add(acc, u[k].y); digits_add(acc, u[k].z); digits_add(acc, u[k].w);
+      } else {
+        digits_add(acc, u[k].x << 16); digits_add(acc, u[k].x & 0xFFFF0000u);
+        digits_add(acc, u[k].y << 16); digits_add(acc, u[k].y & 0xFFFF0000u);
+        digits_add(acc, u[k].z << 16); digits_add(acc, u[k].z & 0xFFFF0000u);
+        digits_add(acc, u[k].w << 16); digits_add(acc, u[k].w & 0xFFFF0000u);
+      }
     }
   }
 #pragma unroll
