@@ -310,7 +310,6 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
     const int ct = threadIdx.x - 64;             // 0..255
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
 
-    int signalled = 0;                           // steps whose conv barrier has been arrived on
     for (int i = 0; i < nk; ++i) {
       const int s = i % S, r = i / S;
       if (!mbar_wait_warp(&bar_wfull[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
@@ -349,18 +348,13 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_empty[s]);
       }
-      // Signal the MMA issuer in bursts: wait for the tensor-memory stores once
-      // for every run of steps whose weights had already landed.
-      const int nx = i + 1;
-      const bool more = nx < nk && __all_sync(0xffffffffu, mbar_test(&bar_wfull[nx % S], (nx / S) & 1));
-      if (!more) {
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0)
-          for (int j = signalled; j <= i; ++j) mbar_arrive(&bar_conv[j % S]);
-        signalled = i + 1;
-      }
+      // Hand every step to the MMA issuer as soon as its operands are in place
+      // (measured on B200: holding steps back to batch the tensor-memory store
+      // waits cost 7 % on the int8 and 20 % on the int4 GEMM).
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_conv[s]);
     }
 
     // ------------------------------------------------------------ epilogue

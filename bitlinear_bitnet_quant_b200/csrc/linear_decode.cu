@@ -23,6 +23,10 @@
 //   two MMAs; the matching activation bytes are one 16-byte load per token.
 //   The K order inside an MMA is permuted identically on both sides, which
 //   leaves the sum unchanged.
+// * More than 8 tokens: the token groups can also be spread over adjacent
+//   CTAs that share a weight slice (the second read of the slice hits L2), so
+//   twice the warps issue MMAs on each SM and every CTA loads fewer
+//   activation bytes after the wait.
 // * Warp w takes the 64-wide K slice w of every segment; the eight partial
 //   tiles meet in shared memory and one pass sums, shifts (>> 6, or >> 10 for
 //   int4 activations held as 16*x) and dequantises:
@@ -37,11 +41,14 @@ namespace bitnet {
 // are loaded while this one's MMAs issue, and consecutive MMAs never depend on
 // each other (with one token group, the two MMAs of a 64-wide slice go to two
 // accumulator sets, summed at the end).
+//
+// `tsplit` CTAs share each weight slice: CTA b takes rows (b / tsplit) * ROWS
+// onwards and tokens 8 * TG * (b % tsplit) onwards.
 template <int ACT_BITS, int TG, int RG, typename TOut>
 __global__ void __launch_bounds__(DEC_THREADS, 2)
 linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict__ Xq,
                      const float* __restrict__ s_x, const float* __restrict__ s_w_ptr, int M, int N, int K,
-                     TOut* __restrict__ Y, int32_t* __restrict__ acc_dbg) {
+                     int tsplit, TOut* __restrict__ Y, int32_t* __restrict__ acc_dbg) {
   using C = DecCfg<TG>;
   constexpr int TOK = C::TOK, PB = C::PASS_BATCH;
   constexpr int ROWS = 16 * RG;
@@ -55,7 +62,16 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int nseg = K / 512;
-  const int n0 = blockIdx.x * ROWS;
+  const int n0 = (blockIdx.x / tsplit) * ROWS;
+  const size_t xrow = ACT_BITS == 8 ? (size_t)K : (size_t)K / 2;
+  {
+    const int m0 = (blockIdx.x % tsplit) * TOK;     // this CTA's first token
+    M = M - m0 < TOK ? M - m0 : TOK;
+    Xq += (size_t)m0 * xrow;
+    s_x += m0;
+    Y += (size_t)m0 * N;
+    if (acc_dbg) acc_dbg += (size_t)m0 * N;
+  }
 
   // This kernel holds no tensor memory, so the next kernel in the stream may
   // be scheduled at once (it only waits for this grid to finish).
@@ -78,7 +94,6 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
 #pragma unroll
         for (int j = 0; j < 4; ++j) d[h][rg][tg][j] = 0;
 
-  const size_t xrow = ACT_BITS == 8 ? (size_t)K : (size_t)K / 2;
   uint32_t wcur[RG][2];
   for (int u0 = 0; u0 < nseg; u0 += PB) {
     // activation bytes of this warp's K slices: 16 consecutive K per token and segment
@@ -138,7 +153,7 @@ bool decode_path_applies(int M, int K) {
 
 template <int ACT_BITS, int TG, int RG, typename TOut>
 static cudaError_t launch_decode_rg(const void* Xq, const float* s_x, const uint8_t* pkW, const float* s_w, int M,
-                                    int N, int K, void* Y, int32_t* acc_dbg, cudaStream_t st) {
+                                    int N, int K, int tsplit, void* Y, int32_t* acc_dbg, cudaStream_t st) {
   constexpr int ROWS = 16 * RG;
   const size_t wbytes = (size_t)ROWS * (size_t)K / 4;
   const size_t rbytes = dec_red_bytes<TG, RG>();
@@ -146,19 +161,19 @@ static cudaError_t launch_decode_rg(const void* Xq, const float* s_x, const uint
   auto kern = linear_decode_kernel<ACT_BITS, TG, RG, TOut>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)((N + ROWS - 1) / ROWS));
+  const dim3 grid((unsigned)((N + ROWS - 1) / ROWS * tsplit));
   return launch_pdl(kern, grid, dim3(DEC_THREADS), smem, st, 1u, pkW, static_cast<const uint8_t*>(Xq), s_x, s_w, M, N,
-                    K, static_cast<TOut*>(Y), acc_dbg);
+                    K, tsplit, static_cast<TOut*>(Y), acc_dbg);
 }
 
 template <int ACT_BITS, int TG, typename TOut>
 static cudaError_t launch_decode_t(const void* Xq, const float* s_x, const uint8_t* pkW, const float* s_w, int M,
-                                   int N, int K, void* Y, int32_t* acc_dbg, cudaStream_t st) {
+                                   int N, int K, int tsplit, void* Y, int32_t* acc_dbg, cudaStream_t st) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int rg = decode_rows(N, K, sms, DecCfg<TG>::MAX_ROWS) / 16;
-#define BN_RG(R) launch_decode_rg<ACT_BITS, TG, (R <= DecCfg<TG>::RG_MAX ? R : 1), TOut>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st)
+#define BN_RG(R) launch_decode_rg<ACT_BITS, TG, (R <= DecCfg<TG>::RG_MAX ? R : 1), TOut>(Xq, s_x, pkW, s_w, M, N, K, tsplit, Y, acc_dbg, st)
   switch (rg) {
     case 1: return BN_RG(1);
     case 2: return BN_RG(2);
@@ -170,10 +185,12 @@ static cudaError_t launch_decode_t(const void* Xq, const float* s_x, const uint8
 
 cudaError_t run_linear_decode(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                               int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, cudaStream_t st) {
-#define BN_DEC(BITS, T)                                                                           \
-  return M <= 8    ? launch_decode_t<BITS, 1, T>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st)       \
-         : M <= 16 ? launch_decode_t<BITS, 2, T>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st)       \
-                   : launch_decode_t<BITS, 4, T>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st)
+  // up to 16 tokens: one token group per CTA (two CTAs per weight slice past
+  // 8 tokens); up to 32: two token groups per CTA, two CTAs per slice
+#define BN_DEC(BITS, T)                                                                                   \
+  return M <= 8    ? launch_decode_t<BITS, 1, T>(Xq, s_x, pkW, s_w, M, N, K, 1, Y, acc_dbg, st)          \
+         : M <= 16 ? launch_decode_t<BITS, 1, T>(Xq, s_x, pkW, s_w, M, N, K, 2, Y, acc_dbg, st)          \
+                   : launch_decode_t<BITS, 2, T>(Xq, s_x, pkW, s_w, M, N, K, (M + 15) / 16, Y, acc_dbg, st)
   if (act_bits == 8) {
     if (y_bf16) { BN_DEC(8, __nv_bfloat16); } else { BN_DEC(8, float); }
   } else {
