@@ -128,7 +128,10 @@ quant_act_i8_kernel(const TIn* __restrict__ X, const float* __restrict__ B, floa
 
   const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
 
-  // ---- codes ----
+  // ---- codes: rint(y * s), clamped to [-128, 127] ----
+  // With s = 127 / max(amax, 1e-5) and |y| <= amax, |y * s| <= 127 (1 + 2^-23)
+  // after both roundings, so every code lies in [-127, 127] and the clamp never
+  // acts; the rounded products go through rint_low_bits.
   int8_t* qrow = Xq + (size_t)m * K;
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
@@ -137,14 +140,10 @@ quant_act_i8_kernel(const TIn* __restrict__ X, const float* __restrict__ B, floa
     uint32_t packed[E / 4];
 #pragma unroll
     for (int q = 0; q < E / 4; ++q) {
-      uint32_t w = 0;
+      uint32_t b[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        int c = __float2int_rn(__fmul_rn(v[it][4 * q + e], s));
-        c = max(-128, min(127, c));
-        w |= (uint32_t)(c & 0xFF) << (8 * e);
-      }
-      packed[q] = w;
+      for (int e = 0; e < 4; ++e) b[e] = rint_low_bits(__fmul_rn(v[it][4 * q + e], s));
+      packed[q] = pack_low_bytes(b[0], b[1], b[2], b[3]);
     }
     if constexpr (E == 8) {
       *reinterpret_cast<uint2*>(qrow + (size_t)j * E) = make_uint2(packed[0], packed[1]);
@@ -200,10 +199,15 @@ BN_DEV int phase2_elem(int tprime, int c) {
   return (blk << L) | within;
 }
 
-BN_DEV uint32_t nib(float t, float s) {
-  int c = __float2int_rn(__fmul_rn(t, s));
-  c = max(-8, min(7, c));
-  return (uint32_t)(c & 0xF);
+// Code of t: rint(t * s) clamped to [-8, 7], in the low nibble.  With
+// s = 7 / max(amax, 1e-5) and |t| <= amax, |t * s| <= 7 (1 + 2^-23) after both
+// roundings, so the code lies in [-7, 7] and the clamp never acts.
+BN_DEV uint32_t nib(float t, float s) { return rint_low_bits(__fmul_rn(t, s)); }
+
+// Eight codes (element 0 in the low nibble) as one word.
+BN_DEV uint32_t pack_nibbles8(const float* t, float s) {
+  return pack_low_bytes(pair_nibbles(nib(t[0], s), nib(t[1], s)), pair_nibbles(nib(t[2], s), nib(t[3], s)),
+                        pair_nibbles(nib(t[4], s), nib(t[5], s)), pair_nibbles(nib(t[6], s), nib(t[7], s)));
 }
 
 template <typename TIn, int L, int PRE>
@@ -335,12 +339,7 @@ hadamard_quant_i4_kernel(const TIn* __restrict__ X, const float* __restrict__ B,
     }
     uint32_t w[16];
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) word |= nib(v[8 * q + e], s) << (4 * e);
-      w[q] = word;
-    }
+    for (int q = 0; q < 16; ++q) w[q] = pack_nibbles8(v + 8 * q, s);
     uint4* dst = reinterpret_cast<uint4*>(Xq4 + (size_t)m * (K / 2) + (size_t)t * (HT_R / 2));
 #pragma unroll
     for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
@@ -356,7 +355,7 @@ hadamard_quant_i4_kernel(const TIn* __restrict__ X, const float* __restrict__ B,
       }
 #pragma unroll
       for (int c = 0; c < HT_R; c += 2)
-        bytes[phase2_elem<L>(t, c) >> 1] = (uint8_t)(nib(v[c], s) | (nib(v[c + 1], s) << 4));
+        bytes[phase2_elem<L>(t, c) >> 1] = (uint8_t)pair_nibbles(nib(v[c], s), nib(v[c + 1], s));
     }
     __syncthreads();
     if (m < M) {
@@ -476,12 +475,7 @@ hadamard_quant_i4_row_kernel(const TIn* __restrict__ X, const float* __restrict_
     const float* src = hrow + 32 * c32;
     uint32_t w[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) word |= nib(src[8 * q + e], s) << (4 * e);
-      w[q] = word;
-    }
+    for (int q = 0; q < 4; ++q) w[q] = pack_nibbles8(src + 8 * q, s);
     *reinterpret_cast<uint4*>(Xq4 + (size_t)m * (K / 2) + 16 * (size_t)c32) = make_uint4(w[0], w[1], w[2], w[3]);
     if (T_dbg != nullptr) {
 #pragma unroll

@@ -127,7 +127,7 @@ BN_DEV float group_quant_row_i8(const TIn* __restrict__ xrow, int K, const float
   for (int w = 0; w < WPT; ++w) amax = fmaxf(amax, red[0][w]);
   const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
 
-  // ---- codes ----
+  // ---- codes: rint(y * s); |y * s| <= 127 (1 + 2^-23), so the clamp to [-128, 127] never acts ----
 #pragma unroll
   for (int it = 0; it < FUSE_QIT; ++it) {
     const int j = it * NT + tid;
@@ -135,14 +135,10 @@ BN_DEV float group_quant_row_i8(const TIn* __restrict__ xrow, int K, const float
       uint32_t packed[E / 4];
 #pragma unroll
       for (int q = 0; q < E / 4; ++q) {
-        uint32_t w = 0;
+        uint32_t b[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          int c = __float2int_rn(__fmul_rn(v[it][4 * q + e], s));
-          c = max(-128, min(127, c));
-          w |= (uint32_t)(c & 0xFF) << (8 * e);
-        }
-        packed[q] = w;
+        for (int e = 0; e < 4; ++e) b[e] = rint_low_bits(__fmul_rn(v[it][4 * q + e], s));
+        packed[q] = pack_low_bytes(b[0], b[1], b[2], b[3]);
       }
       if constexpr (E == 8) {
         *reinterpret_cast<uint2*>(qrow + (size_t)j * E) = make_uint2(packed[0], packed[1]);

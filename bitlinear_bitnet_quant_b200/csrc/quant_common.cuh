@@ -46,4 +46,24 @@ BN_DEV float warp_tree_sum(float v) {
   return v;
 }
 
+// rint(x) for |x| < 2^22, as the low bits (two's complement) of the returned
+// word.  x + 1.5 * 2^23 lies in [2^23, 2^24), where consecutive fp32 values
+// are 1 apart, so the round-to-nearest-even addition rounds x to an integer
+// with ties to even, and the sum's mantissa holds 1.5 * 2^23 + rint(x).  One
+// full-rate fp32 add replaces a float-to-int conversion.
+BN_DEV uint32_t rint_low_bits(float x) { return __float_as_uint(__fadd_rn(x, 12582912.0f)); }
+
+// The low bytes of four rint_low_bits words, first argument in byte 0.
+BN_DEV uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Low nibble of lo in bits 0-3 and low nibble of hi in bits 4-7 (bits 8-31
+// keep lo's: only the low byte is meant).
+BN_DEV uint32_t pair_nibbles(uint32_t lo, uint32_t hi) {
+  uint32_t r;
+  asm("bfi.b32 %0, %1, %2, 4, 4;" : "=r"(r) : "r"(hi), "r"(lo));
+  return r;
+}
+
 }  // namespace bitnet
