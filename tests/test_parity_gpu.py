@@ -101,6 +101,18 @@ def test_quant_act(M, K, dtype, use_gamma):
     assert np.array_equal(host(q), q_o)
 
 
+@pytest.mark.parametrize("K,dtype", [(4096, "bf16"), (2048, "f32"), (2560, "bf16"), (96, "f32")])
+def test_quant_act_rows_independent_of_call_size(K, dtype):
+    """A token's codes and scale do not depend on the other tokens of the call."""
+    x = wl.add_entry_outliers(np.random.default_rng(K), wl.gaussian(np.random.default_rng(K + 1), (65, K)),
+                              0.005, 30.0)
+    xd, _ = x_inputs(x, dtype)
+    q_warp, s_warp = api.bitnet_quant_act(xd[:64].contiguous(), None, 1e-6)
+    q_cta, s_cta = api.bitnet_quant_act(xd, None, 1e-6)
+    assert np.array_equal(host(s_warp).view(np.uint32), host(s_cta)[:64].view(np.uint32))
+    assert np.array_equal(host(q_warp), host(q_cta)[:64])
+
+
 def test_quant_act_edge_rows():
     K = 512
     x = np.zeros((6, K), np.float32)
