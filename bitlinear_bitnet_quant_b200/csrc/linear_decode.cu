@@ -172,7 +172,11 @@ static cudaError_t launch_decode_t(const void* Xq, const float* s_x, const uint8
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int rg = decode_rows(N, K, sms, DecCfg<TG>::MAX_ROWS) / 16;
+  // one CTA per weight slice (up to 8 tokens): slices sized for two CTAs per
+  // SM, which halves each warp's MMA chain (measured on B200: 8 tokens
+  // 3.5 -> 2.9 us at N = 6912, K = 2560); with the token groups spread over
+  // CTAs the grid already holds two per SM
+  const int rg = decode_rows(N, K, sms * (tsplit == 1 ? 2 : 1), DecCfg<TG>::MAX_ROWS) / 16;
 #define BN_RG(R) launch_decode_rg<ACT_BITS, TG, (R <= DecCfg<TG>::RG_MAX ? R : 1), TOut>(Xq, s_x, pkW, s_w, M, N, K, tsplit, Y, acc_dbg, st)
   switch (rg) {
     case 1: return BN_RG(1);
