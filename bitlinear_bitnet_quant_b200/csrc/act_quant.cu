@@ -370,23 +370,72 @@ hadamard_quant_i4_kernel(const TIn* __restrict__ X, const float* __restrict__ B,
 // ---------------------------------------------------------------------------
 // RMSNorm + Hadamard + int4 for a few tokens: one CTA of 256 threads per token.
 // The sum of squares uses the fixed tree (E elements of a chunk, 32 lanes, the
-// 8 warps in order, then the iterations, padded with zero subtrees); the
-// normalised row is kept in shared memory and each radix-2 stage (stride 1, 2,
-// ..., b/2, pairs (a, c) -> (a + c, a - c)) runs over it between barriers, so
-// every value is the one the register kernel produces.
+// 8 warps in order, then the iterations, padded with zero subtrees).  The row
+// is kept in shared memory; the radix-2 stages (stride 1, 2, ..., b/2, pairs
+// (a, c) -> (a + c, a - c)) run three at a time: a thread takes 8 elements at
+// stride 2^st, applies stages st, st+1, st+2 in registers in that order and
+// writes them back, one barrier per pass.  Every value is the one the register
+// kernel produces.  The first pass also applies the norm, the last one c_b
+// and the absmax.
 // ---------------------------------------------------------------------------
 constexpr int HR_THREADS = 256;
 constexpr int HR_MAX_IT = 16;                        // K <= 16384 (fp32: 4 elements per chunk)
+
+// Shared-memory slot of element i: one pad word per 8 keeps every pass's
+// accesses (8 elements at stride 1, 8, 64, ...) free of bank conflicts.
+BN_DEV int hr_pidx(int i) { return i + (i >> 3); }
+
+// Stages st .. st+P-1 over groups of 2^P elements; returns this thread's absmax
+// of the results when LAST (after the factor cb).
+template <int P, bool FIRST, bool LAST>
+BN_DEV float hr_pass(float* hrow, int K, int st, float r, const float* __restrict__ gamma, float cb) {
+  constexpr int G = 1 << P;
+  const int h = 1 << st;
+  float amax = 0.f;
+  for (int q = threadIdx.x; q < K / G; q += HR_THREADS) {
+    const int i0 = ((q >> st) << (st + P)) | (q & (h - 1));
+    float v[G];
+#pragma unroll
+    for (int k = 0; k < G; ++k) v[k] = hrow[hr_pidx(i0 + k * h)];
+    if constexpr (FIRST) {
+#pragma unroll
+      for (int k = 0; k < G; ++k)
+        v[k] = gamma != nullptr ? __fmul_rn(__fmul_rn(v[k], r), __ldg(gamma + i0 + k * h)) : __fmul_rn(v[k], r);
+    }
+#pragma unroll
+    for (int sg = 0; sg < P; ++sg) {
+      const int d = 1 << sg;
+#pragma unroll
+      for (int k = 0; k < G; ++k) {
+        if ((k & d) == 0) {
+          const float a = v[k], c = v[k + d];
+          v[k] = __fadd_rn(a, c);
+          v[k + d] = __fsub_rn(a, c);
+        }
+      }
+    }
+    if constexpr (LAST) {
+#pragma unroll
+      for (int k = 0; k < G; ++k) {
+        v[k] = __fmul_rn(v[k], cb);
+        amax = fmaxf(amax, fabsf(v[k]));
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < G; ++k) hrow[hr_pidx(i0 + k * h)] = v[k];
+  }
+  return amax;
+}
 
 template <typename TIn, int L, int PRE>
 __global__ void __launch_bounds__(HR_THREADS)
 hadamard_quant_i4_row_kernel(const TIn* __restrict__ X, const float* __restrict__ B, int K,
                              const float* __restrict__ gamma, float eps, float cb, uint8_t* __restrict__ Xq4,
                              float* __restrict__ s_x, float* __restrict__ T_dbg) {
+  static_assert(L >= 4, "the first pass takes three stages, the last at least one");
   constexpr int E = InVec<TIn>::E, NW = HR_THREADS / 32;
-  extern __shared__ float hrow[];                    // K floats
+  extern __shared__ float hrow[];                    // K + K/8 floats (hr_pidx)
   __shared__ float red[HR_MAX_IT][NW];
-  __shared__ float bcast[2];
   pdl_launch_dependents();
   pdl_wait();                                        // X may come from, and Xq4 may still be read by, the previous kernel
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -404,8 +453,7 @@ hadamard_quant_i4_row_kernel(const TIn* __restrict__ X, const float* __restrict_
       const size_t off = (size_t)m * K + (size_t)j * E;
       load_chunk<PRE, TIn, E>(X + off, B + off, nullptr, v);
 #pragma unroll
-      for (int q = 0; q < E; q += 4)
-        *reinterpret_cast<float4*>(hrow + (size_t)j * E + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+      for (int e = 0; e < E; ++e) hrow[hr_pidx(j * E + e)] = v[e];
     } else {
 #pragma unroll
       for (int e = 0; e < E; ++e) v[e] = 0.f;
@@ -417,71 +465,54 @@ hadamard_quant_i4_row_kernel(const TIn* __restrict__ X, const float* __restrict_
     if (lane == 0) red[it][warp] = w;
   }
   __syncthreads();
-  if (tid == 0) {
-    float cs[HR_MAX_IT];
+  // every thread forms the same tree from the partials
+  float cs[HR_MAX_IT];
 #pragma unroll
-    for (int it = 0; it < HR_MAX_IT; ++it) {
-      cs[it] = 0.f;                                  // past the padded row: zero subtrees, exact
-      if (it < IT) {
-        float p[NW];
+  for (int it = 0; it < HR_MAX_IT; ++it) {
+    cs[it] = 0.f;                                    // past the padded row: zero subtrees, exact
+    if (it < IT) {
+      float p[NW];
 #pragma unroll
-        for (int w = 0; w < NW; ++w) p[w] = red[it][w];
-        cs[it] = tree_sum<NW>(p);
-      }
+      for (int w = 0; w < NW; ++w) p[w] = red[it][w];
+      cs[it] = tree_sum<NW>(p);
     }
-    const float ss = tree_sum<HR_MAX_IT>(cs);
-    bcast[0] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)K), eps)));
   }
-  __syncthreads();
-  const float r = bcast[0];
-  for (int i = tid; i < K; i += HR_THREADS)
-    hrow[i] = gamma != nullptr ? __fmul_rn(__fmul_rn(hrow[i], r), __ldg(gamma + i)) : __fmul_rn(hrow[i], r);
-  __syncthreads();
+  const float ss = tree_sum<HR_MAX_IT>(cs);
+  const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)K), eps)));
 
-  // ---- radix-2 stages over the row (blocks of 2^L; pairs never cross a block) ----
+  // ---- norm and stages 0-2, then three stages per pass (blocks of 2^L; groups never cross a block) ----
+  hr_pass<3, true, false>(hrow, K, 0, r, gamma, cb);
+  __syncthreads();
+  int st = 3;
 #pragma unroll 1
-  for (int st = 0; st < L; ++st) {
-    const int h = 1 << st;
-    for (int q = tid; q < K / 2; q += HR_THREADS) {
-      const int i = ((q >> st) << (st + 1)) | (q & (h - 1));
-      const float a = hrow[i], c = hrow[i + h];
-      hrow[i] = __fadd_rn(a, c);
-      hrow[i + h] = __fsub_rn(a, c);
-    }
+  for (; st + 3 < L; st += 3) {
+    hr_pass<3, false, false>(hrow, K, st, r, gamma, cb);
     __syncthreads();
   }
-
-  // ---- normalise, absmax ----
-  float amax = 0.f;
-  for (int i = tid; i < K; i += HR_THREADS) {
-    const float tv = __fmul_rn(hrow[i], cb);
-    hrow[i] = tv;
-    amax = fmaxf(amax, fabsf(tv));
-  }
+  float amax = L - st == 3 ? hr_pass<3, false, true>(hrow, K, st, r, gamma, cb)
+             : L - st == 2 ? hr_pass<2, false, true>(hrow, K, st, r, gamma, cb)
+                           : hr_pass<1, false, true>(hrow, K, st, r, gamma, cb);
   amax = warp_max(amax);
-  if (lane == 0) red[0][warp] = amax;
+  if (lane == 0) red[0][warp] = amax;                // red's partial sums were read before the first pass's barrier
   __syncthreads();
-  if (tid == 0) {
-    float a = 0.f;
+  float a = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) a = fmaxf(a, red[0][w]);
-    bcast[1] = __fdiv_rn(7.0f, fmaxf(a, 1e-5f));
-  }
-  __syncthreads();
-  const float s = bcast[1];
+  for (int w = 0; w < NW; ++w) a = fmaxf(a, red[0][w]);
+  const float s = __fdiv_rn(7.0f, fmaxf(a, 1e-5f));
 
   // ---- codes: 32 elements (16 bytes) per step, two per byte ----
   for (int c32 = tid; c32 < K / 32; c32 += HR_THREADS) {
-    const float* src = hrow + 32 * c32;
     uint32_t w[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) w[q] = pack_nibbles8(src + 8 * q, s);
+    for (int q = 0; q < 4; ++q) w[q] = pack_nibbles8(hrow + hr_pidx(32 * c32 + 8 * q), s);   // 8 adjacent slots
     *reinterpret_cast<uint4*>(Xq4 + (size_t)m * (K / 2) + 16 * (size_t)c32) = make_uint4(w[0], w[1], w[2], w[3]);
     if (T_dbg != nullptr) {
 #pragma unroll
-      for (int q = 0; q < 32; q += 4)
+      for (int q = 0; q < 32; q += 4) {
+        const float* src = hrow + hr_pidx(32 * c32 + q);
         *reinterpret_cast<float4*>(T_dbg + (size_t)m * K + 32 * (size_t)c32 + q) =
-            make_float4(src[q], src[q + 1], src[q + 2], src[q + 3]);
+            make_float4(src[0], src[1], src[2], src[3]);
+      }
     }
   }
   if (tid == 0) s_x[m] = s;
@@ -547,7 +578,7 @@ static cudaError_t launch_h4(const void* X, const float* B, int M, int K, const 
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if ((M + TPB - 1) / TPB < 2 * sms) {
     auto rk = hadamard_quant_i4_row_kernel<TIn, L, PRE>;
-    const size_t rsmem = (size_t)K * sizeof(float);
+    const size_t rsmem = (size_t)(K + K / 8) * sizeof(float);
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(rk), rsmem);
     if (e != cudaSuccess) return e;
     return launch_pdl(rk, dim3(M), dim3(HR_THREADS), rsmem, st, 1u, static_cast<const TIn*>(X), B, K, gamma, eps, cb,
