@@ -50,6 +50,11 @@ Readings where the pages are silent (each is listed in the design doc):
   little-endian 32-bit word of 16 consecutive weights, weight 4*j + i sits at
   bits 8*i + 2*j (so byte i holds weights i, 4+i, 8+i, 12+i).  int4 codes:
   byte j holds code 2j in its low nibble and code 2j+1 in its high nibble.
+* Denser weight storage (a reading built on P5's log2(3) = 1.58 bits; the pages
+  give no format): five ternary weights per byte as base-3 digits,
+  byte = sum_i (w_{5g+i} + 1) * 3^i for i = 0..4 (3^5 = 243 <= 256), i.e. 1.6
+  bits per weight.  Weights past K count as 0; each row is padded to a
+  multiple of 16 bytes with bytes of five zero weights (121).
 """
 from __future__ import annotations
 
@@ -140,6 +145,40 @@ def quantize_weights(w: np.ndarray):
     _, s_w = weight_scale(w)
     q = ternarize(w, s_w)
     return pack_ternary(q), s_w, q
+
+
+def trit5_row_bytes(K: int) -> int:
+    """Bytes per row of the five-weights-per-byte format: ceil(K / 5), padded to 16."""
+    groups = (K + 4) // 5
+    return (groups + 15) // 16 * 16
+
+
+def pack_trit5(q: np.ndarray) -> np.ndarray:
+    """Five ternary weights per byte as base-3 digits [P5, log2(3) = 1.58 bits]:
+    byte g of a row = sum_i (q[5g + i] + 1) * 3**i; [N, K] int8 -> [N, trit5_row_bytes(K)] uint8."""
+    q = np.asarray(q, dtype=np.int64)
+    N, K = q.shape
+    assert np.all(np.abs(q) <= 1)
+    R = trit5_row_bytes(K)
+    digits = np.ones((N, R * 5), dtype=np.int64)          # weight 0 (digit 1) past K and in the padding
+    digits[:, :K] = q + 1
+    digits = digits.reshape(N, R, 5)
+    out = np.zeros((N, R), dtype=np.int64)
+    for i in range(5):
+        out += digits[:, :, i] * 3 ** i
+    return out.astype(np.uint8)
+
+
+def unpack_trit5(pk: np.ndarray, K: int) -> np.ndarray:
+    """Inverse of pack_trit5: [N, trit5_row_bytes(K)] uint8 -> [N, K] int8."""
+    b = np.asarray(pk, dtype=np.int64)
+    N, R = b.shape
+    assert R == trit5_row_bytes(K) and np.all(b <= 242)
+    digits = np.zeros((N, R, 5), dtype=np.int64)
+    for i in range(5):
+        digits[:, :, i] = b % 3
+        b = b // 3
+    return (digits.reshape(N, R * 5)[:, :K] - 1).astype(np.int8)
 
 
 # ---------------------------------------------------------------------------

@@ -114,6 +114,28 @@ def _ternarize_no_clamp(w, s_w):
     return np.rint(np.asarray(w, np.float32) * F32(s_w)).astype(np.int8)
 
 
+def _trit5_digits_reversed(q):
+    """Most significant digit first: a plausible slip in the base-3 order."""
+    pk = _orig["pack_trit5"](q).astype(np.int64)
+    out = np.zeros_like(pk)
+    for i in range(5):
+        out = out * 3 + pk % 3
+        pk = pk // 3
+    return out.astype(np.uint8)
+
+
+def _trit5_offset_minus(q):
+    """Digits w mod 3 instead of w + 1 (-1 -> 2, 0 -> 0, +1 -> 1)."""
+    q = np.asarray(q, np.int64)
+    N, K = q.shape
+    R = O.trit5_row_bytes(K)
+    d = np.zeros((N, R * 5), np.int64)
+    d[:, :K] = q % 3
+    d = d.reshape(N, R, 5)
+    return sum(d[:, :, i] * 3 ** i for i in range(5)).astype(np.uint8)
+
+
+
 MUTATIONS = {
     "absmax_numerator_128": ("absmax_quantize", _absmax_128),
     "absmax_truncates": ("absmax_quantize", _absmax_no_rint),
@@ -131,6 +153,8 @@ MUTATIONS = {
     "rms_mean_abs": ("rms_norm", _rms_mean_of_abs),
     "matmul_drops_term": ("int_matmul", _matmul_drop_last_k),
     "dequant_multiplies": ("dequantize", _dequant_times),
+    "trit5_digits_reversed": ("pack_trit5", _trit5_digits_reversed),
+    "trit5_digit_offset": ("pack_trit5", _trit5_offset_minus),
 }
 
 

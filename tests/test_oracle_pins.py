@@ -142,6 +142,35 @@ def check_int4_pack_golden():
     assert O.unpack_int4(O.pack_int4(codes)).tolist() == codes.tolist()
 
 
+def check_trit5_pack_golden():
+    rows = _golden("trit5_pack_layout.txt")
+    g = {r.split()[0]: r.split()[1:] for r in rows if not r.startswith("single")}
+    w = np.array([[int(v) for v in g["weights"]]], dtype=np.int8)
+    pk = O.pack_trit5(w)
+    assert pk.tolist() == [[int(b) for b in g["bytes"]]]
+    assert O.unpack_trit5(pk, w.shape[1]).tolist() == w.tolist()
+    for r in rows:
+        if r.startswith("single"):
+            *ws, b = [int(v) for v in r.split()[1:]]
+            assert O.pack_trit5(np.array([ws], np.int8))[0, 0] == b
+
+
+def check_trit5_is_a_bijection_on_five_weights():
+    """All 3^5 five-weight groups map to the 243 distinct bytes 0..242 and back."""
+    combos = np.array(np.meshgrid(*[[-1, 0, 1]] * 5, indexing="ij")).reshape(5, -1).T.astype(np.int8)
+    b = O.pack_trit5(combos)[:, 0]
+    assert sorted(b.tolist()) == list(range(243))
+    assert np.array_equal(O.unpack_trit5(O.pack_trit5(combos), 5), combos)
+
+
+def check_trit5_agrees_with_two_bit_packing():
+    """Both storage formats hold the same weights; 1.6 bits per weight at K = 2560."""
+    q = np.random.default_rng(5).integers(-1, 2, size=(9, 2560)).astype(np.int8)
+    assert np.array_equal(O.unpack_trit5(O.pack_trit5(q), 2560), O.unpack_ternary(O.pack_ternary(q)))
+    assert O.pack_trit5(q).shape == (9, 512) and 8 * 512 / 2560 == 1.6
+    assert O.trit5_row_bytes(37) == 16 and O.trit5_row_bytes(80) == 16 and O.trit5_row_bytes(81) == 32
+
+
 def check_packing_ratio_llama3_8b():
     """8B -> 2.8B only if the linear weights are four per byte and the
     embedding and output head stay unpacked."""
