@@ -328,6 +328,10 @@ def run_ours(args, rank, world, local_rank):
     # decode: the same weight ring at the other decode batch sizes (linear launches only)
     sweep = []
     if args.workload == "decode":
+        # the same weights five per byte (1.6 bits per weight), repacked on the GPU
+        ring5 = [api.bitnet_repack_trit5(pk, stream=stream) for pk, _ in ring]
+        torch.cuda.synchronize()
+        r5_bytes = N * api.bitnet_trit5_row_bytes(K)
         for Ms in (1, 4, 16):
             cs = wl.decode(Ms, with_weights=False)
             xs = torch.from_numpy(cs["x"].view(np.int16)).view(torch.bfloat16).to(dev)
@@ -344,6 +348,9 @@ def run_ours(args, rank, world, local_rank):
                 pk, s_w = ring[i % copies]
                 api.bitnet_bitlinear(xs, pk, s_w, None, eps, Y=Ys, Xq=xqs, s_x=sxs, stream=stream)
 
+            def lin5_s(i, xqs=xqs, sxs=sxs, Ys=Ys):
+                api.bitnet_linear_trit5(xqs, 8, sxs, ring5[i % copies], ring[i % copies][1], K, Y=Ys, stream=stream)
+
             def step_s(i, xs=xs, xqs=xqs, sxs=sxs, Ys=Ys):
                 api.bitnet_quant_act(xs, None, eps, Xq=xqs, s_x=sxs, stream=stream)
                 lin_s(i)
@@ -358,10 +365,16 @@ def run_ours(args, rank, world, local_rank):
                 step_s(i)
             t_s = timed(graph_of(lin_s, steps)) / steps / 1e3
             t_st = timed(graph_of(step_s, steps)) / steps / 1e3
+            for i in range(warmup):
+                lin5_s(i)
+            t_5 = timed(graph_of(lin5_s, steps)) / steps / 1e3
             hbm = load_peaks()[0]["hbm_gbs"]
             b = packed_bytes + Ms * K + 4 * Ms + 4 + Ms * N * out_bytes
             bf = packed_bytes + 2 * Ms * K + Ms * K + 4 * Ms + 4 + Ms * N * out_bytes
+            b5 = r5_bytes + Ms * K + 4 * Ms + 4 + Ms * N * out_bytes
             sweep.append({"M": Ms, "linear_us": t_s * 1e6, "linear_GBs": b / t_s / 1e9,
+                          "trit5_linear_us": t_5 * 1e6, "trit5_linear_GBs": b5 / t_5 / 1e9,
+                          "trit5_linear_frac": b5 / t_5 / 1e9 / hbm,
                           "linear_frac": b / t_s / 1e9 / hbm, "step_us": t_st * 1e6, "tokens_per_s": Ms / t_st,
                           "fused_kernel_us": t_f * 1e6, "fused_kernel_frac": bf / t_f / 1e9 / hbm})
 

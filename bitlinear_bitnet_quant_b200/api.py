@@ -48,6 +48,10 @@ _SIGNATURES = {
                                                      ctypes.c_int, _c_void_p, _c_void_p, _c_void_p]),
     "bitnet_add": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _i64, _c_void_p]),
     "bitnet_relu2_glu": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _i64, _c_void_p]),
+    "bitnet_trit5_row_bytes": (ctypes.c_size_t, [_i64]),
+    "bitnet_repack_trit5": (ctypes.c_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
+    "bitnet_linear_trit5": (ctypes.c_int, [_c_void_p, ctypes.c_int, _c_void_p, _c_void_p, _c_void_p, _i64, _i64,
+                                           _i64, _c_void_p, ctypes.c_int, _c_void_p, _c_void_p]),
     "bitnet_set_linear_path": (ctypes.c_int, [ctypes.c_int]),
     "bitnet_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
 }
@@ -213,6 +217,36 @@ def bitnet_linear(Xq: torch.Tensor, act_bits: int, s_x: torch.Tensor, pkW: torch
     acc = torch.empty((M, N), dtype=torch.int32, device=Xq.device) if want_acc else None
     _check("bitnet_linear", lib().bitnet_linear(
         _ptr(Xq), int(act_bits), _ptr(s_x), _ptr(pkW), _ptr(s_w), M, N, K, _ptr(Y), _dtype_code(Y),
+        _ptr(acc), _stream(stream)))
+    return Y, acc
+
+
+def bitnet_trit5_row_bytes(K: int) -> int:
+    """Bytes per row of the five-weights-per-byte format."""
+    return int(lib().bitnet_trit5_row_bytes(int(K)))
+
+
+def bitnet_repack_trit5(pkW: torch.Tensor, pk5=None, stream=None):
+    """2-bit packed weights [N, K/4] -> five weights per byte [N, bitnet_trit5_row_bytes(K)] uint8."""
+    _require(pkW, "pkW")
+    N, KB = pkW.shape
+    K = KB * 4
+    pk5 = torch.empty((N, bitnet_trit5_row_bytes(K)), dtype=torch.uint8, device=pkW.device) if pk5 is None else pk5
+    _check("bitnet_repack_trit5", lib().bitnet_repack_trit5(_ptr(pkW), N, K, _ptr(pk5), _stream(stream)))
+    return pk5
+
+
+def bitnet_linear_trit5(Xq: torch.Tensor, act_bits: int, s_x: torch.Tensor, pk5: torch.Tensor, s_w: torch.Tensor,
+                        K: int, out_dtype=torch.float32, Y=None, want_acc: bool = False, stream=None):
+    """bitnet_linear with the weights five per byte (decode shapes).  Returns (Y [M, N], acc int32 or None)."""
+    _require(Xq, "Xq")
+    _require(pk5, "pk5")
+    M = Xq.shape[0]
+    N = pk5.shape[0]
+    Y = torch.empty((M, N), dtype=out_dtype, device=Xq.device) if Y is None else Y
+    acc = torch.empty((M, N), dtype=torch.int32, device=Xq.device) if want_acc else None
+    _check("bitnet_linear_trit5", lib().bitnet_linear_trit5(
+        _ptr(Xq), int(act_bits), _ptr(s_x), _ptr(pk5), _ptr(s_w), M, N, int(K), _ptr(Y), _dtype_code(Y),
         _ptr(acc), _stream(stream)))
     return Y, acc
 

@@ -30,6 +30,11 @@ cudaError_t run_bitlinear(const void* X, int x_bf16, int M, int K, const float* 
 bool decode_path_applies(int M, int K);
 bool fused_path_applies(int M, int N, int K, int x_bf16);
 cudaError_t run_add_f32(const float* a, const float* b, float* out, size_t n, cudaStream_t st);
+cudaError_t run_repack_trit5(const uint8_t* pkW, int N, int K, uint8_t* pk5, cudaStream_t st);
+size_t trit5_row_bytes_host(int K);
+cudaError_t run_linear_decode_trit5(const void* Xq, int act_bits, const float* s_x, const uint8_t* pk5,
+                                    const float* s_w, int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg,
+                                    cudaStream_t st);
 cudaError_t run_relu2_glu(const float* gate, const float* up, float* out, size_t n, cudaStream_t st);
 }  // namespace bitnet
 
@@ -193,6 +198,40 @@ int bitnet_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t*
   return cuda_status(bitnet::run_linear(Xq, act_bits, s_x, pkW, s_w, (int)M, (int)N, (int)K, Y,
                                         y_dtype == BITNET_BF16, acc_dbg, linear_path(),
                                         static_cast<cudaStream_t>(stream)));
+}
+
+size_t bitnet_trit5_row_bytes(int64_t K) {
+  if (K < 1 || K > (int64_t(1) << 30)) return 0;
+  return bitnet::trit5_row_bytes_host((int)K);
+}
+
+int bitnet_repack_trit5(const uint8_t* pkW, int64_t N, int64_t K, uint8_t* pk5, void* stream) {
+  if (N < 1 || K < 16 || K % 16 != 0 || K > (int64_t(1) << 30)) return BITNET_ERR_SHAPE;
+  if (N * (int64_t)bitnet::trit5_row_bytes_host((int)K) >= (int64_t(1) << 31) || N * K / 4 >= (int64_t(1) << 31))
+    return BITNET_ERR_SHAPE;
+  if (!pkW || !pk5) return BITNET_ERR_NULL;
+  if (!aligned16(pkW) || !aligned16(pk5)) return BITNET_ERR_ALIGN;
+  int d = check_device();
+  if (d != BITNET_OK) return d;
+  return cuda_status(bitnet::run_repack_trit5(pkW, (int)N, (int)K, pk5, static_cast<cudaStream_t>(stream)));
+}
+
+int bitnet_linear_trit5(const void* Xq, int act_bits, const float* s_x, const uint8_t* pk5, const float* s_w,
+                        int64_t M, int64_t N, int64_t K, void* Y, int y_dtype, int32_t* acc_dbg, void* stream) {
+  if (act_bits != 8 && act_bits != 4) return BITNET_ERR_DTYPE;
+  if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (M < 1 || M > 32 || N < 1 || N > (int64_t(1) << 30) || K < 512 || K > 16384 ||
+      !bitnet::decode_path_applies((int)M, (int)K))
+    return BITNET_ERR_SHAPE;
+  if (!Xq || !s_x || !pk5 || !s_w || !Y) return BITNET_ERR_NULL;
+  if (!aligned16(Xq) || !aligned16(pk5) || !aligned16(Y) || (acc_dbg && !aligned16(acc_dbg)) ||
+      (reinterpret_cast<uintptr_t>(s_x) & 3u) || (reinterpret_cast<uintptr_t>(s_w) & 3u))
+    return BITNET_ERR_ALIGN;
+  int d = check_device();
+  if (d != BITNET_OK) return d;
+  return cuda_status(bitnet::run_linear_decode_trit5(Xq, act_bits, s_x, pk5, s_w, (int)M, (int)N, (int)K, Y,
+                                                     y_dtype == BITNET_BF16, acc_dbg,
+                                                     static_cast<cudaStream_t>(stream)));
 }
 
 static int elementwise_check(const float* a, const float* b, const float* out, int64_t n) {

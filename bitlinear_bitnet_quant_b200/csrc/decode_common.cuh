@@ -86,6 +86,67 @@ BN_DEV void dec_copy_weights(const uint8_t* __restrict__ pkW, int N, int K, int 
   cp_async_commit();
 }
 
+// ---------------------------------------------------------------------------
+// Weights stored five per byte ("양자화(quantization) 1.58bit", section
+// "1.58비트는 어디서 나온거에요?": three states carry log2(3) = 1.58 bits):
+// byte g of a row holds w[5g .. 5g+4] as base-3 digits w + 1, least
+// significant first, so 3^5 = 243 <= 256 and a weight costs 1.6 bits.  Rows
+// are padded to 16 bytes.  The decode kernel stages a slice of these rows and
+// rewrites it into the 2-bit slice layout above before the dependency wait.
+// ---------------------------------------------------------------------------
+__host__ __device__ inline int trit5_row_bytes(int K) { return ((K + 4) / 5 + 15) / 16 * 16; }
+
+// The five weights of byte b as 2-bit two's complement codes, weight i at bits 2i.
+BN_DEV uint32_t trit5_codes(int b) {
+  uint32_t c = 0;
+#pragma unroll
+  for (int i = 0; i < 5; ++i) {
+    const int d = b % 3;
+    b /= 3;
+    c |= (uint32_t)((d - 1) & 3) << (2 * i);
+  }
+  return c;
+}
+
+// 16-byte asynchronous copies of rows n0 .. n0+ROWS-1 of the five-per-byte
+// weights (row stride r5 bytes) into `stage`; rows past N read as zeros.
+template <int ROWS>
+BN_DEV void dec_copy_trit5(const uint8_t* __restrict__ pk5, int N, int r5, int n0, uint8_t* stage) {
+  const int cpr = r5 / 16;
+  const uint32_t sbase = smem_u32(stage);
+  for (int c = threadIdx.x; c < ROWS * cpr; c += DEC_THREADS) {
+    const int r = c / cpr, q = c - r * cpr;
+    const bool in = n0 + r < N;
+    const uint8_t* src = pk5 + (in ? (size_t)(n0 + r) * r5 + 16 * (size_t)q : 0);
+    cp_async_16(sbase + (uint32_t)(r * r5 + 16 * q), src, in ? 16u : 0u);
+  }
+  cp_async_commit();
+}
+
+// Rewrites the staged slice into the 2-bit slice layout.  Packed word wi of a
+// row (weights 16 wi .. 16 wi + 15) always draws on four consecutive bytes:
+// their codes are laid end to end (weight m at bits 2m), then the 4 x 4 grid
+// of 2-bit cells is transposed by two bit-field swaps, which puts weight
+// 4j + i at bits 8i + 2j.
+template <int ROWS>
+BN_DEV void dec_trit5_to_2bit(const uint8_t* stage, int r5, int K, const uint16_t* lut5, uint8_t* wsm) {
+  const int wpr = K / 16;
+  for (int idx = threadIdx.x; idx < ROWS * wpr; idx += DEC_THREADS) {
+    const int r = idx / wpr, wi = idx - r * wpr;
+    const int k0 = 16 * wi, g0 = k0 / 5, o = k0 - 5 * g0;
+    const uint8_t* src = stage + r * r5 + g0;
+    uint32_t v = (uint32_t)lut5[src[0]] >> (2 * o);
+#pragma unroll
+    for (int n = 1; n < 4; ++n) v |= (uint32_t)lut5[src[n]] << (10 * n - 2 * o);
+    uint32_t t = ((v >> 12) ^ v) & 0x0000F0F0u;     // swap the 2 x 2 blocks of cells
+    v ^= t ^ (t << 12);
+    t = ((v >> 6) ^ v) & 0x00CC00CCu;               // swap the cells inside each block
+    v ^= t ^ (t << 6);
+    const int sg = k0 >> 9, q = (k0 >> 6) & 7, tt = (k0 >> 4) & 3;
+    *reinterpret_cast<uint32_t*>(wsm + (size_t)sg * (ROWS * 128) + r * 128 + 16 * (q ^ (r & 7)) + 4 * tt) = v;
+  }
+}
+
 // This thread's packed words of segment sg: rows 16 rg + g and + 8, word t of
 // chunk `warp` (stored at chunk warp ^ g).
 template <int RG>
@@ -170,6 +231,14 @@ BN_DEV void dec_epilogue(const int (&d)[NACC][RG][TG][4], int32_t* red, const fl
       dec_store(Y + (size_t)m * N + n, __fmul_rn((float)acc, sdq[m]));
     }
   }
+}
+
+// Offset of the five-per-byte staging rows: after the 2-bit slice, which the
+// epilogue's partial tiles reuse.
+template <int TG, int RG>
+__host__ __device__ inline size_t dec_stage_offset(int K) {
+  const size_t wbytes = (size_t)16 * RG * (size_t)K / 4, rbytes = dec_red_bytes<TG, RG>();
+  return wbytes > rbytes ? wbytes : rbytes;
 }
 
 // Weight rows per CTA: spread N over the SMs in multiples of 16, at most

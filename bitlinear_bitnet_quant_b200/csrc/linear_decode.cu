@@ -43,8 +43,10 @@ namespace bitnet {
 // accumulator sets, summed at the end).
 //
 // `tsplit` CTAs share each weight slice: CTA b takes rows (b / tsplit) * ROWS
-// onwards and tokens 8 * TG * (b % tsplit) onwards.
-template <int ACT_BITS, int TG, int RG, typename TOut>
+// onwards and tokens 8 * TG * (b % tsplit) onwards.  W5: pkW holds the weights
+// five per byte (trit5_row_bytes(K) bytes per row), rewritten into the 2-bit
+// slice layout in shared memory before the dependency wait.
+template <int ACT_BITS, int TG, int RG, typename TOut, bool W5>
 __global__ void __launch_bounds__(DEC_THREADS, 2)
 linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict__ Xq,
                      const float* __restrict__ s_x, const float* __restrict__ s_w_ptr, int M, int N, int K,
@@ -57,6 +59,7 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
   static_assert(RG >= 1 && RG <= C::RG_MAX, "row groups");
   extern __shared__ uint8_t dec_smem_raw[];
   __shared__ float sdq[TOK];
+  __shared__ uint16_t lut5[W5 ? 243 : 1];
 
   uint8_t* wsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dec_smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -77,9 +80,21 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
   // be scheduled at once (it only waits for this grid to finish).
   pdl_launch_dependents();
   // the weights do not depend on the previous kernel: stream them now
-  dec_copy_weights<ROWS>(pkW, N, K, n0, wsm);
+  const int r5 = trit5_row_bytes(K);
+  uint8_t* stage = wsm + dec_stage_offset<TG, RG>(K);
+  if constexpr (W5) {
+    dec_copy_trit5<ROWS>(pkW, N, r5, n0, stage);
+    for (int b = threadIdx.x; b < 243; b += DEC_THREADS) lut5[b] = (uint16_t)trit5_codes(b);
+  } else {
+    dec_copy_weights<ROWS>(pkW, N, K, n0, wsm);
+  }
   // s_w belongs to the weights: read it before the wait as well
   const float sw = threadIdx.x < TOK ? ldg_nc_f32(s_w_ptr) : 0.0f;
+  if constexpr (W5) {
+    cp_async_wait_all();
+    __syncthreads();                           // staged bytes and the digit table
+    dec_trit5_to_2bit<ROWS>(stage, r5, K, lut5, wsm);   // made visible by the loop's first barrier
+  }
   pdl_wait();                                  // activations and s_x come from the previous kernel
   // issued now, consumed only in the epilogue
   const float sx = threadIdx.x < M && threadIdx.x < TOK ? ldg_f32(s_x + threadIdx.x) : 1.0f;
@@ -151,14 +166,19 @@ bool decode_path_applies(int M, int K) {
   return M >= 1 && M <= DEC_MAX_TOKENS && K % 512 == 0 && K / 512 <= DEC_MAX_SEGS;
 }
 
-template <int ACT_BITS, int TG, int RG, typename TOut>
+// Shared memory of one CTA: the 2-bit slice (reused by the epilogue's partial
+// tiles), then, for five-per-byte weights, the staged rows.
+template <int TG, int RG>
+static size_t dec_smem_bytes(int K, bool w5) {
+  return dec_stage_offset<TG, RG>(K) + (w5 ? (size_t)16 * RG * trit5_row_bytes(K) : 0) + 1024;
+}
+
+template <int ACT_BITS, int TG, int RG, typename TOut, bool W5>
 static cudaError_t launch_decode_rg(const void* Xq, const float* s_x, const uint8_t* pkW, const float* s_w, int M,
                                     int N, int K, int tsplit, void* Y, int32_t* acc_dbg, cudaStream_t st) {
   constexpr int ROWS = 16 * RG;
-  const size_t wbytes = (size_t)ROWS * (size_t)K / 4;
-  const size_t rbytes = dec_red_bytes<TG, RG>();
-  const size_t smem = (wbytes > rbytes ? wbytes : rbytes) + 1024;
-  auto kern = linear_decode_kernel<ACT_BITS, TG, RG, TOut>;
+  const size_t smem = dec_smem_bytes<TG, RG>(K, W5);
+  auto kern = linear_decode_kernel<ACT_BITS, TG, RG, TOut, W5>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)((N + ROWS - 1) / ROWS * tsplit));
@@ -166,7 +186,7 @@ static cudaError_t launch_decode_rg(const void* Xq, const float* s_x, const uint
                     K, tsplit, static_cast<TOut*>(Y), acc_dbg);
 }
 
-template <int ACT_BITS, int TG, typename TOut>
+template <int ACT_BITS, int TG, typename TOut, bool W5>
 static cudaError_t launch_decode_t(const void* Xq, const float* s_x, const uint8_t* pkW, const float* s_w, int M,
                                    int N, int K, int tsplit, void* Y, int32_t* acc_dbg, cudaStream_t st) {
   int dev = 0, sms = 148;
@@ -177,7 +197,7 @@ static cudaError_t launch_decode_t(const void* Xq, const float* s_x, const uint8
   // 3.5 -> 2.9 us at N = 6912, K = 2560); with the token groups spread over
   // CTAs the grid already holds two per SM
   const int rg = decode_rows(N, K, sms * (tsplit == 1 ? 2 : 1), DecCfg<TG>::MAX_ROWS) / 16;
-#define BN_RG(R) launch_decode_rg<ACT_BITS, TG, (R <= DecCfg<TG>::RG_MAX ? R : 1), TOut>(Xq, s_x, pkW, s_w, M, N, K, tsplit, Y, acc_dbg, st)
+#define BN_RG(R) launch_decode_rg<ACT_BITS, TG, (R <= DecCfg<TG>::RG_MAX ? R : 1), TOut, W5>(Xq, s_x, pkW, s_w, M, N, K, tsplit, Y, acc_dbg, st)
   switch (rg) {
     case 1: return BN_RG(1);
     case 2: return BN_RG(2);
@@ -187,20 +207,35 @@ static cudaError_t launch_decode_t(const void* Xq, const float* s_x, const uint8
 #undef BN_RG
 }
 
-cudaError_t run_linear_decode(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
-                              int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, cudaStream_t st) {
+template <bool W5>
+static cudaError_t dispatch_decode(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW,
+                                   const float* s_w, int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg,
+                                   cudaStream_t st) {
   // up to 16 tokens: one token group per CTA (two CTAs per weight slice past
   // 8 tokens); up to 32: two token groups per CTA, two CTAs per slice
 #define BN_DEC(BITS, T)                                                                                   \
-  return M <= 8    ? launch_decode_t<BITS, 1, T>(Xq, s_x, pkW, s_w, M, N, K, 1, Y, acc_dbg, st)          \
-         : M <= 16 ? launch_decode_t<BITS, 1, T>(Xq, s_x, pkW, s_w, M, N, K, 2, Y, acc_dbg, st)          \
-                   : launch_decode_t<BITS, 2, T>(Xq, s_x, pkW, s_w, M, N, K, (M + 15) / 16, Y, acc_dbg, st)
+  return M <= 8    ? launch_decode_t<BITS, 1, T, W5>(Xq, s_x, pkW, s_w, M, N, K, 1, Y, acc_dbg, st)      \
+         : M <= 16 ? launch_decode_t<BITS, 1, T, W5>(Xq, s_x, pkW, s_w, M, N, K, 2, Y, acc_dbg, st)      \
+                   : launch_decode_t<BITS, 2, T, W5>(Xq, s_x, pkW, s_w, M, N, K, (M + 15) / 16, Y, acc_dbg, st)
   if (act_bits == 8) {
     if (y_bf16) { BN_DEC(8, __nv_bfloat16); } else { BN_DEC(8, float); }
   } else {
     if (y_bf16) { BN_DEC(4, __nv_bfloat16); } else { BN_DEC(4, float); }
   }
 #undef BN_DEC
+}
+
+cudaError_t run_linear_decode(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
+                              int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, cudaStream_t st) {
+  return dispatch_decode<false>(Xq, act_bits, s_x, pkW, s_w, M, N, K, Y, y_bf16, acc_dbg, st);
+}
+
+// Weights five per byte (trit5_row_bytes(K) bytes per row); same shapes as the
+// 2-bit decode path, results bit-identical to it.
+cudaError_t run_linear_decode_trit5(const void* Xq, int act_bits, const float* s_x, const uint8_t* pk5,
+                                    const float* s_w, int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg,
+                                    cudaStream_t st) {
+  return dispatch_decode<true>(Xq, act_bits, s_x, pk5, s_w, M, N, K, Y, y_bf16, acc_dbg, st);
 }
 
 }  // namespace bitnet

@@ -185,6 +185,30 @@ BITNET_API int bitnet_linear(const void* Xq, int act_bits, const float* s_x, con
                   void* Y, int y_dtype, int32_t* acc_dbg, void* stream);
 
 /*
+ * Denser weight storage: five ternary weights per byte as base-3 digits,
+ * 1.6 bits per weight instead of 2 ("양자화(quantization) 1.58bit", section
+ * "1.58비트는 어디서 나온거에요?": three states carry log2(3) = 1.58 bits).
+ * Byte g of a row = sum_i (w[5g + i] + 1) * 3^i for i = 0..4; weights past K
+ * count as 0; each row is padded to bitnet_trit5_row_bytes(K) bytes (a
+ * multiple of 16) with the byte of five zero weights, 121.
+ *
+ * bitnet_trit5_row_bytes: bytes per row, ceil(K / 5) rounded up to 16.
+ * bitnet_repack_trit5: pkW [N][K/4] (bitnet_quantize_weights' 2-bit format,
+ *   read) -> pk5 [N][bitnet_trit5_row_bytes(K)] (written).  Limits: N >= 1,
+ *   16 <= K, K % 16 == 0, N * row bytes < 2^31; pointers 16-byte aligned.
+ * bitnet_linear_trit5: bitnet_linear with the weights in this format, for the
+ *   decode shapes only (1 <= M <= 32, K % 512 == 0, K <= 16384; otherwise
+ *   BITNET_ERR_SHAPE).  Each CTA stages its rows and rewrites them into the
+ *   2-bit layout in shared memory before it waits for the previous kernel;
+ *   results are bit-identical to bitnet_linear.  Other arguments as there.
+ */
+BITNET_API size_t bitnet_trit5_row_bytes(int64_t K);
+BITNET_API int bitnet_repack_trit5(const uint8_t* pkW, int64_t N, int64_t K, uint8_t* pk5, void* stream);
+BITNET_API int bitnet_linear_trit5(const void* Xq, int act_bits, const float* s_x, const uint8_t* pk5,
+                        const float* s_w, int64_t M, int64_t N, int64_t K,
+                        void* Y, int y_dtype, int32_t* acc_dbg, void* stream);
+
+/*
  * Fused BitLinear forward with int8 activations: bitnet_quant_act followed by
  * bitnet_linear (act_bits = 8) in one call, with bit-identical results
  * [P4 양자화 메커니즘, 계산 패러다임, 추론 최적화 및 커스텀 커널].

@@ -123,6 +123,26 @@ def test_fused_quantiser_validation(L):
     assert gh(u=None) == 1 and gh(g=MISALIGNED) == 3
 
 
+def test_trit5_validation(L):
+    assert L.bitnet_trit5_row_bytes(2560) == 512 and L.bitnet_trit5_row_bytes(37) == 16
+    assert L.bitnet_trit5_row_bytes(81) == 32 and L.bitnet_trit5_row_bytes(0) == 0
+    rp = lambda **kw: L.bitnet_repack_trit5(kw.get("pk", ALIGNED), kw.get("N", 8), kw.get("K", 512),
+                                            kw.get("out", ALIGNED), None)
+    assert rp(K=24) == 2 and rp(K=0) == 2 and rp(N=0) == 2
+    assert rp(pk=None) == 1 and rp(out=None) == 1
+    assert rp(pk=MISALIGNED) == 3 and rp(out=MISALIGNED) == 3
+
+    def lt(**kw):
+        a = dict(Xq=ALIGNED, bits=8, s_x=ALIGNED, pk=ALIGNED, s_w=ALIGNED, M=4, N=256, K=2560, Y=ALIGNED, yt=0)
+        a.update(kw)
+        return L.bitnet_linear_trit5(a["Xq"], a["bits"], a["s_x"], a["pk"], a["s_w"], a["M"], a["N"], a["K"],
+                                     a["Y"], a["yt"], None, None)
+    assert lt(bits=2) == 4 and lt(yt=5) == 4
+    assert lt(M=33) == 2 and lt(M=0) == 2 and lt(K=384) == 2 and lt(K=16384 + 512) == 2 and lt(N=0) == 2
+    assert lt(pk=None) == 1 and lt(Y=None) == 1
+    assert lt(pk=MISALIGNED) == 3 and lt(s_w=ALIGNED + 2) == 3
+
+
 def test_linear_path_selector(L):
     assert L.bitnet_set_linear_path(5) == 2
     assert L.bitnet_set_linear_path(4) == 0

@@ -260,6 +260,62 @@ def test_linear_decode_kernel(M, N, K, act_bits, out):
     _check_linear(qx, qw, s_x, s_w, act_bits, out, path=3)
 
 
+# ------------------------------------------------- five weights per byte ----
+
+@pytest.mark.parametrize("N,K", [(3, 16), (7, 48), (64, 2560), (300, 8192), (1, 16384), (5, 1040), (129, 80)])
+def test_repack_trit5(N, K):
+    """2-bit packed -> five per byte, bit-exact against the oracle's packing of the same codes."""
+    qw = np.random.default_rng(N * K).integers(-1, 2, size=(N, K)).astype(np.int8)
+    pk5 = api.bitnet_repack_trit5(dev(O.pack_ternary(qw)))
+    torch.cuda.synchronize()
+    assert np.array_equal(host(pk5), O.pack_trit5(qw))
+
+
+@pytest.mark.parametrize("M,N,K,act_bits,out", [
+    (1, 16, 512, 8, "f32"), (1, 1, 512, 8, "f32"), (4, 6912, 2560, 8, "f32"), (8, 1000, 1536, 8, "bf16"),
+    (9, 4096, 512, 8, "f32"), (16, 6912, 2560, 8, "f32"), (16, 300, 8192, 8, "f32"), (5, 64, 16384, 8, "f32"),
+    (17, 1000, 2048, 8, "f32"), (32, 2048, 5632, 4, "f32"), (7, 333, 2560, 4, "bf16"), (24, 333, 512, 4, "f32")])
+def test_linear_trit5(M, N, K, act_bits, out):
+    """The decode kernel reading five-per-byte weights (packed by the oracle): int32
+    accumulators and outputs bit-exact against the oracle and against the 2-bit path."""
+    qx, qw, s_x, s_w = _random_codes(M, N, K, act_bits, M * 17 + N + K)
+    xq_dev = dev(qx) if act_bits == 8 else dev(O.pack_int4(qx))
+    odt = torch.float32 if out == "f32" else torch.bfloat16
+    Y5, acc5 = api.bitnet_linear_trit5(xq_dev, act_bits, dev(s_x), dev(O.pack_trit5(qw)),
+                                       dev(np.array([s_w], np.float32)), K, out_dtype=odt, want_acc=True)
+    torch.cuda.synchronize()
+    Y2, _ = _run_linear(qx, qw, s_x, s_w, act_bits, out, path=3)
+    Y5h = host(Y5.float() if out == "bf16" else Y5)
+    acc_o, y_o = O.linear(qx, s_x, qw, s_w)
+    assert np.array_equal(host(acc5), acc_o)
+    if out == "f32":
+        assert np.array_equal(Y5h.view(np.uint32), y_o.view(np.uint32))
+    else:
+        assert np.array_equal(O.bf16_round(Y5h), O.bf16_round(y_o))
+    assert torch.equal(Y5.view(torch.int16 if out == "bf16" else torch.int32),
+                       Y2.view(torch.int16 if out == "bf16" else torch.int32))
+
+
+def test_trit5_end_to_end_from_fp32_weights():
+    """bitnet_quantize_weights -> bitnet_repack_trit5 -> bitnet_linear_trit5 on the decode
+    workload's weights (sampled rows), against the oracle."""
+    c = wl.decode(4)
+    w = c["w"]
+    pk, s_w = api.bitnet_quantize_weights(dev(w))
+    pk5 = api.bitnet_repack_trit5(pk)
+    xd, x_or = x_inputs(c["x"], "bf16")
+    xq, s_x = api.bitnet_quant_act(xd, None, 1e-6)
+    Y, acc = api.bitnet_linear_trit5(xq, 8, s_x, pk5, s_w, w.shape[1], want_acc=True)
+    torch.cuda.synchronize()
+    _, s_o, q_o = O.quantize_weights(w)
+    assert np.array_equal(host(pk5), O.pack_trit5(q_o))
+    qx_o, sx_o = O.quant_act(x_or, None, 1e-6)
+    rows = np.random.default_rng(3).choice(w.shape[0], 256, replace=False)
+    acc_o, y_o = O.linear(qx_o, sx_o, q_o[rows], s_o)
+    assert np.array_equal(host(acc)[:, rows], acc_o)
+    assert np.array_equal(host(Y)[:, rows].view(np.uint32), y_o.view(np.uint32))
+
+
 def test_linear_decode_kernel_rejects_other_shapes():
     qx, qw, s_x, s_w = _random_codes(33, 64, 512, 8, 1)
     with pytest.raises(api.BitnetError):
