@@ -240,7 +240,7 @@ BN_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_depend
 BN_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
-// TMA (no multicast anywhere)
+// TMA (plain per-CTA loads and stores)
 // ---------------------------------------------------------------------------
 BN_DEV void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" :: "l"(tmap) : "memory");

@@ -33,7 +33,7 @@ do not fix a precision.  Sources, cited by page title and section:
      "quantization factor" is 127/5.4 = 23.5 and dequantisation divides by it.
      Section "1.58비트는 어디서 나온거에요?": three states, log2(3) = 1.58 bits.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * Mean |W| is the exact sum of |W| rounded once to fp64, divided by N*K in
   fp64, rounded to fp32.  s_w = 1 / max(mean, 1e-5) in fp32.
