@@ -610,6 +610,38 @@ def cpu_baseline(c, budget_s=10.0):
             "sample": f"{n} oracle steps of {len(rows)} tokens of {c['name']} (numpy, single thread)"}
 
 
+def cpu_baseline_omp(c, budget_s=5.0):
+    """The same oracle step through the plain C++ oracle, its loops over tokens and
+    output rows on all host cores (bit-identical results to the numpy oracle)."""
+    from oracle import c_oracle as C
+    w = wl.weights(c["N"], c["K"], seed=0)
+    _, s_w, qw = C.quantize_weights(w)
+    x = (c["x"].astype(np.uint32) << 16).view(np.float32) if c["x_dtype"] == "bf16" else c["x"]
+    rows = np.arange(c["M"]) if c["M"] <= 16 else np.arange(128)
+
+    def step():
+        xs = x[rows]
+        if c["act_bits"] == 8:
+            q, s = C.quant_act(xs, None, 1e-6)
+        else:
+            _, s, q, _ = C.hadamard_quant_act(xs, None, 1e-6, c.get("had_block", 0))
+        C.linear(q, s, qw, s_w)
+        return len(rows)
+
+    step()                                           # warm-up
+    t0 = time.perf_counter()
+    tokens, n = 0, 0
+    while True:
+        tokens += step()
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": C.threads(), "kind": "oracle (C++, OpenMP)",
+            "sample": f"{n} oracle steps of {len(rows)} tokens of {c['name']} (C++ oracle, OpenMP over tokens "
+                      f"and output rows)"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -685,6 +717,10 @@ def main():
             line = run_ours(args, rank, world, local_rank)
             if line is not None and world == 1 and not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline(WORKLOADS[args.workload]())
+                try:
+                    line["cpu_baseline_all_cores"] = cpu_baseline_omp(WORKLOADS[args.workload]())
+                except Exception as e:                   # e.g. no C++ compiler on the host
+                    line["cpu_baseline_all_cores"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
         if line is not None:
             print(json.dumps(line), flush=True)
     finally:

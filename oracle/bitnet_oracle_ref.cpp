@@ -4,7 +4,10 @@
 // It shares no code with the CUDA path or with the numpy oracle; the tests
 // require the two oracles to agree bit for bit, so a slip in either shows.
 // Built with -O2 -ffp-contract=off and no fast-math: every float operation is
-// one IEEE-754 round-to-nearest-even operation, as written.
+// one IEEE-754 round-to-nearest-even operation, as written.  With -fopenmp the
+// loops over tokens and output rows run on all cores; every element is still
+// computed by the same operations in the same order, so the results do not
+// change.
 //
 // Sources, by page title and section:
 //  "LLM을 1.58비트로 파인튜닝: BitNet을 이용한 극단적인 양자화", section 양자화
@@ -24,6 +27,9 @@
 #include <cstdint>
 #include <cstring>
 #include <vector>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 namespace {
 
@@ -100,6 +106,15 @@ int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
 
 extern "C" {
 
+// threads the row loops use
+int oc_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
 // sum |w| exactly, then one rounding to double.
 double oc_exact_sum_abs(const float* w, int64_t n) {
   BigSum acc;
@@ -160,8 +175,9 @@ void oc_pack_trit5(const int8_t* q, int64_t N, int64_t K, int64_t row_bytes, uin
 // y = (x * r) * gamma with r = 1 / sqrt(sum(x*x) / K + eps), the sum by the
 // balanced pairwise tree
 void oc_rms_norm(const float* x, int64_t M, int64_t K, const float* gamma, float eps, float* y, float* r_out) {
-  std::vector<float> sq((size_t)K);
+#pragma omp parallel for schedule(static)
   for (int64_t m = 0; m < M; ++m) {
+    std::vector<float> sq((size_t)K);
     const float* row = x + m * K;
     for (int64_t k = 0; k < K; ++k) sq[(size_t)k] = row[k] * row[k];
     const float ms = pairwise_sum(sq.data(), K) / (float)K;
@@ -177,6 +193,7 @@ void oc_rms_norm(const float* x, int64_t M, int64_t K, const float* gamma, float
 
 // s = qmax / max(max|y|, 1e-5); q = clamp(rint(y * s), qmin, qmax)
 void oc_absmax_quantize(const float* y, int64_t M, int64_t K, int qmax, int qmin, int8_t* q, float* s) {
+#pragma omp parallel for schedule(static)
   for (int64_t m = 0; m < M; ++m) {
     float amax = 0.0f;
     for (int64_t k = 0; k < K; ++k) amax = std::fabs(y[m * K + k]) > amax ? std::fabs(y[m * K + k]) : amax;
@@ -192,6 +209,7 @@ void oc_absmax_quantize(const float* y, int64_t M, int64_t K, int qmax, int qmin
 // then every value times fp32(1 / sqrt(block))
 void oc_hadamard(float* y, int64_t M, int64_t K, int64_t block) {
   const float c = (float)(1.0 / std::sqrt((double)block));
+#pragma omp parallel for schedule(static)
   for (int64_t m = 0; m < M; ++m)
     for (int64_t b0 = 0; b0 < K; b0 += block) {
       float* u = y + m * K + b0;
@@ -215,6 +233,7 @@ void oc_pack_int4(const int8_t* q, int64_t M, int64_t K, uint8_t* pk) {
 
 // acc[m][n] = sum_k qx[m][k] * qw[n][k] in 64-bit integers
 void oc_int_matmul(const int8_t* qx, const int8_t* qw, int64_t M, int64_t N, int64_t K, int64_t* acc) {
+#pragma omp parallel for collapse(2) schedule(static)
   for (int64_t m = 0; m < M; ++m)
     for (int64_t n = 0; n < N; ++n) {
       int64_t s = 0;
@@ -226,6 +245,7 @@ void oc_int_matmul(const int8_t* qx, const int8_t* qw, int64_t M, int64_t N, int
 // y = float(acc) * ((1 / s_x) * (1 / s_w)) in fp32
 void oc_dequantize(const int64_t* acc, int64_t M, int64_t N, const float* s_x, float s_w, float* y) {
   const float rw = 1.0f / s_w;
+#pragma omp parallel for schedule(static)
   for (int64_t m = 0; m < M; ++m) {
     const float dq = (1.0f / s_x[m]) * rw;
     for (int64_t n = 0; n < N; ++n) y[m * N + n] = (float)acc[m * N + n] * dq;

@@ -1,8 +1,9 @@
 """numpy-facing binding of the plain C++ oracle (bitnet_oracle_ref.cpp).
 
-TEST INFRASTRUCTURE: only tests/ use it, to hold the numpy oracle and the C++
-one to the same bits.  build() compiles the library with g++ in-tree
-(oracle/_build), with -ffp-contract=off and no fast-math.
+TEST INFRASTRUCTURE: only tests/ (which hold the numpy oracle and the C++ one
+to the same bits) and bench.py's CPU-baseline leg use it.  build() compiles the library with g++ in-tree
+(oracle/_build), with -ffp-contract=off, no fast-math, and OpenMP over tokens
+and output rows (which changes no result).
 """
 from __future__ import annotations
 
@@ -17,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "bitnet_oracle_ref.cpp")
 OUT_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(OUT_DIR, "libbitnet_oracle_ref.so")
-FLAGS = ["-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+FLAGS = ["-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared"]
 
 _lib = None
 
@@ -39,6 +40,7 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(build())
         P, I64, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
         sig = {
+            "oc_threads": (ctypes.c_int, []),
             "oc_exact_sum_abs": (ctypes.c_double, [P, I64]),
             "oc_weight_scale": (None, [P, I64, P, P]),
             "oc_ternarize": (None, [P, I64, F, P]),
@@ -56,6 +58,10 @@ def lib() -> ctypes.CDLL:
             fn.restype, fn.argtypes = res, args
         _lib = L
     return _lib
+
+
+def threads() -> int:
+    return int(lib().oc_threads())
 
 
 def _p(a):

@@ -69,3 +69,10 @@ def test_profiled_traffic_only_for_current_sources(tmp_path, monkeypatch):
     (csrc / "a.cu").write_text("// kernel a, changed\n")
     assert bench.kernel_source_hash() != h
     assert bench.profiled_traffic("linear_x") is None
+
+
+def test_all_cores_cpu_baseline_line():
+    c = bench.WORKLOADS["tiny"]()
+    r = bench.cpu_baseline_omp(c, budget_s=0.2)
+    assert r["value"] > 0 and r["unit"] == "tokens/s" and r["cores"] >= 1
+    assert r["kind"] == "oracle (C++, OpenMP)" and c["name"] in r["sample"]
