@@ -149,3 +149,31 @@ def test_linear_path_selector(L):
     assert L.bitnet_set_linear_path(3) == 0
     assert L.bitnet_set_linear_path(-1) == 2
     assert L.bitnet_set_linear_path(0) == 0
+
+
+def test_oracle_and_product_share_no_code():
+    """The product package never imports the oracle, the oracle never imports the
+    product, and the C++ oracle includes nothing from the CUDA sources."""
+    import ast
+    import glob
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+    def imports(path):
+        tree = ast.parse(open(path).read())
+        names = set()
+        for node in ast.walk(tree):
+            if isinstance(node, ast.Import):
+                names.update(a.name.split(".")[0] for a in node.names)
+            elif isinstance(node, ast.ImportFrom) and node.module:
+                names.add(node.module.split(".")[0])
+        return names
+
+    for path in glob.glob(os.path.join(root, "bitlinear_bitnet_quant_b200", "*.py")):
+        assert "oracle" not in imports(path), path
+    for path in glob.glob(os.path.join(root, "oracle", "*.py")):
+        assert "bitlinear_bitnet_quant_b200" not in imports(path), path
+    cpp = open(os.path.join(root, "oracle", "bitnet_oracle_ref.cpp")).read()
+    assert "csrc" not in cpp and ".cuh" not in cpp and "bitnet.h" not in cpp
+    for path in glob.glob(os.path.join(root, "bitlinear_bitnet_quant_b200", "csrc", "*")):
+        assert "oracle" not in open(path).read().lower(), path
