@@ -1,7 +1,6 @@
 """Host-side checks of the C ABI that need no GPU: the library loads, exports
 every function include/bitnet.h declares, and rejects bad arguments on the
 host before touching CUDA (no compute call is made here)."""
-import ctypes
 
 import pytest
 

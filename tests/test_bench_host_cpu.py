@@ -5,7 +5,6 @@ sources."""
 import os
 import shutil
 import stat
-import sys
 import time
 
 import pytest
