@@ -158,6 +158,7 @@ MUTATIONS = {
 }
 
 
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")      # planted mistakes may divide by zero
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_mutation_is_caught(name, monkeypatch):
     attr, fn = MUTATIONS[name]
