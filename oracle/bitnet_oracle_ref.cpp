@@ -252,4 +252,17 @@ void oc_dequantize(const int64_t* acc, int64_t M, int64_t N, const float* s_x, f
   }
 }
 
+// a = (g * g) * up with g = max(gate, 0), fp32 (squared-ReLU gated unit)
+void oc_relu2_glu(const float* gate, const float* up, int64_t n, float* a) {
+  for (int64_t i = 0; i < n; ++i) {
+    const float g = gate[i] > 0.0f ? gate[i] : 0.0f;
+    a[i] = (g * g) * up[i];
+  }
+}
+
+// out = a + b, fp32 (residual adds)
+void oc_add(const float* a, const float* b, int64_t n, float* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = a[i] + b[i];
+}
+
 }  // extern "C"

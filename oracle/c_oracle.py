@@ -52,6 +52,8 @@ def lib() -> ctypes.CDLL:
             "oc_pack_int4": (None, [P, I64, I64, P]),
             "oc_int_matmul": (None, [P, P, I64, I64, I64, P]),
             "oc_dequantize": (None, [P, I64, I64, P, F, P]),
+            "oc_relu2_glu": (None, [P, P, I64, P]),
+            "oc_add": (None, [P, P, I64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -142,3 +144,37 @@ def linear(qx, s_x, qw, s_w):
     y = np.empty((M, N), np.float32)
     lib().oc_dequantize(_p(acc), M, N, _p(s_x), float(s_w), _p(y))
     return acc, y
+
+
+def relu2_glu(gate, up):
+    gate, up = _c(gate, np.float32), _c(up, np.float32)
+    a = np.empty_like(gate)
+    lib().oc_relu2_glu(_p(gate), _p(up), gate.size, _p(a))
+    return a
+
+
+def add(a, b):
+    a, b = _c(a, np.float32), _c(b, np.float32)
+    out = np.empty_like(a)
+    lib().oc_add(_p(a), _p(b), a.size, _p(out))
+    return out
+
+
+def chain_layer(x, layer: dict, eps: float = 1e-6):
+    """One layer of the stacked chain from the C++ primitives; layer[name] = (codes, s_w).
+    Q/K/V/up/gate take int8 activations, O and down int4 after the Hadamard transform;
+    O's input is V's output (attention over one token); residual adds in fp32."""
+    x = _c(x, np.float32)
+    qx, sx = quant_act(x, None, eps)
+    y = {}
+    for name in ("q", "k", "v"):
+        _, y[name] = linear(qx, sx, *layer[name])
+    _, so, co, _ = hadamard_quant_act(y["v"], None, eps)
+    _, o = linear(co, so, *layer["o"])
+    h = add(x, o)
+    qh, sh = quant_act(h, None, eps)
+    _, up = linear(qh, sh, *layer["up"])
+    _, gate = linear(qh, sh, *layer["gate"])
+    _, sd, cd, _ = hadamard_quant_act(relu2_glu(gate, up), None, eps)
+    _, d = linear(cd, sd, *layer["down"])
+    return add(h, d)

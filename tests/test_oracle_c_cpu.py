@@ -65,3 +65,18 @@ def test_linear_agrees():
 def test_trit5_agrees(N, K):
     q = np.random.default_rng(N + K).integers(-1, 2, size=(N, K)).astype(np.int8)
     assert np.array_equal(C.pack_trit5(q, O.trit5_row_bytes(K)), O.pack_trit5(q))
+
+
+def test_chain_layer_agrees():
+    """One stacked layer (int8 and int4 projections, squared-ReLU GLU, fp32
+    residuals) at a reduced width, through both oracles."""
+    H, F = 256, 704                                  # 704 = 11 blocks of 64 for the Hadamard
+    shapes = {"q": (H, H), "k": (H, H), "v": (H, H), "o": (H, H), "up": (F, H), "gate": (F, H), "down": (H, F)}
+    layer = {}
+    for i, (name, (n, k)) in enumerate(sorted(shapes.items())):
+        _, s_w, q = O.quantize_weights(wl.weights(n, k, seed=i))
+        layer[name] = (q, s_w)
+    x = wl.gaussian(np.random.default_rng(4), (6, H))
+    y_o = O.chain_layer(x, layer)
+    y_c = C.chain_layer(x, layer)
+    assert np.array_equal(_bits(y_c), _bits(y_o))
