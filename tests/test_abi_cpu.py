@@ -176,3 +176,29 @@ def test_oracle_and_product_share_no_code():
     assert "csrc" not in cpp and ".cuh" not in cpp and "bitnet.h" not in cpp
     for path in glob.glob(os.path.join(root, "bitlinear_bitnet_quant_b200", "csrc", "*")):
         assert "oracle" not in open(path).read().lower(), path
+
+
+def test_python_binding_refuses_host_tensors():
+    """No CPU fallback: every compute entry of the binding refuses host tensors
+    before anything runs."""
+    import torch
+    from bitlinear_bitnet_quant_b200 import api
+    x = torch.zeros(4, 512)
+    w = torch.zeros(256, 512)
+    pk = torch.zeros(256, 128, dtype=torch.uint8)
+    sw = torch.ones(1)
+    xq = torch.zeros(4, 512, dtype=torch.int8)
+    sx = torch.ones(4)
+    calls = [
+        lambda: api.bitnet_quantize_weights(w),
+        lambda: api.bitnet_quant_act(x),
+        lambda: api.bitnet_hadamard_quant_act(x),
+        lambda: api.bitnet_linear(xq, 8, sx, pk, sw),
+        lambda: api.bitnet_bitlinear(x, pk, sw),
+        lambda: api.bitnet_repack_trit5(pk),
+        lambda: api.bitnet_linear_trit5(xq, 8, sx, torch.zeros(256, 112, dtype=torch.uint8), sw, 512),
+        lambda: api.bitlinear_forward(x, pk, sw),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            call()
