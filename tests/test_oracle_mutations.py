@@ -135,6 +135,51 @@ def _trit5_offset_minus(q):
     return sum(d[:, :, i] * 3 ** i for i in range(5)).astype(np.uint8)
 
 
+def _glu_no_square(gate, up):
+    """relu(gate) * up: the square dropped."""
+    return np.maximum(np.asarray(gate, np.float32), F32(0.0)) * np.asarray(up, np.float32)
+
+
+def _glu_gate_up_swapped(gate, up):
+    return _orig["squared_relu_glu"](up, gate)
+
+
+def _glu_abs_instead_of_relu(gate, up):
+    g = np.abs(np.asarray(gate, np.float32))
+    return (g * g) * np.asarray(up, np.float32)
+
+
+def _chain_o_from_q(x, layer, eps=O.DEFAULT_EPS):
+    """The O projection fed from Q instead of V."""
+    swapped = dict(layer)
+    swapped["v"] = layer["q"]
+    return _orig["chain_layer"](x, swapped, eps)
+
+
+def _chain_no_attention_residual(x, layer, eps=O.DEFAULT_EPS):
+    """The attention residual dropped: the FFN runs on o instead of h = x + o."""
+    x = np.asarray(x, np.float32)
+    qx, sx = O.quant_act(x, None, eps)
+    _, v = O.linear(qx, sx, *layer["v"])
+    _, so, co, _ = O.hadamard_quant_act(v, None, eps)
+    _, o = O.linear(co, so, *layer["o"])
+    h = o
+    qh, sh = O.quant_act(h, None, eps)
+    _, up = O.linear(qh, sh, *layer["up"])
+    _, gate = O.linear(qh, sh, *layer["gate"])
+    _, sd, cd, _ = O.hadamard_quant_act(O.squared_relu_glu(gate, up), None, eps)
+    _, d = O.linear(cd, sd, *layer["down"])
+    return x + o + d
+
+
+def _bf16_truncate(y):
+    return (np.ascontiguousarray(y, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _bf16_ties_away(y):
+    u = np.ascontiguousarray(y, np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x8000) >> 16).astype(np.uint16)
+
 
 MUTATIONS = {
     "absmax_numerator_128": ("absmax_quantize", _absmax_128),
@@ -155,6 +200,13 @@ MUTATIONS = {
     "dequant_multiplies": ("dequantize", _dequant_times),
     "trit5_digits_reversed": ("pack_trit5", _trit5_digits_reversed),
     "trit5_digit_offset": ("pack_trit5", _trit5_offset_minus),
+    "glu_no_square": ("squared_relu_glu", _glu_no_square),
+    "glu_gate_up_swapped": ("squared_relu_glu", _glu_gate_up_swapped),
+    "glu_abs_not_relu": ("squared_relu_glu", _glu_abs_instead_of_relu),
+    "chain_o_from_q": ("chain_layer", _chain_o_from_q),
+    "chain_drops_residual": ("chain_layer", _chain_no_attention_residual),
+    "bf16_truncates": ("bf16_round", _bf16_truncate),
+    "bf16_ties_away": ("bf16_round", _bf16_ties_away),
 }
 
 

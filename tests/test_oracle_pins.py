@@ -322,6 +322,59 @@ def check_chain_zero_weights_is_identity():
     assert np.array_equal(O.chain_layer(x, layer), x)
 
 
+def check_squared_relu_glu_golden():
+    gate, up, want = [], [], []
+    for row in _golden("squared_relu_glu_cases.txt"):
+        lhs, rhs = row.split(";")
+        g, u = lhs.split()
+        gate.append(float(g))
+        up.append(float(u))
+        want.append(float(rhs))
+    got = O.squared_relu_glu(np.array([gate], np.float32), np.array([up], np.float32))
+    assert got.dtype == np.float32
+    assert np.array_equal(got[0], np.array(want, np.float32)), (got, want)
+
+
+def check_bf16_round_golden():
+    src, want = [], []
+    for row in _golden("bf16_rne_cases.txt"):
+        a, b = row.split()
+        src.append(int(a, 16))
+        want.append(int(b, 16))
+    got = O.bf16_round(np.array(src, np.uint32).view(np.float32))
+    assert [int(v) for v in got] == want, [hex(int(v)) for v in got]
+
+
+def _tiny_chain_layer():
+    """The hand-built layer of tests/golden/chain_layer_tiny.txt: (codes, s_w = 1) per projection."""
+    H = F = 16
+    n = np.arange(16)
+    z = lambda r, c: np.zeros((r, c), np.int8)
+    wq, wk, wv, wo = z(H, H), z(H, H), z(H, H), z(H, H)
+    wup, wgate, wdown = z(F, H), z(F, H), z(H, F)
+    wq[:, 0] = np.where(n % 2 == 0, 1, -1)
+    wk[:, 0] = np.where(n % 4 < 2, 1, -1)
+    wv[:, 0] = 1
+    wo[:, 1] = 1
+    wo[:, 2] = 1
+    wup[:, 0] = 1
+    wgate[:, 0] = 1
+    wgate[n % 2 == 1, 1] = 1
+    wdown[:, 1] = np.where(n % 2 == 0, 1, -1)
+    wdown[:8, 0] = 1
+    one = np.float32(1.0)
+    return {"q": (wq, one), "k": (wk, one), "v": (wv, one), "o": (wo, one),
+            "up": (wup, one), "gate": (wgate, one), "down": (wdown, one)}
+
+
+def check_chain_layer_tiny_golden():
+    want = np.array([float(r.split()[1]) for r in _golden("chain_layer_tiny.txt")])
+    x = np.ones((1, 16), np.float32)
+    got = O.chain_layer(x, _tiny_chain_layer())
+    assert got.shape == (1, 16) and got.dtype == np.float32
+    assert np.max(np.abs(got[0] - want) / np.abs(want)) < 1e-5, (got, want)
+
+
 CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]
 
 
