@@ -1,21 +1,35 @@
 """Benchmark of the BitLinear hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|hbitlinear|tiny]
-                    [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all|<name>]
+                    [--impl ours|reference] [--min-time S] [--no-cpu-baseline]
 
-One step = one BitLinear forward over one batch: the activation quantiser
-(RMSNorm + absmax int8, or RMSNorm + Hadamard + int4) and the ternary product
-with its dequantisation.  Weights are quantised offline, outside the timed
-region.  The default workload is the decode GEMV: X bf16 [16, 2560],
-W ternary [6912, 2560].  Rank 0 prints one JSON line.
+With no --workload every configuration runs in one invocation, and rank 0
+prints one JSON line.  Its top-level keys describe the headline: the largest
+configuration, 24 stacked BitLinear layers (hidden 2048, FFN 5632) on a
+512-token prefill batch.  The key "configs" holds one object per other
+configuration (tiny BitLinear, decode GEMV at 1, 4 and 16 tokens, batched
+prefill GEMM, the H-BitLinear a4 layer, the chain at 32 decode tokens), each
+with its own throughput, roofline, cpu_baseline and e2e.
 
-Device timing: the K timed steps are captured in one CUDA graph and replayed
-between CUDA events on the launching stream, with a barrier and a device
-synchronise on both sides; each step reads the next of a ring of weight copies
-whose total size exceeds twice the 126 MB L2.  The dominant kernel is timed the
-same way on its own for the roofline.  e2e: the same steps through the Python
-API with pinned host input/output buffers, the host<->device copies inside the
-timed region.  The CPU oracle is timed on a bounded sample on the host.
+A step is one pass of the whole path over one batch: for a single layer the
+activation quantiser (RMSNorm + absmax int8, or RMSNorm + Hadamard + int4) and
+the ternary product with its dequantisation; for the chain every quantiser,
+product and element-wise step of all 24 layers.  Weights are quantised
+offline, outside the timed region.
+
+Device timing: the K steps are captured in one CUDA graph.  The timed region
+is R back-to-back replays of that graph (R chosen so the region lasts at
+least --min-time seconds), between a barrier and a device synchronise on both
+sides; each replay is bracketed by CUDA events on the launching stream.  The
+step time is the median replay time / K (max over ranks), with the spread
+over replays reported.  Every single-layer step reads the next of a ring of
+weight (and, where the activations are large, activation) copies whose total
+exceeds twice the 126 MB L2; the chain's 308 MB of packed weights exceed it
+by themselves.  The dominant kernel is timed the same way in a graph of its
+own launches for the roofline.  e2e: the same steps through the public Python
+API with pinned host buffers, host<->device copies inside the timed region.
+Clocks are sampled with nvidia-smi during every timed region.  The CPU oracle
+is timed on a bounded sample on the host.
 
 Under torchrun (N > 1) each rank runs its own batches (independent tokens:
 weak scaling, no data-path collective); time is the max over ranks.
@@ -42,23 +56,26 @@ from bitlinear_bitnet_quant_b200 import workloads as wl  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_INT8_TOPS = 4500.0
 METRIC = "BitLinear tokens/sec and GB/s|TOPS vs HBM/int8 roofline, 1xB200"
-
+EPS = 1e-6
 
 # ----------------------------------------------------------------------------
 # workloads
 # ----------------------------------------------------------------------------
 
 WORKLOADS = {
-    "decode": lambda: wl.decode(16, with_weights=False),
-    "decode_m4": lambda: wl.decode(4, with_weights=False),
+    "tiny": lambda: wl.tiny(),
     "decode_m1": lambda: wl.decode(1, with_weights=False),
+    "decode_m4": lambda: wl.decode(4, with_weights=False),
+    "decode_m16": lambda: wl.decode(16, with_weights=False),
     "prefill": lambda: wl.prefill(with_weights=False),
     "hbitlinear": lambda: wl.hbitlinear(with_weights=False),
-    "tiny": lambda: wl.tiny(),
 }
 CHAIN_WORKLOADS = {"chain_decode": 32, "chain_prefill": 512}    # tokens per step
 CHAIN_LAYERS = 24
+ORDER = ["tiny", "decode_m1", "decode_m4", "decode_m16", "prefill", "hbitlinear", "chain_decode", "chain_prefill"]
+HEADLINE = "chain_prefill"
 
 
 def kernel_source_hash() -> str:
@@ -81,6 +98,11 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def int8_peak(peaks) -> float:
+    """Dense int8 peak in TOPS: the measured bf16 burst x the nominal int8 : bf16 ratio (4.5 : 2.25)."""
+    return 2.0 * float(peaks["bf16_tflops"])
+
+
 def profiled_traffic(kernel_tag: str):
     """Per-launch DRAM bytes from the committed ncu summary, if it was taken
     on the current kernel sources (else None)."""
@@ -100,31 +122,53 @@ def profiled_traffic(kernel_tag: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled in the background; each
+    sample carries the host time it arrived, so a window can be summarised."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: str, period_ms: int = 100):
         self.gpu = gpu_index
+        self.period_ms = period_ms
         self.proc = None
-        self.lines = []
+        self.samples = []            # (host time, sm MHz, max MHz, reasons)
         self.thread = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(self.period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except Exception:
             self.proc = None
+        return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            f = [x.strip() for x in line.strip().split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm, mx = float(f[1]), float(f[2])
+            except ValueError:
+                continue
+            reasons = {n for n, v in zip(self.REASONS, f[5:9]) if v.lower().startswith("active")}
+            self.samples.append((time.monotonic(), sm, mx, reasons))
+
+    def summary(self, t0=None, t1=None):
+        sel = [s for s in self.samples if (t0 is None or s[0] >= t0) and (t1 is None or s[0] <= t1)]
+        if not sel:
+            return None
+        reasons = set()
+        for s in sel:
+            reasons |= s[3]
+        return {"sm_mhz": statistics.median(s[1] for s in sel), "sm_max_mhz": max(s[2] for s in sel),
+                "reasons": sorted(reasons), "samples": len(sel)}
 
     def stop(self):
         if self.proc is None:
@@ -137,28 +181,11 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=1)
-        sm, mx, reasons = [], 0.0, set()
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = max(mx, float(f[2]))
-            except ValueError:
-                continue
-            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
-                                 f[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return self.summary()
 
 
 # ----------------------------------------------------------------------------
-# our implementation
+# device timing
 # ----------------------------------------------------------------------------
 
 def max_over_ranks(ms: float, world: int, dev) -> float:
@@ -172,45 +199,109 @@ def max_over_ranks(ms: float, world: int, dev) -> float:
     return float(t.item())
 
 
-def timed_replay(g, stream, world, dev) -> float:
-    """One warm replay, then a timed replay between CUDA events on the
-    launching stream, with a barrier and a device synchronise on both sides."""
+class Timer:
+    """Times CUDA graphs of K steps: R replays (at least min_time seconds in
+    all) between a barrier and a device synchronise on both sides, CUDA events
+    around each replay on the launching stream."""
+
+    def __init__(self, stream, world, dev, steps, min_time_s, clocks):
+        self.stream, self.world, self.dev = stream, world, dev
+        self.steps, self.min_time_s, self.clocks = steps, min_time_s, clocks
+        self.windows = []
+
+    def graph(self, fn, count=None):
+        import torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            for i in range(self.steps if count is None else count):
+                fn(i)
+        return g
+
+    def time(self, g, count=None):
+        """Returns dict(ms per step: median / min / max over replays, replays)."""
+        import torch
+        import torch.distributed as dist
+        count = self.steps if count is None else count
+        g.replay()
+        torch.cuda.synchronize()
+        if self.world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_host0 = time.monotonic()
+        events = []
+        batch = 1
+        while True:
+            for _ in range(batch):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(self.stream)
+                g.replay()
+                e1.record(self.stream)
+                events.append((e0, e1))
+            torch.cuda.synchronize()
+            if time.monotonic() - t_host0 >= self.min_time_s or len(events) >= 100000:
+                break
+            batch = min(2 * batch, 4096)
+        t_host1 = time.monotonic()
+        if self.world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        per = sorted(e0.elapsed_time(e1) / count for e0, e1 in events)
+        med = max_over_ranks(statistics.median(per), self.world, self.dev)
+        self.windows.append((t_host0, t_host1))
+        return {"ms": med, "min_ms": per[0], "max_ms": per[-1], "replays": len(per), "steps_per_replay": count,
+                "window": (t_host0, t_host1)}
+
+
+def spread(t):
+    return {"replays": t["replays"], "steps_per_replay": t["steps_per_replay"], "median_ms_per_step": t["ms"],
+            "min_ms_per_step": t["min_ms"], "max_ms_per_step": t["max_ms"]}
+
+
+def e2e_time(step_fn, stream, world, dev, steps, min_time_s):
+    """Seconds per step of step_fn run eagerly (host copies included), at least
+    `steps` steps and min_time_s seconds, between CUDA events."""
     import torch
     import torch.distributed as dist
-    g.replay()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.monotonic()
+    n = 0
     e0.record(stream)
-    g.replay()
+    while n < steps or time.monotonic() - t0 < min_time_s:
+        step_fn(n)
+        n += 1
+        if n % 64 == 0:
+            stream.synchronize()
     e1.record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    return max_over_ranks(e0.elapsed_time(e1), world, dev)
+    return max_over_ranks(e0.elapsed_time(e1) / n, world, dev) / 1e3
 
 
-def run_ours(args, rank, world, local_rank):
+def to_device_x(c, dev):
     import torch
-    import torch.distributed as dist
+    if c["x_dtype"] == "bf16":
+        return torch.from_numpy(c["x"].view(np.int16)).view(torch.bfloat16).to(dev)
+    return torch.from_numpy(c["x"]).to(dev)
 
-    from bitlinear_bitnet_quant_b200 import api, build_lib
 
-    build_lib.build()
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    stream = torch.cuda.Stream(device=dev)
-    torch.cuda.set_stream(stream)
+# ----------------------------------------------------------------------------
+# our implementation: one BitLinear layer
+# ----------------------------------------------------------------------------
 
-    c = WORKLOADS[args.workload]()
+def run_layer(name, args, ctx):
+    import torch
+
+    api, rank, world, dev, stream, timer = ctx["api"], ctx["rank"], ctx["world"], ctx["dev"], ctx["stream"], \
+        ctx["timer"]
+    c = WORKLOADS[name]()
     M, K, N, bits = c["M"], c["K"], c["N"], c["act_bits"]
-    eps = 1e-6
-    out_dtype = torch.bfloat16 if args.workload == "prefill" else torch.float32
+    had_block = c.get("had_block", 0)
+    out_dtype = torch.bfloat16 if name == "prefill" else torch.float32
     out_bytes = 2 if out_dtype == torch.bfloat16 else 4
 
-    # ---- weights: quantised offline, a ring of copies larger than 2x L2 ----
+    # weights, quantised offline: a ring of copies larger than 2x L2
     packed_bytes = N * K // 4
     copies = max(2, min(64, math.ceil(2.2 * L2_BYTES / packed_bytes)))
     rng = np.random.default_rng(1234 + rank)
@@ -218,242 +309,192 @@ def run_ours(args, rank, world, local_rank):
     ring = []
     for i in range(copies):
         w = base_w if i == 0 else base_w[torch.from_numpy(rng.permutation(N)).to(dev)]
-        pk, s_w = api.bitnet_quantize_weights(w.contiguous())
-        ring.append((pk, s_w))
+        ring.append(api.bitnet_quantize_weights(w.contiguous(), stream=stream))
     del base_w
+    # activations: a ring too when one input is a sizeable part of the L2
+    x0 = to_device_x(c, dev)
+    x_bytes = x0.numel() * x0.element_size()
+    xcopies = 1 if x_bytes * 8 < L2_BYTES else max(2, math.ceil(2.2 * L2_BYTES / x_bytes))
+    xring = [x0] + [x0[torch.from_numpy(rng.permutation(M)).to(dev)].contiguous() for _ in range(xcopies - 1)]
     torch.cuda.synchronize()
 
-    x_host = c["x"]
-    if c["x_dtype"] == "bf16":
-        x = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).to(dev)
-    else:
-        x = torch.from_numpy(x_host).to(dev)
-    # preallocated outputs (the graph reuses them)
-    if bits == 8:
-        xq = torch.empty((M, K), dtype=torch.int8, device=dev)
-    else:
-        xq = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    xq = torch.empty((M, K) if bits == 8 else (M, K // 2), dtype=torch.int8 if bits == 8 else torch.uint8,
+                     device=dev)
     s_x = torch.empty((M,), dtype=torch.float32, device=dev)
     Y = torch.empty((M, N), dtype=out_dtype, device=dev)
 
-    def quant():
+    def quant(i):
+        x = xring[i % xcopies]
         if bits == 8:
-            api.bitnet_quant_act(x, None, eps, Xq=xq, s_x=s_x, stream=stream)
+            api.bitnet_quant_act(x, None, EPS, Xq=xq, s_x=s_x, stream=stream)
         else:
-            api.bitnet_hadamard_quant_act(x, None, eps, c.get("had_block", 0), Xq4=xq, s_x=s_x, stream=stream)
+            api.bitnet_hadamard_quant_act(x, None, EPS, had_block, Xq4=xq, s_x=s_x, stream=stream)
 
     def linear(i):
         pk, s_w = ring[i % copies]
         api.bitnet_linear(xq, bits, s_x, pk, s_w, Y=Y, stream=stream)
 
-    # the step is the quantiser and the linear kernel (the single-kernel path
-    # of bitnet_bitlinear is slower on B200; the decode sweep reports it)
     def step(i):
-        quant()
+        quant(i)
         linear(i)
 
     warmup = max(3, args.warmup)
     for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
+    t_step = timer.time(timer.graph(step))
+    t_lin = timer.time(timer.graph(linear))
+    t_q = timer.time(timer.graph(quant))
 
-    def graph_of(fn, count):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(count):
-                fn(i)
-        return g
-
-    def timed(g):
-        return timed_replay(g, stream, world, dev)
-
-    steps = args.steps
-    g_step = graph_of(step, steps)
-    g_lin = graph_of(linear, steps)
-    g_q = graph_of(lambda i: quant(), steps)
-
-    visible = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
-    clocks = ClockSampler(visible[local_rank] if local_rank < len(visible) else str(local_rank))
-    clocks.start()
-    t_step = timed(g_step)
-    t_lin = timed(g_lin)
-    t_q = timed(g_q)
-    clk = clocks.stop()
-
-    # ---- e2e through the public API with pinned host buffers ----
-    x_pin = torch.empty_like(x, device="cpu").pin_memory()
-    x_pin.copy_(x.cpu())
+    # e2e through the public API: pinned host input in, host output back
+    x_pin = torch.empty_like(x0, device="cpu").pin_memory()
+    x_pin.copy_(x0.cpu())
+    x_dev = torch.empty_like(x0)
     y_pin = torch.empty((M, N), dtype=out_dtype).pin_memory()
-    h2d = x_pin.numel() * x_pin.element_size()
-    d2h = y_pin.numel() * y_pin.element_size()
 
     def e2e_step(i):
-        x.copy_(x_pin, non_blocking=True)
+        x_dev.copy_(x_pin, non_blocking=True)
         pk, s_w = ring[i % copies]
-        Yo = api.bitlinear_forward(x, pk, s_w, act_bits=bits, eps=eps, had_block=c.get("had_block", 0),
+        Yo = api.bitlinear_forward(x_dev, pk, s_w, act_bits=bits, eps=EPS, had_block=had_block,
                                    out_dtype=out_dtype, Y=Y, Xq=xq, s_x=s_x, stream=stream)
         y_pin.copy_(Yo, non_blocking=True)
 
     for i in range(warmup):
         e2e_step(i)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(steps):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    t_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    t_e2e = e2e_time(e2e_step, stream, world, dev, args.steps, args.min_time / 2)
 
-    # the offline weight path (absmean ternarisation + packing) on fp32 weights of this layer's
-    # shape, timed on its own: it is not part of a forward step
-    wq = None
-    if args.workload in ("decode", "prefill", "hbitlinear"):
-        w32 = torch.from_numpy(wl.weights(N, K, seed=rank + 7)).to(dev)
-        pk_o = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
-        sw_o = torch.empty((1,), dtype=torch.float32, device=dev)
-        ws_o = torch.empty((api.bitnet_quantize_weights_workspace_size(N, K),), dtype=torch.uint8, device=dev)
-        for _ in range(3):
-            api.bitnet_quantize_weights(w32, pkW=pk_o, s_w=sw_o, workspace=ws_o, stream=stream)
-        reps = 10
-        t_wq = timed(graph_of(lambda i: api.bitnet_quantize_weights(w32, pkW=pk_o, s_w=sw_o, workspace=ws_o,
-                                                                    stream=stream), reps)) / reps / 1e3
-        wbytes = N * K * 4 * 2 + N * K // 4 + 4          # fp32 weights read twice (mean, codes), packed written
-        wq = {"us": t_wq * 1e6, "achieved_GBs": wbytes / t_wq / 1e9, "frac": wbytes / t_wq / 1e9 /
-              load_peaks()[0]["hbm_gbs"], "algorithmic_bytes": wbytes, "weights": N * K, "input": "fp32"}
-        del w32
-
-    # decode: the same weight ring at the other decode batch sizes (linear launches only)
-    sweep = []
-    if args.workload == "decode":
-        # the same weights five per byte (1.6 bits per weight), repacked on the GPU
-        ring5 = [api.bitnet_repack_trit5(pk, stream=stream) for pk, _ in ring]
-        torch.cuda.synchronize()
-        r5_bytes = N * api.bitnet_trit5_row_bytes(K)
-        for Ms in (1, 4, 16):
-            cs = wl.decode(Ms, with_weights=False)
-            xs = torch.from_numpy(cs["x"].view(np.int16)).view(torch.bfloat16).to(dev)
-            xqs = torch.empty((Ms, K), dtype=torch.int8, device=dev)
-            sxs = torch.empty((Ms,), dtype=torch.float32, device=dev)
-            Ys = torch.empty((Ms, N), dtype=out_dtype, device=dev)
-            api.bitnet_quant_act(xs, None, eps, Xq=xqs, s_x=sxs, stream=stream)
-
-            def lin_s(i, xqs=xqs, sxs=sxs, Ys=Ys):
-                pk, s_w = ring[i % copies]
-                api.bitnet_linear(xqs, 8, sxs, pk, s_w, Y=Ys, stream=stream)
-
-            def fused_s(i, xs=xs, xqs=xqs, sxs=sxs, Ys=Ys):
-                pk, s_w = ring[i % copies]
-                api.bitnet_bitlinear(xs, pk, s_w, None, eps, Y=Ys, Xq=xqs, s_x=sxs, stream=stream)
-
-            def lin5_s(i, xqs=xqs, sxs=sxs, Ys=Ys):
-                api.bitnet_linear_trit5(xqs, 8, sxs, ring5[i % copies], ring[i % copies][1], K, Y=Ys, stream=stream)
-
-            def step_s(i, xs=xs, xqs=xqs, sxs=sxs, Ys=Ys):
-                api.bitnet_quant_act(xs, None, eps, Xq=xqs, s_x=sxs, stream=stream)
-                lin_s(i)
-
-            api.bitnet_set_linear_path(4)
-            for i in range(warmup):
-                fused_s(i)
-            t_f = timed(graph_of(fused_s, steps)) / steps / 1e3
-            api.bitnet_set_linear_path(0)
-            for i in range(warmup):
-                lin_s(i)
-                step_s(i)
-            t_s = timed(graph_of(lin_s, steps)) / steps / 1e3
-            t_st = timed(graph_of(step_s, steps)) / steps / 1e3
-            for i in range(warmup):
-                lin5_s(i)
-            t_5 = timed(graph_of(lin5_s, steps)) / steps / 1e3
-            hbm = load_peaks()[0]["hbm_gbs"]
-            b = packed_bytes + Ms * K + 4 * Ms + 4 + Ms * N * out_bytes
-            bf = packed_bytes + 2 * Ms * K + Ms * K + 4 * Ms + 4 + Ms * N * out_bytes
-            b5 = r5_bytes + Ms * K + 4 * Ms + 4 + Ms * N * out_bytes
-            sweep.append({"M": Ms, "linear_us": t_s * 1e6, "linear_GBs": b / t_s / 1e9,
-                          "trit5_linear_us": t_5 * 1e6, "trit5_linear_GBs": b5 / t_5 / 1e9,
-                          "trit5_linear_frac": b5 / t_5 / 1e9 / hbm,
-                          "linear_frac": b / t_s / 1e9 / hbm, "step_us": t_st * 1e6, "tokens_per_s": Ms / t_st,
-                          "fused_kernel_us": t_f * 1e6, "fused_kernel_frac": bf / t_f / 1e9 / hbm})
-
-    if rank != 0:
-        return None
-
-    tokens_per_step = M * world
-    value = tokens_per_step * steps / (t_step / 1e3)
-    ms_per_step = t_step / steps
-    peaks, peak_src = load_peaks()
-    lin_s = t_lin / steps / 1e3
-    q_s = t_q / steps / 1e3
+    sub = {"workload": c["name"], "M_tokens": M, "K": K, "N": N, "act_bits": bits, "x_dtype": c["x_dtype"],
+           "out_dtype": "bf16" if out_bytes == 2 else "f32",
+           "l2": (f"ring of {copies} packed-weight copies ({copies * packed_bytes / 1e6:.0f} MB)"
+                  + (f" and {xcopies} activation copies ({xcopies * x_bytes / 1e6:.0f} MB)" if xcopies > 1 else "")
+                  + ": > 2x L2")}
+    lin_s = t_lin["ms"] / 1e3
+    q_s = t_q["ms"] / 1e3
+    step_s = t_step["ms"] / 1e3
+    peaks, peak_src = ctx["peaks"]
     x_in_bytes = M * K * (2 if c["x_dtype"] == "bf16" else 4)
     xq_bytes = M * K if bits == 8 else M * K // 2
-    if args.workload.startswith("decode") or args.workload == "tiny":
+    if M <= 32:
         alg_bytes = packed_bytes + xq_bytes + 4 * M + 4 + M * N * out_bytes
         roof = {"bound": "hbm", "achieved": alg_bytes / lin_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "kernel": "bitnet_linear (warp-MMA decode)" if M <= 32 and K % 512 == 0 else "bitnet_linear (tcgen05)",
+                "kernel": "bitnet_linear (warp-MMA decode)" if K % 512 == 0 else "bitnet_linear (tcgen05)",
                 "algorithmic_bytes_per_launch": alg_bytes}
-        tag = f"linear_{args.workload}"
     else:
         ops = 2.0 * M * N * K
-        int8_peak = 2.0 * peaks["bf16_tflops"]          # nominal int8 : bf16 = 4.5 : 2.25
-        roof = {"bound": "tensor", "achieved": ops / lin_s / 1e12, "peak": int8_peak, "unit": "TOPS",
+        roof = {"bound": "tensor", "achieved": ops / lin_s / 1e12, "peak": int8_peak(peaks), "unit": "TOPS",
                 "kernel": "bitnet_linear (tcgen05 kind::i8)", "algorithmic_ops_per_launch": ops,
-                "peak_note": "2 x measured bf16 burst (nominal int8/bf16 ratio)"}
-        tag = f"linear_{args.workload}"
+                "peak_note": "2 x measured bf16 burst (nominal int8 : bf16 ratio)",
+                "frac_of_nominal_4500_tops": ops / lin_s / 1e12 / NOMINAL_INT8_TOPS}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = profiled_traffic(tag)
+    roof["traffic"] = profiled_traffic(f"linear_{name}")
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     quant_bytes = x_in_bytes + xq_bytes + 4 * M
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
-        "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int8xternary->int32" if bits == 8 else "int4xternary->int32",
-        "data": "synthetic",
-        "config": {"workload": c["name"], "M_tokens": M, "K": K, "N": N, "act_bits": bits,
-                   "x_dtype": c["x_dtype"], "out_dtype": "bf16" if out_bytes == 2 else "f32",
-                   "l2": f"ring of {copies} packed-weight copies ({copies * packed_bytes / 1e6:.0f} MB > 2x L2)",
-                   "timing": "CUDA graph of the K steps, CUDA events on the launching stream",
-                   "parallelism": f"dp{world} (independent batches per rank)"},
+    sub.update({
+        "value": M * world / step_s, "unit": "tokens/s", "ms_per_step": t_step["ms"],
+        "timing": spread(t_step),
         "roofline": roof,
-        "kernels_us": {"quant": q_s * 1e6, "linear": lin_s * 1e6},
+        "kernels_us": {"quant": q_s * 1e6, "linear": lin_s * 1e6, "step": step_s * 1e6},
         "quant_roofline": {"bound": "hbm", "achieved": quant_bytes / q_s / 1e9, "peak": peaks["hbm_gbs"],
-                           "unit": "GB/s", "frac": quant_bytes / q_s / 1e9 / peaks["hbm_gbs"]},
-        "e2e": {"value": tokens_per_step * steps / (t_e2e / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * steps,
-        "clocks": clk,
-    }
-    if sweep:
-        line["decode_sweep"] = sweep
-    if wq is not None:
-        line["weights_quant"] = wq
-    return line
+                           "unit": "GB/s", "frac": quant_bytes / q_s / 1e9 / peaks["hbm_gbs"],
+                           "algorithmic_bytes_per_launch": quant_bytes},
+        "e2e": {"value": M * world / t_e2e, "unit": "tokens/s",
+                "h2d_bytes_per_step": x_pin.numel() * x_pin.element_size(),
+                "d2h_bytes_per_step": y_pin.numel() * y_pin.element_size()},
+        "gpu_launches_per_step": 2,
+        "clocks": ctx["clocks"].summary(t_step["window"][0], t_q["window"][1]),
+    })
+
+    if name.startswith("decode"):
+        sub["decode_variants"] = decode_variants(ctx, c, ring, copies, xq, s_x, Y, x0, packed_bytes, out_bytes)
+    if name in ("decode_m16", "prefill", "hbitlinear"):
+        sub["weights_quant"] = weights_quant(ctx, N, K)
+    del ring, xring
+    return sub
 
 
-def run_chain(args, rank, world, local_rank):
-    """24 stacked layers (hidden 2048, FFN 5632) on M tokens per step."""
+def decode_variants(ctx, c, ring, copies, xq, s_x, Y, x0, packed_bytes, out_bytes):
+    """The same decode shape through the single fused kernel and with the
+    weights five per byte (linear launches only), for comparison."""
     import torch
-    import torch.distributed as dist
-
-    from bitlinear_bitnet_quant_b200 import api, build_lib, chain
-
-    build_lib.build()
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    stream = torch.cuda.Stream(device=dev)
-    torch.cuda.set_stream(stream)
-    M = CHAIN_WORKLOADS[args.workload]
-    H, F = wl.CHAIN_HIDDEN, wl.CHAIN_FFN
-    g = torch.Generator(device=dev)
-    g.manual_seed(1000 + rank)
-    layers = []
-    for _ in range(CHAIN_LAYERS):          # N(0, 0.02) weights drawn on the device, quantised offline
-        w = {name: torch.randn((n, k), generator=g, device=dev) * 0.02 for name, n, k, _ in wl.CHAIN_PROJ}
-        layers.append(chain.quantize_layer(w))
-        del w
+    api, stream, timer = ctx["api"], ctx["stream"], ctx["timer"]
+    M, K, N = c["M"], c["K"], c["N"]
+    hbm = ctx["peaks"][0]["hbm_gbs"]
+    ring5 = [api.bitnet_repack_trit5(pk, stream=stream) for pk, _ in ring]
     torch.cuda.synchronize()
+    r5_bytes = N * api.bitnet_trit5_row_bytes(K)
+    Xq2 = torch.empty_like(xq)
+    s_x2 = torch.empty_like(s_x)
+
+    def fused(i):
+        pk, s_w = ring[i % copies]
+        api.bitnet_bitlinear(x0, pk, s_w, None, EPS, Y=Y, Xq=Xq2, s_x=s_x2, stream=stream, kernel=4)
+
+    def lin5(i):
+        api.bitnet_linear_trit5(xq, 8, s_x, ring5[i % copies], ring[i % copies][1], K, Y=Y, stream=stream)
+
+    for i in range(3):
+        fused(i)
+        lin5(i)
+    t_f = timer.time(timer.graph(fused))["ms"] / 1e3
+    t_5 = timer.time(timer.graph(lin5))["ms"] / 1e3
+    bf = packed_bytes + 2 * M * K + M * K + 4 * M + 4 + M * N * out_bytes
+    b5 = r5_bytes + M * K + 4 * M + 4 + M * N * out_bytes
+    del ring5
+    return {"fused_kernel_us": t_f * 1e6, "fused_kernel_frac": bf / t_f / 1e9 / hbm,
+            "trit5_linear_us": t_5 * 1e6, "trit5_linear_frac": b5 / t_5 / 1e9 / hbm,
+            "trit5_algorithmic_bytes": b5}
+
+
+def weights_quant(ctx, N, K):
+    """The offline weight path (absmean ternarisation + packing) on fp32 weights
+    of this layer's shape, timed on its own: it is not part of a step."""
+    import torch
+    api, stream, timer, dev = ctx["api"], ctx["stream"], ctx["timer"], ctx["dev"]
+    w32 = torch.from_numpy(wl.weights(N, K, seed=ctx["rank"] + 7)).to(dev)
+    pk_o = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
+    sw_o = torch.empty((1,), dtype=torch.float32, device=dev)
+    ws_o = torch.empty((api.bitnet_quantize_weights_workspace_size(N, K),), dtype=torch.uint8, device=dev)
+
+    def wq(i):
+        api.bitnet_quantize_weights(w32, pkW=pk_o, s_w=sw_o, workspace=ws_o, stream=stream)
+
+    for i in range(3):
+        wq(i)
+    t = timer.time(timer.graph(wq, 4), 4)["ms"] / 1e3
+    # algorithmic bytes: the fp32 weights read once, the packed codes written once (the
+    # second pass over the weights, for the codes, is counted only where it cannot hit L2)
+    reads = 2 if N * K * 4 > L2_BYTES else 1
+    wbytes = N * K * 4 * reads + N * K // 4 + 4
+    hbm = ctx["peaks"][0]["hbm_gbs"]
+    return {"us": t * 1e6, "achieved_GBs": wbytes / t / 1e9, "frac": wbytes / t / 1e9 / hbm,
+            "algorithmic_bytes": wbytes, "weights": N * K, "input": "fp32",
+            "note": f"fp32 weights counted {'twice (larger than L2)' if reads == 2 else 'once (they fit in L2)'}"}
+
+
+# ----------------------------------------------------------------------------
+# our implementation: the stacked chain
+# ----------------------------------------------------------------------------
+
+def run_chain(name, args, ctx):
+    import torch
+
+    from bitlinear_bitnet_quant_b200 import chain
+
+    api, rank, world, dev, stream, timer = ctx["api"], ctx["rank"], ctx["world"], ctx["dev"], ctx["stream"], \
+        ctx["timer"]
+    M = CHAIN_WORKLOADS[name]
+    H, F = wl.CHAIN_HIDDEN, wl.CHAIN_FFN
+    layers = ctx.get("chain_layers")
+    if layers is None:
+        g = torch.Generator(device=dev)
+        g.manual_seed(1000 + rank)
+        layers = []
+        for _ in range(CHAIN_LAYERS):      # N(0, 0.02) weights drawn on the device, quantised offline
+            w = {pn: torch.randn((n, k), generator=g, device=dev) * 0.02 for pn, n, k, _ in wl.CHAIN_PROJ}
+            layers.append(chain.quantize_layer(w, stream=stream))
+            del w
+        torch.cuda.synchronize()
+        ctx["chain_layers"] = layers
     ch = chain.BitLinearChain(layers, M, H, F, dev)
     x = torch.from_numpy(wl.chain_input(M)).to(dev)
 
@@ -462,128 +503,100 @@ def run_chain(args, rank, world, local_rank):
         ch.forward(x, stream)
     torch.cuda.synchronize()
 
-    def graph_of(fn):
-        gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr, stream=stream):
-            for _ in range(args.steps):
-                fn()
-        return gr
-
-    def lin_only():                          # the chain's linear layers alone, same operands
+    def lin_only(i):                       # the chain's linear layers alone, same operands
         for w in layers:
-            for name, Xq, sx, Y, bits in (("q", ch.xq, ch.sx, ch.q, 8), ("k", ch.xq, ch.sx, ch.k, 8),
-                                          ("v", ch.xq, ch.sx, ch.v, 8), ("o", ch.v4, ch.sv, ch.o, 4),
-                                          ("up", ch.hq, ch.sh, ch.up, 8), ("gate", ch.hq, ch.sh, ch.gate, 8),
-                                          ("down", ch.a4, ch.sa, ch.d, 4)):
-                api.bitnet_linear(Xq, bits, sx, *w[name], Y=Y, stream=stream)
+            for pn, Xq, sx, Y, bits in (("q", ch.xq, ch.sx, ch.q, 8), ("k", ch.xq, ch.sx, ch.k, 8),
+                                        ("v", ch.xq, ch.sx, ch.v, 8), ("o", ch.v4, ch.sv, ch.o, 4),
+                                        ("up", ch.hq, ch.sh, ch.up, 8), ("gate", ch.hq, ch.sh, ch.gate, 8),
+                                        ("down", ch.a4, ch.sa, ch.d, 4)):
+                api.bitnet_linear(Xq, bits, sx, *w[pn], Y=Y, stream=stream)
 
-    g_step = graph_of(lambda: ch.forward(x, stream))
-    g_lin = graph_of(lin_only)
-    visible = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
-    clocks = ClockSampler(visible[local_rank] if local_rank < len(visible) else str(local_rank))
-    clocks.start()
-    t_step = timed_replay(g_step, stream, world, dev)
-    t_lin = timed_replay(g_lin, stream, world, dev)
-    clk = clocks.stop()
+    t_step = timer.time(timer.graph(lambda i: ch.forward(x, stream)))
+    t_lin = timer.time(timer.graph(lin_only))
 
     # e2e: host input in, host output back, through the Python API
     x_pin = torch.empty((M, H), dtype=torch.float32).pin_memory()
     x_pin.copy_(x.cpu())
     y_pin = torch.empty((M, H), dtype=torch.float32).pin_memory()
-    for _ in range(warmup):
+
+    def e2e_step(i):
         x.copy_(x_pin, non_blocking=True)
         y_pin.copy_(ch.forward(x, stream), non_blocking=True)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        x.copy_(x_pin, non_blocking=True)
-        y_pin.copy_(ch.forward(x, stream), non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    t_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    if rank != 0:
-        return None
-    peaks, peak_src = load_peaks()
-    steps = args.steps
-    step_s = t_step / steps / 1e3
-    lin_s = t_lin / steps / 1e3                       # all 7 x 24 linear launches of one step
+
+    for i in range(warmup):
+        e2e_step(i)
+    t_e2e = e2e_time(e2e_step, stream, world, dev, args.steps, args.min_time / 2)
+
+    peaks, peak_src = ctx["peaks"]
+    step_s = t_step["ms"] / 1e3
+    lin_s = t_lin["ms"] / 1e3                       # all 7 x 24 linear launches of one step
     packed = ch.packed_bytes()
     ops = 2.0 * M * sum(n * k for _, n, k, _ in wl.CHAIN_PROJ) * CHAIN_LAYERS
     act_bytes = CHAIN_LAYERS * M * (4 * (5 * H + 3 * F) + 2 * H + H // 2 + F // 2 + 7 * 4)
     if M <= 64:
         roof = {"bound": "hbm", "achieved": (packed + act_bytes) / lin_s / 1e9, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "kernel": "bitnet_linear, all 168 launches of a step",
+                "unit": "GB/s", "kernel": f"bitnet_linear, all {7 * CHAIN_LAYERS} launches of a step",
                 "algorithmic_bytes_per_step": packed + act_bytes}
     else:
-        roof = {"bound": "tensor", "achieved": ops / lin_s / 1e12, "peak": 2.0 * peaks["bf16_tflops"],
-                "unit": "TOPS", "kernel": "bitnet_linear, all 168 launches of a step",
-                "algorithmic_ops_per_step": ops, "peak_note": "2 x measured bf16 burst (nominal int8/bf16 ratio)"}
+        roof = {"bound": "tensor", "achieved": ops / lin_s / 1e12, "peak": int8_peak(peaks),
+                "unit": "TOPS", "kernel": f"bitnet_linear, all {7 * CHAIN_LAYERS} launches of a step",
+                "algorithmic_ops_per_step": ops, "peak_note": "2 x measured bf16 burst (nominal int8 : bf16 ratio)",
+                "frac_of_nominal_4500_tops": ops / lin_s / 1e12 / NOMINAL_INT8_TOPS}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = profiled_traffic(f"linear_{args.workload}")
+    roof["traffic"] = profiled_traffic(f"linear_{name}")
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    tokens = M * world
+    # whole-step view: the slower of the weight stream and the integer work, against the step time
+    ideal = max((packed + act_bytes) / (peaks["hbm_gbs"] * 1e9), ops / (int8_peak(peaks) * 1e12))
     return {
-        "metric": METRIC, "value": tokens * steps / (t_step / 1e3), "unit": "tokens/s", "n_gpus": world,
-        "steps": steps, "warmup": warmup, "ms_per_step": t_step / steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8/int4 x ternary -> int32, fp32 glue",
-        "data": "synthetic",
-        "config": {"workload": f"bitlinear_chain_{CHAIN_LAYERS}layers_m{M}_hidden{H}_ffn{F}", "M_tokens": M,
-                   "layers": CHAIN_LAYERS, "l2": f"{packed / 1e6:.0f} MB of packed weights per step (> 2x L2)",
-                   "timing": "CUDA graph of the K steps, CUDA events on the launching stream",
-                   "parallelism": f"dp{world} (independent batches per rank)"},
+        "workload": f"bitlinear_chain_{CHAIN_LAYERS}layers_m{M}_hidden{H}_ffn{F}", "M_tokens": M,
+        "layers": CHAIN_LAYERS, "hidden": H, "ffn": F,
+        "l2": f"{packed / 1e6:.0f} MB of packed weights per step (> 2x L2)",
+        "value": M * world / step_s, "unit": "tokens/s", "ms_per_step": t_step["ms"],
+        "timing": spread(t_step),
         "roofline": roof,
+        "step_roofline": {"ideal_us": ideal * 1e6, "achieved_us": step_s * 1e6, "frac": ideal / step_s,
+                          "note": "max(bytes / HBM peak, int ops / int8 peak) over the step time"},
         "kernels_us": {"linear_all_per_step": lin_s * 1e6, "step": step_s * 1e6},
-        "e2e": {"value": tokens * steps / (t_e2e / 1e3), "unit": "tokens/s",
+        "e2e": {"value": M * world / t_e2e, "unit": "tokens/s",
                 "h2d_bytes_per_step": M * H * 4, "d2h_bytes_per_step": M * H * 4},
-        "gpu_launches": ch.launches * steps,
-        "clocks": clk,
+        "gpu_launches_per_step": ch.launches,
+        "clocks": ctx["clocks"].summary(t_step["window"][0], t_lin["window"][1]),
     }
 
 
-def chain_cpu_baseline(M, budget_s=10.0):
-    """Oracle tokens/s through the chain: two layers, scaled to 24."""
-    from oracle import bitnet_oracle as O
-    layers = []
-    for l in range(2):
-        lw = {}
-        for name, w in wl.chain_weights(l).items():
-            _, s_w, q = O.quantize_weights(w)
-            lw[name] = (q, s_w)
-        layers.append(lw)
-    x = wl.chain_input(min(M, 4))
-    t0 = time.perf_counter()
-    n = 0
-    while True:
-        y = x
-        for lw in layers:
-            y = O.chain_layer(y, lw)
-        n += 1
-        if time.perf_counter() - t0 >= budget_s:
-            break
-    dt = (time.perf_counter() - t0) * CHAIN_LAYERS / 2
-    return {"value": n * len(x) / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} passes of {len(x)} tokens through 2 oracle layers, time scaled to {CHAIN_LAYERS} layers"}
+# ----------------------------------------------------------------------------
+# CPU oracle (the cpu_baseline legs and the reference arm)
+# ----------------------------------------------------------------------------
+
+_ORACLE_WEIGHTS = {}
 
 
-# ----------------------------------------------------------------------------
-# CPU oracle (the reference arm and the cpu_baseline leg)
-# ----------------------------------------------------------------------------
+def _oracle_weights(N, K, which):
+    """Quantised weights of the (N, K) workload layer by one of the two oracles,
+    computed once per process (the decode batch sizes share their layer)."""
+    key = (N, K, which)
+    if key not in _ORACLE_WEIGHTS:
+        if which == "numpy":
+            from oracle import bitnet_oracle as O
+            _, s_w, qw = O.quantize_weights(wl.weights(N, K, seed=0))
+        else:
+            from oracle import c_oracle as C
+            _, s_w, qw = C.quantize_weights(wl.weights(N, K, seed=0))
+        _ORACLE_WEIGHTS[key] = (s_w, qw)
+    return _ORACLE_WEIGHTS[key]
+
 
 def oracle_step_fn(c):
     from oracle import bitnet_oracle as O
-    w = wl.weights(c["N"], c["K"], seed=0)
-    _, s_w, qw = O.quantize_weights(w)
+    s_w, qw = _oracle_weights(c["N"], c["K"], "numpy")
     x = O.bf16_bits_to_f32(c["x"]) if c["x_dtype"] == "bf16" else c["x"]
 
     def step(rows):
         xs = x[rows]
         if c["act_bits"] == 8:
-            q, s = O.quant_act(xs, None, 1e-6)
+            q, s = O.quant_act(xs, None, EPS)
         else:
-            _, s, q, _ = O.hadamard_quant_act(xs, None, 1e-6, c.get("had_block", 0))
+            _, s, q, _ = O.hadamard_quant_act(xs, None, EPS, c.get("had_block", 0))
         O.linear(q, s, qw, s_w)
         return len(xs)
     return step
@@ -594,41 +607,7 @@ def sample_rows(c):
     return np.arange(c["M"]) if c["M"] <= 16 else np.arange(8)
 
 
-def cpu_baseline(c, budget_s=10.0):
-    step = oracle_step_fn(c)
-    rows = sample_rows(c)
-    step(rows[:1])                                   # warm-up (allocations)
-    t0 = time.perf_counter()
-    tokens, n = 0, 0
-    while True:
-        tokens += step(rows)
-        n += 1
-        if time.perf_counter() - t0 >= budget_s:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} oracle steps of {len(rows)} tokens of {c['name']} (numpy, single thread)"}
-
-
-def cpu_baseline_omp(c, budget_s=5.0):
-    """The same oracle step through the plain C++ oracle, its loops over tokens and
-    output rows on all host cores (bit-identical results to the numpy oracle)."""
-    from oracle import c_oracle as C
-    w = wl.weights(c["N"], c["K"], seed=0)
-    _, s_w, qw = C.quantize_weights(w)
-    x = (c["x"].astype(np.uint32) << 16).view(np.float32) if c["x_dtype"] == "bf16" else c["x"]
-    rows = np.arange(c["M"]) if c["M"] <= 16 else np.arange(128)
-
-    def step():
-        xs = x[rows]
-        if c["act_bits"] == 8:
-            q, s = C.quant_act(xs, None, 1e-6)
-        else:
-            _, s, q, _ = C.hadamard_quant_act(xs, None, 1e-6, c.get("had_block", 0))
-        C.linear(q, s, qw, s_w)
-        return len(rows)
-
-    step()                                           # warm-up
+def _timed_loop(step, budget_s):
     t0 = time.perf_counter()
     tokens, n = 0, 0
     while True:
@@ -636,64 +615,217 @@ def cpu_baseline_omp(c, budget_s=5.0):
         n += 1
         if time.perf_counter() - t0 >= budget_s:
             break
-    dt = time.perf_counter() - t0
+    return tokens, n, time.perf_counter() - t0
+
+
+def cpu_baseline(c, budget_s=2.0):
+    step = oracle_step_fn(c)
+    rows = sample_rows(c)
+    step(rows[:1])                                   # warm-up (allocations)
+    tokens, n, dt = _timed_loop(lambda: step(rows), budget_s)
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} oracle steps of {len(rows)} tokens of {c['name']} (numpy, single thread)"}
+
+
+def cpu_baseline_omp(c, budget_s=1.5):
+    """The same oracle step through the plain C++ oracle, its loops over tokens and
+    output rows on all host cores (bit-identical results to the numpy oracle)."""
+    from oracle import c_oracle as C
+    s_w, qw = _oracle_weights(c["N"], c["K"], "c")
+    x = (c["x"].astype(np.uint32) << 16).view(np.float32) if c["x_dtype"] == "bf16" else c["x"]
+    rows = np.arange(c["M"]) if c["M"] <= 16 else np.arange(128)
+
+    def step():
+        xs = x[rows]
+        if c["act_bits"] == 8:
+            q, s = C.quant_act(xs, None, EPS)
+        else:
+            _, s, q, _ = C.hadamard_quant_act(xs, None, EPS, c.get("had_block", 0))
+        C.linear(q, s, qw, s_w)
+        return len(rows)
+
+    step()                                           # warm-up
+    tokens, n, dt = _timed_loop(step, budget_s)
     return {"value": tokens / dt, "unit": "tokens/s", "cores": C.threads(), "kind": "oracle (C++, OpenMP)",
             "sample": f"{n} oracle steps of {len(rows)} tokens of {c['name']} (C++ oracle, OpenMP over tokens "
                       f"and output rows)"}
 
 
+class ChainOracle:
+    """The numpy oracle's stacked layer over all 24 layers.  Two layers' weights
+    are quantised and alternated (a token's work does not depend on the weight
+    values), which keeps the set-up to seconds."""
+
+    def __init__(self):
+        from oracle import bitnet_oracle as O
+        self.O = O
+        self.layers = []
+        for l in range(2):
+            lw = {}
+            for pn, w in wl.chain_weights(l).items():
+                _, s_w, q = O.quantize_weights(w)
+                lw[pn] = (q, s_w)
+            self.layers.append(lw)
+
+    def step(self, x):
+        y = x
+        for l in range(CHAIN_LAYERS):
+            y = self.O.chain_layer(y, self.layers[l % 2])
+        return len(x)
+
+
+def chain_cpu_baseline(budget_s=4.0, oracle=None):
+    o = oracle or ChainOracle()
+    x = wl.chain_input(1)
+    tokens, n, dt = _timed_loop(lambda: o.step(x), budget_s)
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} passes of 1 token through all {CHAIN_LAYERS} layers of the numpy oracle "
+                      f"(numpy, single thread)"}
+
+
 def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle as it stands, on the headline workload
+    (or --workload), rank 0 only; each step is a bounded sample of it."""
     if rank != 0:
         return None
-    c = WORKLOADS[args.workload]()
-    step = oracle_step_fn(c)
-    rows = sample_rows(c)
-    for _ in range(max(3, args.warmup)):
-        step(rows)
-    t0 = time.perf_counter()
-    tokens = 0
-    for _ in range(args.steps):
-        tokens += step(rows)
-    dt = time.perf_counter() - t0
+    name = HEADLINE if args.workload == "all" else args.workload
+    warmup = max(3, args.warmup)
+    if name in CHAIN_WORKLOADS:
+        o = ChainOracle()
+        x = wl.chain_input(1)
+        for _ in range(warmup):
+            o.step(x)
+        t0 = time.perf_counter()
+        tokens = sum(o.step(x) for _ in range(args.steps))
+        dt = time.perf_counter() - t0
+        sample = f"each step: 1 token through all {CHAIN_LAYERS} layers of the numpy oracle"
+        config = {"workload": f"bitlinear_chain_{CHAIN_LAYERS}layers_m{CHAIN_WORKLOADS[name]}_hidden"
+                              f"{wl.CHAIN_HIDDEN}_ffn{wl.CHAIN_FFN}", "M_tokens": CHAIN_WORKLOADS[name],
+                  "layers": CHAIN_LAYERS}
+        dtype = "int8/int4 x ternary -> int64, fp32 glue"
+    else:
+        c = WORKLOADS[name]()
+        step = oracle_step_fn(c)
+        rows = sample_rows(c)
+        for _ in range(warmup):
+            step(rows)
+        t0 = time.perf_counter()
+        tokens = sum(step(rows) for _ in range(args.steps))
+        dt = time.perf_counter() - t0
+        sample = f"each step: {len(rows)} tokens of {c['name']} through the numpy oracle"
+        config = {"workload": c["name"], "M_tokens": c["M"], "K": c["K"], "N": c["N"], "act_bits": c["act_bits"]}
+        dtype = "int8xternary->int64" if c["act_bits"] == 8 else "int4xternary->int64"
     value = tokens / dt
+    config["parallelism"] = "rank 0 only (CPU oracle)"
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": dt / args.steps * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int8xternary->int64" if c["act_bits"] == 8 else "int4xternary->int64",
-            "data": "synthetic",
-            "config": {"workload": c["name"], "M_tokens": c["M"], "K": c["K"], "N": c["N"],
-                       "act_bits": c["act_bits"], "parallelism": "rank 0 only (CPU oracle)"},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": f"each step: {len(rows)} tokens of {c['name']} through the numpy oracle"},
+            "steps": args.steps, "warmup": warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
+            "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def add_cpu_baselines(subs):
+    """cpu_baseline (numpy oracle, one core) and cpu_baseline_all_cores (C++
+    oracle, OpenMP) for every configuration that ran."""
+    chain_oracle = None
+    for name, sub in subs.items():
+        if name in CHAIN_WORKLOADS:
+            chain_oracle = chain_oracle or ChainOracle()
+            sub["cpu_baseline"] = chain_cpu_baseline(oracle=chain_oracle)
+            continue
+        c = WORKLOADS[name]()
+        sub["cpu_baseline"] = cpu_baseline(c)
+        try:
+            sub["cpu_baseline_all_cores"] = cpu_baseline_omp(c)
+        except Exception as e:                       # e.g. no C++ compiler on the host
+            sub["cpu_baseline_all_cores"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+
+
+# ----------------------------------------------------------------------------
+# driver
+# ----------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    from bitlinear_bitnet_quant_b200 import api, build_lib
+
+    build_lib.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    visible = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    clocks = ClockSampler(visible[local_rank] if local_rank < len(visible) else str(local_rank)).start()
+    timer = Timer(stream, world, dev, args.steps, args.min_time, clocks)
+    ctx = {"api": api, "rank": rank, "world": world, "dev": dev, "stream": stream, "timer": timer,
+           "clocks": clocks, "peaks": load_peaks()}
+    names = ORDER if args.workload == "all" else [args.workload]
+    subs = {}
+    try:
+        for name in names:
+            subs[name] = (run_chain if name in CHAIN_WORKLOADS else run_layer)(name, args, ctx)
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+        if api.bitnet_device_error() != 0:
+            raise RuntimeError("a kernel reported a device-side wait timeout")
+    finally:
+        overall = clocks.stop()
+    if rank != 0:
+        return None
+    if world == 1 and not args.no_cpu_baseline:
+        add_cpu_baselines(subs)
+
+    head_name = HEADLINE if HEADLINE in subs else names[-1]
+    head = subs[head_name]
+    steps = args.steps
+    launches = head["gpu_launches_per_step"] * head["timing"]["steps_per_replay"] * head["timing"]["replays"]
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": max(3, args.warmup), "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": ("int8/int4 x ternary -> int32, fp32 glue" if head_name in CHAIN_WORKLOADS else
+                  "int8xternary->int32" if head["act_bits"] == 8 else "int4xternary->int32"),
+        "data": "synthetic",
+        "config": {k: head[k] for k in ("workload", "M_tokens", "layers", "hidden", "ffn", "K", "N", "act_bits",
+                                        "l2") if k in head},
+        "roofline": head["roofline"],
+        "timing": head["timing"],
+        "e2e": head["e2e"],
+        "gpu_launches": launches,
+        "clocks": head["clocks"] or overall,
+        "kernels_us": head["kernels_us"],
+    }
+    line["config"]["timing"] = ("R replays of a CUDA graph of K steps between a barrier and a device synchronise "
+                                "on both sides; CUDA events around each replay on the launching stream; median")
+    line["config"]["parallelism"] = f"dp{world} (independent batches per rank)"
+    for k in ("step_roofline", "cpu_baseline", "cpu_baseline_all_cores"):
+        if k in head:
+            line[k] = head[k]
+    line["configs"] = {n: s for n, s in subs.items() if n != head_name}
+    line["clocks_whole_run"] = overall
+    return line
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(CHAIN_WORKLOADS), default="decode")
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", choices=["all"] + ORDER, default="all")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--min-time", type=float, default=0.5, help="seconds of graph replays per timed region")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        world = max(world, 1)
+    world = max(world, 1)
 
     if args.impl == "reference":
-        line = run_reference(args, rank, world) if args.workload in WORKLOADS else None
-        if args.workload in CHAIN_WORKLOADS and rank == 0:
-            cb = chain_cpu_baseline(CHAIN_WORKLOADS[args.workload], budget_s=2.0 * max(1, args.steps))
-            line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
-                    "n_gpus": world, "steps": args.steps, "warmup": 0, "higher_is_better": True,
-                    "scaling": "weak", "vs_baseline": None, "data": "synthetic",
-                    "config": {"workload": args.workload, "parallelism": "rank 0 only (CPU oracle)"},
-                    "cpu_baseline": cb, "e2e": {"value": cb["value"], "unit": "tokens/s",
-                                                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        line = run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
         return
@@ -709,18 +841,7 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
         pg = True
     try:
-        if args.workload in CHAIN_WORKLOADS:
-            line = run_chain(args, rank, world, local_rank)
-            if line is not None and world == 1 and not args.no_cpu_baseline:
-                line["cpu_baseline"] = chain_cpu_baseline(CHAIN_WORKLOADS[args.workload])
-        else:
-            line = run_ours(args, rank, world, local_rank)
-            if line is not None and world == 1 and not args.no_cpu_baseline:
-                line["cpu_baseline"] = cpu_baseline(WORKLOADS[args.workload]())
-                try:
-                    line["cpu_baseline_all_cores"] = cpu_baseline_omp(WORKLOADS[args.workload]())
-                except Exception as e:                   # e.g. no C++ compiler on the host
-                    line["cpu_baseline_all_cores"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+        line = run_ours(args, rank, world, local_rank)
         if line is not None:
             print(json.dumps(line), flush=True)
     finally:

@@ -52,7 +52,11 @@ _SIGNATURES = {
     "bitnet_repack_trit5": (ctypes.c_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
     "bitnet_linear_trit5": (ctypes.c_int, [_c_void_p, ctypes.c_int, _c_void_p, _c_void_p, _c_void_p, _i64, _i64,
                                            _i64, _c_void_p, ctypes.c_int, _c_void_p, _c_void_p]),
-    "bitnet_set_linear_path": (ctypes.c_int, [ctypes.c_int]),
+    "bitnet_linear_kernel": (ctypes.c_int, [_c_void_p, ctypes.c_int, _c_void_p, _c_void_p, _c_void_p, _i64, _i64,
+                                            _i64, _c_void_p, ctypes.c_int, _c_void_p, ctypes.c_int, _c_void_p]),
+    "bitnet_bitlinear_kernel": (ctypes.c_int, [_c_void_p, ctypes.c_int, _i64, _i64, _c_void_p, ctypes.c_float,
+                                               _c_void_p, _c_void_p, _i64, _c_void_p, ctypes.c_int, _c_void_p,
+                                               _c_void_p, ctypes.c_int, _c_void_p]),
     "bitnet_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
 }
 
@@ -206,8 +210,9 @@ def bitnet_glu_hadamard_quant_act(gate: torch.Tensor, up: torch.Tensor, gamma=No
 
 
 def bitnet_linear(Xq: torch.Tensor, act_bits: int, s_x: torch.Tensor, pkW: torch.Tensor, s_w: torch.Tensor,
-                  out_dtype=torch.float32, Y=None, want_acc: bool = False, stream=None):
-    """Ternary x int8/int4 product + dequantisation.  Returns (Y [M, N], acc int32 or None)."""
+                  out_dtype=torch.float32, Y=None, want_acc: bool = False, stream=None, kernel: int = 0):
+    """Ternary x int8/int4 product + dequantisation.  Returns (Y [M, N], acc int32 or None).
+    kernel != 0 picks the kernel family for this call (bitnet_linear_kernel)."""
     _require(Xq, "Xq")
     _require(pkW, "pkW")
     M = Xq.shape[0]
@@ -215,9 +220,11 @@ def bitnet_linear(Xq: torch.Tensor, act_bits: int, s_x: torch.Tensor, pkW: torch
     K = KB * 4
     Y = torch.empty((M, N), dtype=out_dtype, device=Xq.device) if Y is None else Y
     acc = torch.empty((M, N), dtype=torch.int32, device=Xq.device) if want_acc else None
-    _check("bitnet_linear", lib().bitnet_linear(
-        _ptr(Xq), int(act_bits), _ptr(s_x), _ptr(pkW), _ptr(s_w), M, N, K, _ptr(Y), _dtype_code(Y),
-        _ptr(acc), _stream(stream)))
+    args = (_ptr(Xq), int(act_bits), _ptr(s_x), _ptr(pkW), _ptr(s_w), M, N, K, _ptr(Y), _dtype_code(Y), _ptr(acc))
+    if kernel:
+        _check("bitnet_linear_kernel", lib().bitnet_linear_kernel(*args, int(kernel), _stream(stream)))
+    else:
+        _check("bitnet_linear", lib().bitnet_linear(*args, _stream(stream)))
     return Y, acc
 
 
@@ -252,9 +259,10 @@ def bitnet_linear_trit5(Xq: torch.Tensor, act_bits: int, s_x: torch.Tensor, pk5:
 
 
 def bitnet_bitlinear(X: torch.Tensor, pkW: torch.Tensor, s_w: torch.Tensor, gamma=None, eps: float = 1e-6,
-                     out_dtype=torch.float32, Y=None, Xq=None, s_x=None, stream=None):
+                     out_dtype=torch.float32, Y=None, Xq=None, s_x=None, stream=None, kernel: int = 0):
     """Fused BitLinear forward with int8 activations (RMSNorm + absmax int8 +
-    ternary product + dequantisation).  Returns (Y [M, N], Xq [M, K], s_x [M])."""
+    ternary product + dequantisation).  Returns (Y [M, N], Xq [M, K], s_x [M]).
+    kernel != 0 picks the kernels for this call (bitnet_bitlinear_kernel; 4 = one fused kernel)."""
     _require(X, "X")
     _require(pkW, "pkW")
     M, K = X.shape
@@ -263,9 +271,12 @@ def bitnet_bitlinear(X: torch.Tensor, pkW: torch.Tensor, s_w: torch.Tensor, gamm
     Y = torch.empty((M, N), dtype=out_dtype, device=dev) if Y is None else Y
     Xq = torch.empty((M, K), dtype=torch.int8, device=dev) if Xq is None else Xq
     s_x = torch.empty((M,), dtype=torch.float32, device=dev) if s_x is None else s_x
-    _check("bitnet_bitlinear", lib().bitnet_bitlinear(
-        _ptr(X), _dtype_code(X), M, K, _ptr(gamma), float(eps), _ptr(pkW), _ptr(s_w), N, _ptr(Y), _dtype_code(Y),
-        _ptr(Xq), _ptr(s_x), _stream(stream)))
+    args = (_ptr(X), _dtype_code(X), M, K, _ptr(gamma), float(eps), _ptr(pkW), _ptr(s_w), N, _ptr(Y), _dtype_code(Y),
+            _ptr(Xq), _ptr(s_x))
+    if kernel:
+        _check("bitnet_bitlinear_kernel", lib().bitnet_bitlinear_kernel(*args, int(kernel), _stream(stream)))
+    else:
+        _check("bitnet_bitlinear", lib().bitnet_bitlinear(*args, _stream(stream)))
     return Y, Xq, s_x
 
 
@@ -282,10 +293,6 @@ def bitnet_relu2_glu(gate: torch.Tensor, up: torch.Tensor, out=None, stream=None
     _check("bitnet_relu2_glu", lib().bitnet_relu2_glu(_ptr(gate), _ptr(up), _ptr(out), gate.numel(),
                                                       _stream(stream)))
     return out
-
-
-def bitnet_set_linear_path(path: int) -> None:
-    _check("bitnet_set_linear_path", lib().bitnet_set_linear_path(int(path)))
 
 
 def bitnet_device_error() -> int:

@@ -68,11 +68,6 @@ int cuda_status(cudaError_t e) {
   return BITNET_ERR_CUDA;
 }
 
-// 0 = automatic, 1 = SIMT, 2 = tcgen05, 3 = warp-MMA decode, 4 = fused BitLinear kernel
-// (set by bitnet_set_linear_path).
-std::atomic<int> g_linear_path{0};
-int linear_path() { return g_linear_path.load(std::memory_order_relaxed); }
-
 }  // namespace
 
 extern "C" {
@@ -91,7 +86,7 @@ const char* bitnet_status_string(int status) {
   return "unknown status";
 }
 
-int bitnet_abi_version(void) { return 1; }
+int bitnet_abi_version(void) { return 2; }
 
 size_t bitnet_quantize_weights_workspace_size(int64_t N, int64_t K) {
   (void)N; (void)K;
@@ -102,7 +97,9 @@ int bitnet_quantize_weights(const void* W, int w_dtype, int64_t N, int64_t K, ui
                             void* workspace, size_t workspace_bytes, void* stream) {
   if (!W || !pkW || !s_w) return BITNET_ERR_NULL;
   if (w_dtype != BITNET_F32 && w_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
-  if (N < 1 || K < 16 || K % 16 != 0 || N * K >= (int64_t(1) << 31)) return BITNET_ERR_SHAPE;
+  if (N < 1 || K < 16 || K % 16 != 0 || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) ||
+      N * K >= (int64_t(1) << 31))                       // each factor < 2^31: the product cannot overflow
+    return BITNET_ERR_SHAPE;
   if (!workspace || workspace_bytes < bitnet::weights_workspace_bytes()) return BITNET_ERR_WORKSPACE;
   if (!aligned16(W) || !aligned16(pkW) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(s_w) & 3u))
     return BITNET_ERR_ALIGN;
@@ -179,8 +176,11 @@ int bitnet_hadamard_quant_act(const void* X, int x_dtype, int64_t M, int64_t K, 
                                                    Xq4, s_x, T_dbg, static_cast<cudaStream_t>(stream)));
 }
 
-int bitnet_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
-                  int64_t M, int64_t N, int64_t K, void* Y, int y_dtype, int32_t* acc_dbg, void* stream) {
+// kernel: 0 = automatic, 1 = CUDA-core dp4a, 2 = tcgen05, 3 = warp-MMA decode
+static int linear_impl(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
+                       int64_t M, int64_t N, int64_t K, void* Y, int y_dtype, int32_t* acc_dbg, int kernel,
+                       void* stream) {
+  if (kernel < 0 || kernel > 3) return BITNET_ERR_SHAPE;
   if (act_bits != 8 && act_bits != 4) return BITNET_ERR_DTYPE;
   if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
   if (M < 0 || M > (int64_t(1) << 30) || N < 1 || N > (int64_t(1) << 30) || K < 128 || K > 65536 ||
@@ -191,13 +191,24 @@ int bitnet_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t*
   if (!aligned16(Xq) || !aligned16(pkW) || !aligned16(Y) || (acc_dbg && !aligned16(acc_dbg)) ||
       (reinterpret_cast<uintptr_t>(s_x) & 3u) || (reinterpret_cast<uintptr_t>(s_w) & 3u))
     return BITNET_ERR_ALIGN;
+  if (kernel == 3 && !bitnet::decode_path_applies((int)M, (int)K)) return BITNET_ERR_SHAPE;
   int d = check_device();
   if (d != BITNET_OK) return d;
   if (!bitnet::tensor_map_encoder_available()) return BITNET_ERR_UNSUPPORTED;
-  if (linear_path() == 3 && !bitnet::decode_path_applies((int)M, (int)K)) return BITNET_ERR_SHAPE;
   return cuda_status(bitnet::run_linear(Xq, act_bits, s_x, pkW, s_w, (int)M, (int)N, (int)K, Y,
-                                        y_dtype == BITNET_BF16, acc_dbg, linear_path(),
+                                        y_dtype == BITNET_BF16, acc_dbg, kernel,
                                         static_cast<cudaStream_t>(stream)));
+}
+
+int bitnet_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
+                  int64_t M, int64_t N, int64_t K, void* Y, int y_dtype, int32_t* acc_dbg, void* stream) {
+  return linear_impl(Xq, act_bits, s_x, pkW, s_w, M, N, K, Y, y_dtype, acc_dbg, 0, stream);
+}
+
+int bitnet_linear_kernel(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
+                         int64_t M, int64_t N, int64_t K, void* Y, int y_dtype, int32_t* acc_dbg, int kernel,
+                         void* stream) {
+  return linear_impl(Xq, act_bits, s_x, pkW, s_w, M, N, K, Y, y_dtype, acc_dbg, kernel, stream);
 }
 
 size_t bitnet_trit5_row_bytes(int64_t K) {
@@ -206,7 +217,7 @@ size_t bitnet_trit5_row_bytes(int64_t K) {
 }
 
 int bitnet_repack_trit5(const uint8_t* pkW, int64_t N, int64_t K, uint8_t* pk5, void* stream) {
-  if (N < 1 || K < 16 || K % 16 != 0 || K > (int64_t(1) << 30)) return BITNET_ERR_SHAPE;
+  if (N < 1 || N >= (int64_t(1) << 31) || K < 16 || K % 16 != 0 || K > (int64_t(1) << 30)) return BITNET_ERR_SHAPE;
   if (N * (int64_t)bitnet::trit5_row_bytes_host((int)K) >= (int64_t(1) << 31) || N * K / 4 >= (int64_t(1) << 31))
     return BITNET_ERR_SHAPE;
   if (!pkW || !pk5) return BITNET_ERR_NULL;
@@ -242,9 +253,12 @@ static int elementwise_check(const float* a, const float* b, const float* out, i
   return check_device();
 }
 
-int bitnet_bitlinear(const void* X, int x_dtype, int64_t M, int64_t K, const float* gamma, float eps,
-                     const uint8_t* pkW, const float* s_w, int64_t N, void* Y, int y_dtype, int8_t* Xq, float* s_x,
-                     void* stream) {
+// kernel: 0 = automatic (the quantiser, then bitnet_linear's choice), 1-3 = the
+// quantiser, then that linear kernel family, 4 = the fused single kernel
+static int bitlinear_impl(const void* X, int x_dtype, int64_t M, int64_t K, const float* gamma, float eps,
+                          const uint8_t* pkW, const float* s_w, int64_t N, void* Y, int y_dtype, int8_t* Xq,
+                          float* s_x, int kernel, void* stream) {
+  if (kernel < 0 || kernel > 4) return BITNET_ERR_SHAPE;
   if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
   if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
   if (M < 0 || M > (int64_t(1) << 30) || N < 1 || N > (int64_t(1) << 30) || K < 128 || K > 16384 ||
@@ -255,15 +269,27 @@ int bitnet_bitlinear(const void* X, int x_dtype, int64_t M, int64_t K, const flo
   if (!aligned16(X) || !aligned16(pkW) || !aligned16(Y) || !aligned16(Xq) || (gamma && !aligned16(gamma)) ||
       (reinterpret_cast<uintptr_t>(s_x) & 3u) || (reinterpret_cast<uintptr_t>(s_w) & 3u))
     return BITNET_ERR_ALIGN;
+  if (kernel == 3 && !bitnet::decode_path_applies((int)M, (int)K)) return BITNET_ERR_SHAPE;
   int d = check_device();
   if (d != BITNET_OK) return d;
   if (!bitnet::tensor_map_encoder_available()) return BITNET_ERR_UNSUPPORTED;
-  const int path = linear_path();
-  if (path == 3 && !bitnet::decode_path_applies((int)M, (int)K)) return BITNET_ERR_SHAPE;
-  if (path == 4 && !bitnet::fused_path_applies((int)M, (int)N, (int)K, x_dtype == BITNET_BF16)) return BITNET_ERR_SHAPE;
+  if (kernel == 4 && !bitnet::fused_path_applies((int)M, (int)N, (int)K, x_dtype == BITNET_BF16))
+    return BITNET_ERR_SHAPE;
   return cuda_status(bitnet::run_bitlinear(X, x_dtype == BITNET_BF16, (int)M, (int)K, gamma, eps, pkW, s_w, (int)N,
-                                           Y, y_dtype == BITNET_BF16, Xq, s_x, path,
+                                           Y, y_dtype == BITNET_BF16, Xq, s_x, kernel,
                                            static_cast<cudaStream_t>(stream)));
+}
+
+int bitnet_bitlinear(const void* X, int x_dtype, int64_t M, int64_t K, const float* gamma, float eps,
+                     const uint8_t* pkW, const float* s_w, int64_t N, void* Y, int y_dtype, int8_t* Xq, float* s_x,
+                     void* stream) {
+  return bitlinear_impl(X, x_dtype, M, K, gamma, eps, pkW, s_w, N, Y, y_dtype, Xq, s_x, 0, stream);
+}
+
+int bitnet_bitlinear_kernel(const void* X, int x_dtype, int64_t M, int64_t K, const float* gamma, float eps,
+                            const uint8_t* pkW, const float* s_w, int64_t N, void* Y, int y_dtype, int8_t* Xq,
+                            float* s_x, int kernel, void* stream) {
+  return bitlinear_impl(X, x_dtype, M, K, gamma, eps, pkW, s_w, N, Y, y_dtype, Xq, s_x, kernel, stream);
 }
 
 int bitnet_add(const float* a, const float* b, float* out, int64_t n, void* stream) {
@@ -276,12 +302,6 @@ int bitnet_relu2_glu(const float* gate, const float* up, float* out, int64_t n, 
   const int c = elementwise_check(gate, up, out, n);
   if (c != BITNET_OK) return c < 0 ? BITNET_OK : c;
   return cuda_status(bitnet::run_relu2_glu(gate, up, out, (size_t)n, static_cast<cudaStream_t>(stream)));
-}
-
-int bitnet_set_linear_path(int path) {
-  if (path < 0 || path > 4) return BITNET_ERR_SHAPE;
-  g_linear_path.store(path, std::memory_order_relaxed);
-  return BITNET_OK;
 }
 
 int bitnet_device_error(int* code_out) {

@@ -45,7 +45,7 @@ BN_DEV void widen8(uint32_t p, uint32_t& lo4, uint32_t& hi4) {
 // ===========================================================================
 // SIMT kernel: one warp per output row n and block of 16 tokens; lanes split
 // K; dp4a accumulation.  A second, independent GPU implementation, selected
-// only through bitnet_set_linear_path (the tcgen05 kernel is faster at every M).
+// only through bitnet_linear_kernel (the tcgen05 kernel is faster at every M).
 // ===========================================================================
 template <int ACT_BITS, typename TOut>
 __global__ void __launch_bounds__(256)

@@ -12,6 +12,8 @@
 
 namespace bitnet {
 
+cudaError_t enqueue_weights_ready(cudaStream_t st);
+
 // One thread per output byte: five 2-bit codes in, one base-3 byte out.
 __global__ void __launch_bounds__(256)
 trit5_pack_kernel(const uint32_t* __restrict__ pkW, int N, int K, int r5, uint8_t* __restrict__ pk5) {
@@ -41,8 +43,10 @@ cudaError_t run_repack_trit5(const uint8_t* pkW, int N, int K, uint8_t* pk5, cud
   const int r5 = trit5_row_bytes(K);
   const size_t total = (size_t)N * r5;
   const unsigned blocks = (unsigned)((total + 255) / 256);
-  return launch_pdl(trit5_pack_kernel, dim3(blocks), dim3(256), 0, st, 1u, reinterpret_cast<const uint32_t*>(pkW),
-                    N, K, r5, pk5);
+  const cudaError_t e = launch_pdl(trit5_pack_kernel, dim3(blocks), dim3(256), 0, st, 1u,
+                                   reinterpret_cast<const uint32_t*>(pkW), N, K, r5, pk5);
+  if (e != cudaSuccess) return e;
+  return enqueue_weights_ready(st);             // the decode kernel reads pk5 before its dependency wait
 }
 
 size_t trit5_row_bytes_host(int K) { return (size_t)trit5_row_bytes(K); }

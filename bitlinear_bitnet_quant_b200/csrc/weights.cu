@@ -166,6 +166,20 @@ ternary_pack_kernel(const TIn* __restrict__ W, size_t ngroups, const float* __re
 
 size_t weights_workspace_bytes() { return 128; }
 
+// Ends the weight path.  The linear kernels stream their weights before they
+// wait for the kernel ahead of them in the stream (programmatic dependent
+// launch), and that wait alone orders memory.  This empty kernel is launched
+// without the programmatic attribute, so it starts only once the kernel that
+// wrote the weights has completed; and as it never signals its dependents
+// early, the next kernel can start only after it has exited.  A linear kernel
+// enqueued right after a weight call therefore cannot read the weights early.
+__global__ void weights_ready_kernel() {}
+
+cudaError_t enqueue_weights_ready(cudaStream_t st) {
+  weights_ready_kernel<<<1, 32, 0, st>>>();
+  return cudaGetLastError();
+}
+
 cudaError_t run_quantize_weights(const void* W, int bf16, int64_t N, int64_t K, uint8_t* pkW,
                                  float* s_w, void* ws, cudaStream_t st) {
   const size_t n = (size_t)N * (size_t)K;
@@ -191,7 +205,8 @@ cudaError_t run_quantize_weights(const void* W, int bf16, int64_t N, int64_t K, 
     ternary_pack_kernel<uint16_t><<<pb, 256, 0, st>>>(static_cast<const uint16_t*>(W), ng, s_w, reinterpret_cast<uint32_t*>(pkW));
   else
     ternary_pack_kernel<float><<<pb, 256, 0, st>>>(static_cast<const float*>(W), ng, s_w, reinterpret_cast<uint32_t*>(pkW));
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return enqueue_weights_ready(st);
 }
 
 }  // namespace bitnet

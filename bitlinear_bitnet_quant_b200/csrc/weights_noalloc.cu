@@ -13,7 +13,9 @@
 // uses it.  Host code cannot use the array's name as a device address, so the
 // first call on each device looks the address up with cudaGetSymbolAddress
 // (with that device current) and caches it; do that first call before any
-// stream capture.  All calls share the one array: the counters are cleared at
+// stream capture.  The cached address belongs to the device's primary context:
+// after cudaDeviceReset, or under a context the caller created itself, it no
+// longer names the array, and this entry point must not be called.  All calls share the one array: the counters are cleared at
 // the start of each call, and two calls whose kernels overlap on the GPU (for
 // example on two streams) race on it.
 #include <cuda_runtime.h>
@@ -73,7 +75,8 @@ extern "C" int bitnet_quantize_weights_noalloc(const void* W, int w_dtype, int64
   if (w_dtype != BITNET_F32 && w_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
   if (N < 1 || K < 16 || K % 16 != 0) return BITNET_ERR_SHAPE;
   // the fixed 64-bit counters absorb at most 2^31 - 1 weights without overflow
-  if (N * K > BITNET_NOALLOC_MAX_WEIGHTS) return BITNET_ERR_SHAPE;
+  // (compared by division first, so that N * K is never formed when it could overflow)
+  if (K > BITNET_NOALLOC_MAX_WEIGHTS / N || N * K > BITNET_NOALLOC_MAX_WEIGHTS) return BITNET_ERR_SHAPE;
   if (!aligned16(W) || !aligned16(pkW) || (reinterpret_cast<uintptr_t>(s_w) & 3u)) return BITNET_ERR_ALIGN;
   if (bitnet::weights_workspace_bytes() > kNoallocScratchBytes) return BITNET_ERR_WORKSPACE;
   void* scratch = nullptr;

@@ -84,6 +84,14 @@ BITNET_API size_t bitnet_quantize_weights_workspace_size(int64_t N, int64_t K);
  * workspace: device scratch of at least bitnet_quantize_weights_workspace_size
  *            bytes, 16-byte aligned, caller-owned; it is overwritten.
  * Limits   : N >= 1, K >= 16, K % 16 == 0, N*K < 2^31.
+ * Ordering : the linear kernels load pkW and s_w before they wait for the
+ *            kernel ahead of them in the stream (programmatic dependent
+ *            launch).  This call therefore ends with an empty kernel launched
+ *            without that attribute, so a bitnet_linear enqueued right after
+ *            it on the same stream starts only once the weights are complete.
+ *            Weights written by other means (a copy, another library) must be
+ *            complete before the bitnet_linear call is enqueued, or be
+ *            separated from it by a stream synchronisation or an event wait.
  */
 BITNET_API int bitnet_quantize_weights(const void* W, int w_dtype, int64_t N, int64_t K,
                             uint8_t* pkW, float* s_w,
@@ -101,7 +109,9 @@ BITNET_API int bitnet_quantize_weights(const void* W, int w_dtype, int64_t N, in
  * pkW and s_w.  No cudaMalloc, cudaFree or allocating routine is called.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is cached for the device's
+ *     primary context: do not call this entry point after cudaDeviceReset or
+ *     under a context the caller created itself (cuCtxCreate).
  *   - Every call shares the one array and clears it before use; calls whose
  *     kernels overlap on the GPU (e.g. on two streams) race on it.
  *   - Limit: N*K <= BITNET_NOALLOC_MAX_WEIGHTS (what the fixed 64-bit counters
@@ -196,6 +206,9 @@ BITNET_API int bitnet_linear(const void* Xq, int act_bits, const float* s_x, con
  * bitnet_repack_trit5: pkW [N][K/4] (bitnet_quantize_weights' 2-bit format,
  *   read) -> pk5 [N][bitnet_trit5_row_bytes(K)] (written).  Limits: N >= 1,
  *   16 <= K, K % 16 == 0, N * row bytes < 2^31; pointers 16-byte aligned.
+ *   Like bitnet_quantize_weights it ends with an empty kernel launched without
+ *   the programmatic attribute, so a bitnet_linear_trit5 enqueued right after
+ *   it (which loads pk5 before its dependency wait) sees complete weights.
  * bitnet_linear_trit5: bitnet_linear with the weights in this format, for the
  *   decode shapes only (1 <= M <= 32, K % 512 == 0, K <= 16384; otherwise
  *   BITNET_ERR_SHAPE).  Each CTA stages its rows and rewrites them into the
@@ -216,15 +229,14 @@ BITNET_API int bitnet_linear_trit5(const void* Xq, int act_bits, const float* s_
  * pkW    : [N][K/4] packed ternary weights.  s_w: one fp32 (device).
  * Y      : out, [M][N] fp32 or bf16 (y_dtype).
  * Xq, s_x: out, [M][K] int8 codes and [M] fp32 scales (always written).
- * Kernels: by default the two kernels of bitnet_quant_act and bitnet_linear
- *          (on B200 the faster choice for every decode shape measured: the
- *          quantiser overlaps the linear kernel's weight stream).  After
- *          bitnet_set_linear_path(4), one fused kernel: thread-block clusters
+ * Kernels: the two kernels of bitnet_quant_act and bitnet_linear (on B200
+ *          the faster choice for every decode shape measured: the quantiser
+ *          overlaps the linear kernel's weight stream).  bitnet_bitlinear_kernel
+ *          with kernel 4 runs one fused kernel instead: thread-block clusters
  *          of 8 CTAs share the quantisation (each CTA quantises every eighth
  *          token and copies codes and scale into the shared memory of the
  *          other seven), then the one-pass decode product; it covers up to
  *          32 tokens with K % 512 == 0 and K <= 8192 (else BITNET_ERR_SHAPE).
- *          Paths 1-3 select the linear kernel family as for bitnet_linear.
  * Limits : M >= 0, N >= 1, 128 <= K <= 16384, K % 128 == 0; gamma, X, Xq,
  *          pkW and Y 16-byte aligned.
  */
@@ -244,15 +256,25 @@ BITNET_API int bitnet_add(const float* a, const float* b, float* out, int64_t n,
 BITNET_API int bitnet_relu2_glu(const float* gate, const float* up, float* out, int64_t n, void* stream);
 
 /*
- * Diagnostics: selects the kernel family bitnet_linear uses in this process.
- * 0 = automatic (default: warp-MMA decode kernel where it applies, else the
- * tcgen05 tensor-core kernel), 1 = CUDA-core dp4a kernel, 2 = tcgen05 kernel,
- * 3 = warp-MMA decode kernel (bitnet_linear then returns BITNET_ERR_SHAPE for
- * shapes it does not cover: M > 32, K % 512 != 0 or K > 16384), 4 = the fused
- * kernel of bitnet_bitlinear (bitnet_linear as with 0).  All compute the same
- * bit-exact result.  Returns BITNET_ERR_SHAPE for any other value.
+ * Diagnostics: bitnet_linear and bitnet_bitlinear with the kernel family
+ * chosen per call instead of automatically; every choice computes the same
+ * bit-exact result.  Arguments as for the plain calls, plus `kernel`:
+ *   bitnet_linear_kernel:    0 = automatic (as bitnet_linear), 1 = CUDA-core
+ *                            dp4a kernel, 2 = tcgen05 tensor-core kernel,
+ *                            3 = warp-MMA decode kernel (BITNET_ERR_SHAPE for
+ *                            shapes it does not cover: M > 32, K % 512 != 0 or
+ *                            K > 16384).
+ *   bitnet_bitlinear_kernel: 0-3 = the int8 quantiser, then that linear
+ *                            kernel; 4 = the fused single kernel described at
+ *                            bitnet_bitlinear (BITNET_ERR_SHAPE outside its range).
+ * Any other value returns BITNET_ERR_SHAPE.  No state is kept between calls.
  */
-BITNET_API int bitnet_set_linear_path(int path);
+BITNET_API int bitnet_linear_kernel(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW,
+                                    const float* s_w, int64_t M, int64_t N, int64_t K, void* Y, int y_dtype,
+                                    int32_t* acc_dbg, int kernel, void* stream);
+BITNET_API int bitnet_bitlinear_kernel(const void* X, int x_dtype, int64_t M, int64_t K, const float* gamma,
+                                       float eps, const uint8_t* pkW, const float* s_w, int64_t N, void* Y,
+                                       int y_dtype, int8_t* Xq, float* s_x, int kernel, void* stream);
 
 /*
  * Reads and clears the library's device-side error flag on the current

@@ -29,7 +29,7 @@ def test_status_strings(L):
         assert api.status_string(code)
     assert api.status_string(0) == "ok"
     assert api.status_string(99) == "unknown status"
-    assert L.bitnet_abi_version() == 1
+    assert L.bitnet_abi_version() == 2
     assert L.bitnet_quantize_weights_workspace_size(4096, 4096) >= 80
 
 
@@ -88,6 +88,7 @@ def test_weights_validation(L):
                                                kw.get("ws", ALIGNED), kw.get("wsb", 128), None)
     assert w(dt=2) == 4
     assert w(K=24) == 2 and w(N=0) == 2 and w(N=1 << 20, K=1 << 12) == 2
+    assert w(N=1 << 40, K=1 << 40) == 2 and w(N=1 << 62, K=16) == 2      # products that would overflow
     assert w(ws=None) == 7 and w(wsb=8) == 7
     assert w(W=None) == 1
     assert w(pk=MISALIGNED) == 3
@@ -127,7 +128,7 @@ def test_trit5_validation(L):
     assert L.bitnet_trit5_row_bytes(81) == 32 and L.bitnet_trit5_row_bytes(0) == 0
     rp = lambda **kw: L.bitnet_repack_trit5(kw.get("pk", ALIGNED), kw.get("N", 8), kw.get("K", 512),
                                             kw.get("out", ALIGNED), None)
-    assert rp(K=24) == 2 and rp(K=0) == 2 and rp(N=0) == 2
+    assert rp(K=24) == 2 and rp(K=0) == 2 and rp(N=0) == 2 and rp(N=1 << 62, K=1 << 20) == 2
     assert rp(pk=None) == 1 and rp(out=None) == 1
     assert rp(pk=MISALIGNED) == 3 and rp(out=MISALIGNED) == 3
 
@@ -142,12 +143,19 @@ def test_trit5_validation(L):
     assert lt(pk=MISALIGNED) == 3 and lt(s_w=ALIGNED + 2) == 3
 
 
-def test_linear_path_selector(L):
-    assert L.bitnet_set_linear_path(5) == 2
-    assert L.bitnet_set_linear_path(4) == 0
-    assert L.bitnet_set_linear_path(3) == 0
-    assert L.bitnet_set_linear_path(-1) == 2
-    assert L.bitnet_set_linear_path(0) == 0
+def test_kernel_choice_is_per_call(L):
+    """The kernel family is an argument of the call (no process-wide switch):
+    values outside the documented ones are refused before anything is enqueued."""
+    lk = lambda kernel, **kw: L.bitnet_linear_kernel(ALIGNED, 8, ALIGNED, ALIGNED, ALIGNED, kw.get("M", 4), 256,
+                                                     kw.get("K", 256), ALIGNED, 0, None, kernel, None)
+    assert lk(4) == 2 and lk(-1) == 2
+    assert lk(3, M=33, K=512) == 2 and lk(3, K=384) == 2          # outside the decode kernel's range
+    assert lk(1, M=0) == 0 and lk(2, M=0) == 0
+    bk = lambda kernel, **kw: L.bitnet_bitlinear_kernel(ALIGNED, 1, kw.get("M", 4), kw.get("K", 512), None, 1e-6,
+                                                        ALIGNED, ALIGNED, 256, ALIGNED, 0, ALIGNED, ALIGNED, kernel,
+                                                        None)
+    assert bk(5) == 2 and bk(-1) == 2 and bk(4, M=0) == 0
+    assert not hasattr(api, "bitnet_set_linear_path")
 
 
 def test_oracle_and_product_share_no_code():

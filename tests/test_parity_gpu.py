@@ -205,15 +205,12 @@ def _random_codes(M, N, K, act_bits, seed):
 
 
 def _run_linear(qx, qw, s_x, s_w, act_bits, out, path):
-    api.bitnet_set_linear_path(path)
-    try:
-        xq_dev = dev(qx) if act_bits == 8 else dev(O.pack_int4(qx))
-        Y, acc = api.bitnet_linear(xq_dev, act_bits, dev(s_x), dev(O.pack_ternary(qw)),
-                                   dev(np.array([s_w], np.float32)),
-                                   out_dtype=torch.float32 if out == "f32" else torch.bfloat16, want_acc=True)
-        torch.cuda.synchronize()
-    finally:
-        api.bitnet_set_linear_path(0)
+    xq_dev = dev(qx) if act_bits == 8 else dev(O.pack_int4(qx))
+    Y, acc = api.bitnet_linear(xq_dev, act_bits, dev(s_x), dev(O.pack_ternary(qw)),
+                               dev(np.array([s_w], np.float32)),
+                               out_dtype=torch.float32 if out == "f32" else torch.bfloat16, want_acc=True,
+                               kernel=path)
+    torch.cuda.synchronize()
     return Y, acc
 
 
@@ -348,13 +345,9 @@ def _check_bitlinear(M, N, K, dtype, use_gamma, out, path=0, seed=0):
     gamma = rng.uniform(0.5, 1.5, K).astype(np.float32) if use_gamma else None
     w = wl.weights(N, K, seed=seed + N)
     pk, s_w = api.bitnet_quantize_weights(dev(w))
-    api.bitnet_set_linear_path(path)
-    try:
-        Y, q, s = api.bitnet_bitlinear(xd, pk, s_w, dev(gamma) if use_gamma else None, 1e-6,
-                                       out_dtype=torch.float32 if out == "f32" else torch.bfloat16)
-        torch.cuda.synchronize()
-    finally:
-        api.bitnet_set_linear_path(0)
+    Y, q, s = api.bitnet_bitlinear(xd, pk, s_w, dev(gamma) if use_gamma else None, 1e-6,
+                                   out_dtype=torch.float32 if out == "f32" else torch.bfloat16, kernel=path)
+    torch.cuda.synchronize()
     assert api.bitnet_device_error() == 0
     _, s_wo, qw_o = O.quantize_weights(w)
     q_o, s_o = O.quant_act(x_or, gamma, 1e-6)
@@ -466,6 +459,35 @@ def test_chain_two_layers(M, rows):
     for lw in ora_w:
         ref = O.chain_layer(ref, lw)
     assert np.array_equal(out[sel].view(np.uint32), ref.view(np.uint32))
+
+
+def test_chain_24_layers():
+    """All 24 stacked layers of the chain workload, each with its own weights, at
+    both batch sizes (32 decode tokens, 512 prefill tokens).  Every op is per
+    token, so the plain C++ oracle (held bit for bit to the numpy oracle by the
+    CPU tests; OpenMP over rows) follows sampled token rows through all 24
+    layers, from its own quantisation of the fp32 weights."""
+    from bitlinear_bitnet_quant_b200 import chain
+    from oracle import c_oracle as C
+    gpu_w, ora_w = [], []
+    for l in range(24):
+        w = wl.chain_weights(l)
+        gpu_w.append(chain.quantize_layer({k: dev(v) for k, v in w.items()}))
+        oq = {}
+        for k, v in w.items():
+            _, s_w, q = C.quantize_weights(v)
+            oq[k] = (q, s_w)
+        ora_w.append(oq)
+        del w
+    for M, rows in ((32, [0, 5, 18, 31]), (512, [0, 129, 300, 511])):
+        x = wl.chain_input(M)
+        ch = chain.BitLinearChain(gpu_w, M, wl.CHAIN_HIDDEN, wl.CHAIN_FFN, torch.device("cuda"))
+        out = host(ch.forward(dev(x)))
+        ref = x[rows]
+        for lw in ora_w:
+            ref = C.chain_layer(ref, lw)
+        assert np.all(np.isfinite(ref))
+        assert np.array_equal(out[rows].view(np.uint32), ref.view(np.uint32)), M
 
 
 @pytest.mark.parametrize("M,K,use_gamma", [(3, 2048, False), (32, 2048, True), (5, 16, False), (17, 5632, False),

@@ -67,8 +67,25 @@ def test_noalloc_matches_workspace_version_twice(L):
     assert np.array_equal(again[0], ref1[0]) and again[1] == ref1[1]
 
 
+def test_noalloc_zero_tensor_after_a_nonzero_one(L):
+    # an all-zero tensor right after a nonzero one: the floor scale 1/1e-5 and
+    # all-zero codes, exactly as the workspace version gives
+    w1 = torch.from_numpy(wl.weights(128, 512, seed=13)).cuda()
+    z = torch.zeros((128, 512), dtype=torch.float32, device="cuda")
+    _noalloc(L, w1, 0)
+    got = _noalloc(L, z, 0)
+    ref = _reference(z)
+    assert np.all(got[0] == 0) and np.array_equal(got[0], ref[0])
+    assert got[1].view(np.uint32) == ref[1].view(np.uint32)
+    assert got[1][0] == np.float32(1.0) / np.float32(1e-5)
+
+
 def test_noalloc_rejects_tensors_beyond_its_limit(L):
     big = 1 << 16                      # N*K = 2^32 > 2^31 - 1 weights
     st = L.bitnet_quantize_weights_noalloc(ctypes.c_void_p(0x10000), 0, big, big,
                                            ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10000), None)
     assert st == 2                     # BITNET_ERR_SHAPE, nothing enqueued
+    huge = 1 << 40                     # N*K would overflow 64 bits: still refused
+    st = L.bitnet_quantize_weights_noalloc(ctypes.c_void_p(0x10000), 0, huge, huge,
+                                           ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10000), None)
+    assert st == 2
