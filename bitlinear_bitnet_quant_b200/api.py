@@ -57,6 +57,10 @@ _SIGNATURES = {
     "bitnet_bitlinear_kernel": (ctypes.c_int, [_c_void_p, ctypes.c_int, _i64, _i64, _c_void_p, ctypes.c_float,
                                                _c_void_p, _c_void_p, _i64, _c_void_p, ctypes.c_int, _c_void_p,
                                                _c_void_p, ctypes.c_int, _c_void_p]),
+    "bitnet_linear_group": (ctypes.c_int, [_c_void_p, ctypes.c_int, _c_void_p, _i64, _i64, ctypes.c_int,
+                                           ctypes.POINTER(_c_void_p), ctypes.POINTER(_c_void_p),
+                                           ctypes.POINTER(_i64), ctypes.POINTER(_c_void_p), ctypes.c_int,
+                                           _c_void_p]),
     "bitnet_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
 }
 
@@ -226,6 +230,26 @@ def bitnet_linear(Xq: torch.Tensor, act_bits: int, s_x: torch.Tensor, pkW: torch
     else:
         _check("bitnet_linear", lib().bitnet_linear(*args, _stream(stream)))
     return Y, acc
+
+
+def bitnet_linear_group(Xq: torch.Tensor, act_bits: int, s_x: torch.Tensor, weights, out_dtype=torch.float32,
+                        Ys=None, stream=None):
+    """Several products sharing Xq and s_x in one launch.  weights: [(pkW, s_w), ...]
+    (1 to 4 entries, same K).  Returns the list of outputs [M, N_g]."""
+    _require(Xq, "Xq")
+    M = Xq.shape[0]
+    count = len(weights)
+    K = weights[0][0].shape[1] * 4
+    for pk, _ in weights:
+        _require(pk, "pkW")
+    if Ys is None:
+        Ys = [torch.empty((M, pk.shape[0]), dtype=out_dtype, device=Xq.device) for pk, _ in weights]
+    arr = lambda ts: (_c_void_p * count)(*[t.data_ptr() for t in ts])
+    Ns = (_i64 * count)(*[pk.shape[0] for pk, _ in weights])
+    _check("bitnet_linear_group", lib().bitnet_linear_group(
+        _ptr(Xq), int(act_bits), _ptr(s_x), M, K, count, arr([w[0] for w in weights]), arr([w[1] for w in weights]),
+        Ns, arr(Ys), _dtype_code(Ys[0]), _stream(stream)))
+    return Ys
 
 
 def bitnet_trit5_row_bytes(K: int) -> int:

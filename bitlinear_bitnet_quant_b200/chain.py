@@ -5,11 +5,13 @@ linear layers of attention and FFN are BitLinear (int8 activations), and in
 BitNet v2 the O and down projections are H-BitLinear (Hadamard + int4).
 Per layer, with fp32 residuals:
 
-    q, k, v = BitLinear(x)                      (one int8 quantisation of x)
+    q, k, v = BitLinear(x)                      (one int8 quantisation of x,
+                                                 one launch for the three)
     o = H-BitLinear(v)                          (attention over a one-token
                                                  context returns V)
     h = x + o
-    up, gate = BitLinear(h)                     (one int8 quantisation of h)
+    up, gate = BitLinear(h)                     (one int8 quantisation of h,
+                                                 one launch for the two)
     a = relu(gate)^2 * up                       (squared-ReLU gated unit)
     x' = h + H-BitLinear(a)                     (down projection)
 
@@ -66,13 +68,11 @@ class BitLinearChain:
         else:
             x = self.x[0]
             A.bitnet_add_quant_act(x_parts[0], x_parts[1], None, self.eps, H=x, Xq=self.xq, s_x=self.sx, stream=s)
-        for name, Y in (("q", self.q), ("k", self.k), ("v", self.v)):
-            A.bitnet_linear(self.xq, 8, self.sx, *w[name], Y=Y, stream=s)
+        A.bitnet_linear_group(self.xq, 8, self.sx, [w["q"], w["k"], w["v"]], Ys=[self.q, self.k, self.v], stream=s)
         A.bitnet_hadamard_quant_act(self.v, None, self.eps, 0, Xq4=self.v4, s_x=self.sv, stream=s)
         A.bitnet_linear(self.v4, 4, self.sv, *w["o"], Y=self.o, stream=s)
         A.bitnet_add_quant_act(x, self.o, None, self.eps, H=self.h, Xq=self.hq, s_x=self.sh, stream=s)
-        A.bitnet_linear(self.hq, 8, self.sh, *w["up"], Y=self.up, stream=s)
-        A.bitnet_linear(self.hq, 8, self.sh, *w["gate"], Y=self.gate, stream=s)
+        A.bitnet_linear_group(self.hq, 8, self.sh, [w["up"], w["gate"]], Ys=[self.up, self.gate], stream=s)
         A.bitnet_glu_hadamard_quant_act(self.gate, self.up, None, self.eps, 0, Xq4=self.a4, s_x=self.sa, stream=s)
         A.bitnet_linear(self.a4, 4, self.sa, *w["down"], Y=self.d, stream=s)
         return self.h, self.d
@@ -87,12 +87,13 @@ class BitLinearChain:
         return self.x[1]
 
     # kernels launched per forward: per layer 2 int8 quantisers (the second, and
-    # from the second layer on the first, with the residual add folded in), 7
-    # linear layers, 2 Hadamard quantisers (one with the gated unit folded in);
-    # one residual add after the last layer
+    # from the second layer on the first, with the residual add folded in), 4
+    # linear launches (Q/K/V in one, O, up/gate in one, down), 2 Hadamard
+    # quantisers (one with the gated unit folded in); one residual add after
+    # the last layer
     @property
     def launches(self) -> int:
-        return 11 * len(self.layers) + 1
+        return 8 * len(self.layers) + 1
 
     def packed_bytes(self) -> int:
         return sum(pk.numel() for w in self.layers for pk, _ in w.values())

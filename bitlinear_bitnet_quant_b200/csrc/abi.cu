@@ -6,6 +6,7 @@
 #include <atomic>
 
 #include "../../include/bitnet.h"
+#include "common.cuh"
 
 namespace bitnet {
 __device__ int g_device_error = 0;
@@ -19,6 +20,8 @@ cudaError_t run_hadamard_quant_i4(const void* X, int bf16, int M, int K, int L, 
                                   float eps, uint8_t* Xq4, float* s_x, float* T_dbg, cudaStream_t st);
 cudaError_t run_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                        int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, int path, cudaStream_t st);
+cudaError_t run_linear_group(const LinGroup& grp, const void* Xq, int act_bits, const float* s_x, int M, int K,
+                             int y_bf16, int path, cudaStream_t st);
 bool tensor_map_encoder_available();
 cudaError_t run_add_quant_act_i8(const float* A, const float* B, int M, int K, const float* gamma, float eps,
                                  float* H, int8_t* Xq, float* s_x, cudaStream_t st);
@@ -209,6 +212,39 @@ int bitnet_linear_kernel(const void* Xq, int act_bits, const float* s_x, const u
                          int64_t M, int64_t N, int64_t K, void* Y, int y_dtype, int32_t* acc_dbg, int kernel,
                          void* stream) {
   return linear_impl(Xq, act_bits, s_x, pkW, s_w, M, N, K, Y, y_dtype, acc_dbg, kernel, stream);
+}
+
+int bitnet_linear_group(const void* Xq, int act_bits, const float* s_x, int64_t M, int64_t K, int count,
+                        const uint8_t* const* pkW, const float* const* s_w, const int64_t* N, void* const* Y,
+                        int y_dtype, void* stream) {
+  if (act_bits != 8 && act_bits != 4) return BITNET_ERR_DTYPE;
+  if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (count < 1 || count > bitnet::GROUP_MAX) return BITNET_ERR_SHAPE;
+  if (!pkW || !s_w || !N || !Y) return BITNET_ERR_NULL;
+  if (M < 0 || M > (int64_t(1) << 30) || K < 128 || K > 65536 || K % 128 != 0) return BITNET_ERR_SHAPE;
+  for (int g = 0; g < count; ++g)
+    if (N[g] < 1 || N[g] > (int64_t(1) << 30) || M * N[g] >= (int64_t(1) << 40)) return BITNET_ERR_SHAPE;
+  if (M == 0) return BITNET_OK;
+  if (!Xq || !s_x) return BITNET_ERR_NULL;
+  for (int g = 0; g < count; ++g) {
+    if (!pkW[g] || !s_w[g] || !Y[g]) return BITNET_ERR_NULL;
+    if (!aligned16(pkW[g]) || !aligned16(Y[g]) || (reinterpret_cast<uintptr_t>(s_w[g]) & 3u)) return BITNET_ERR_ALIGN;
+  }
+  if (!aligned16(Xq) || (reinterpret_cast<uintptr_t>(s_x) & 3u)) return BITNET_ERR_ALIGN;
+  int d = check_device();
+  if (d != BITNET_OK) return d;
+  if (!bitnet::tensor_map_encoder_available()) return BITNET_ERR_UNSUPPORTED;
+  bitnet::LinGroup grp = {};
+  for (int g = 0; g < count; ++g) {
+    grp.pkW[g] = pkW[g];
+    grp.s_w[g] = s_w[g];
+    grp.Y[g] = Y[g];
+    grp.acc_dbg[g] = nullptr;
+    grp.N[g] = (int)N[g];
+  }
+  grp.count = count;
+  return cuda_status(bitnet::run_linear_group(grp, Xq, act_bits, s_x, (int)M, (int)K, y_dtype == BITNET_BF16, 0,
+                                              static_cast<cudaStream_t>(stream)));
 }
 
 size_t bitnet_trit5_row_bytes(int64_t K) {

@@ -31,6 +31,32 @@ enum DeviceError : int {
 };
 
 // ---------------------------------------------------------------------------
+// A group of ternary weight matrices that share one activation tensor (the
+// Q/K/V projections of an attention block, the up/gate projections of a gated
+// FFN), computed by one launch.  A single product is a group of one.  CTAs (or
+// output tiles) first[g] .. first[g+1]-1 of the grid work on matrix g.
+// ---------------------------------------------------------------------------
+constexpr int GROUP_MAX = 4;
+
+struct LinGroup {
+  const uint8_t* pkW[GROUP_MAX];
+  const float* s_w[GROUP_MAX];
+  void* Y[GROUP_MAX];
+  int32_t* acc_dbg[GROUP_MAX];
+  int N[GROUP_MAX];
+  int first[GROUP_MAX + 1];
+  int count;
+};
+
+// Index of the matrix that block b works on (uniform across the CTA).
+BN_DEV int group_of(const LinGroup& g, int b) {
+  int gi = 0;
+#pragma unroll
+  for (int j = 1; j < GROUP_MAX; ++j) gi += (j < g.count && b >= g.first[j]) ? 1 : 0;
+  return gi;
+}
+
+// ---------------------------------------------------------------------------
 // bf16 / vector helpers
 // ---------------------------------------------------------------------------
 BN_DEV float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }

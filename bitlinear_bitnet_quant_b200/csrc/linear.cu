@@ -165,12 +165,17 @@ BN_DEV void load_cols(uint32_t taddr, uint32_t (&v)[G][16]) {
   tmem_wait_ld();
 }
 
+// Tensor maps of a group's weight matrices and outputs (see LinGroup).
+struct TcMaps {
+  CUtensorMap w[GROUP_MAX];
+  CUtensorMap y[GROUP_MAX];
+};
+
 template <int BN, int ACT_BITS, typename TOut>
 __global__ void __launch_bounds__(TC_THREADS, BN <= 128 ? 2 : 1)
-linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                 const __grid_constant__ CUtensorMap tmY, int use_tma_store,
-                 const float* __restrict__ s_x, const float* __restrict__ s_w_ptr,
-                 int M, int N, int K, int ksplit, TOut* __restrict__ Y, int32_t* __restrict__ acc_dbg) {
+linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CUtensorMap tmX,
+                 const __grid_constant__ LinGroup grp, int use_tma_store, const float* __restrict__ s_x,
+                 int M, int K, int ksplit) {
   using C = TcCfg<BN, ACT_BITS>;
   constexpr int S = C::S;
   constexpr uint32_t XTX = ACT_BITS == 8 ? BN * 128 : BN * 64;      // activation bytes per stage
@@ -198,7 +203,15 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
   TOut* ostage = reinterpret_cast<TOut*>(base);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * 128;
+  // the weight matrix of this tile (one of a group that shares the activations)
+  const int gi = group_of(grp, blockIdx.x);
+  const CUtensorMap* tmW = &maps.w[gi];
+  const CUtensorMap* tmY = &maps.y[gi];
+  const float* __restrict__ s_w_ptr = grp.s_w[gi];
+  TOut* __restrict__ Y = static_cast<TOut*>(grp.Y[gi]);
+  int32_t* __restrict__ acc_dbg = grp.acc_dbg[gi];
+  const int N = grp.N[gi];
+  const int n0 = (blockIdx.x - grp.first[gi]) * 128;
   const int m0 = blockIdx.y * BN;
   const int kr = blockIdx.z;                    // rank inside the cluster (cluster = 1 x 1 x ksplit)
   const int nk_all = K / TC_BK;
@@ -217,7 +230,7 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
     mbar_init(&bar_red, 1);
     fence_barrier_init();
     if (kr == 0 && ksplit > 1) mbar_arrive_expect_tx(&bar_red, (uint32_t)(ksplit - 1) * PART_BYTES);
-    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(tmW);
     tma_prefetch_desc(&tmX);
   }
   if (warp == 1) {
@@ -241,7 +254,7 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       // weights do not depend on the previous kernel: start streaming them now
       for (int i = 0; i < pre; ++i) {
         mbar_arrive_expect_tx(&bar_wfull[i], TC_WBYTES);
-        tma_load_2d(ws(i), &tmW, &bar_wfull[i], (kb + i) * (TC_BK / 4), n0);
+        tma_load_2d(ws(i), tmW, &bar_wfull[i], (kb + i) * (TC_BK / 4), n0);
       }
     }
     __syncwarp();
@@ -255,7 +268,7 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
     if (lane == 0)
       for (int i = 0; i < pre; ++i) load_x(i);    // first: the activations are on the critical path
     if (kr == 0) {
-      if (lane == 0 && use_tma_store) tma_prefetch_desc(&tmY);
+      if (lane == 0 && use_tma_store) tma_prefetch_desc(tmY);
       const float sw = ldg_nc_f32(s_w_ptr);
       for (int j = lane; j < BN; j += 32) {
         const int m = m0 + j;
@@ -270,7 +283,7 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
         const int s = i % S, r = i / S;
         if (!mbar_wait(&bar_empty[s], (r - 1) & 1, DEV_ERR_TIMEOUT_EMPTY)) break;
         mbar_arrive_expect_tx(&bar_wfull[s], TC_WBYTES);
-        tma_load_2d(ws(s), &tmW, &bar_wfull[s], (kb + i) * (TC_BK / 4), n0);
+        tma_load_2d(ws(s), tmW, &bar_wfull[s], (kb + i) * (TC_BK / 4), n0);
         load_x(i);
         issued = i + 1;
       }
@@ -426,7 +439,7 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
         fence_proxy_async_smem();
         asm volatile("bar.sync 1, 256;" ::: "memory");
         if (ct == 0 && ok) {
-          tma_store_2d(&tmY, ostage, n0, m0);
+          tma_store_2d(tmY, ostage, n0, m0);
           bulk_wait_all();
         }
       }
@@ -485,26 +498,39 @@ template <> struct MapType<float> { static constexpr CUtensorMapDataType v = CU_
 template <> struct MapType<__nv_bfloat16> { static constexpr CUtensorMapDataType v = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; };
 
 template <int BN, int ACT_BITS, typename TOut>
-static cudaError_t launch_tc(const void* Xq, const float* s_x, const uint8_t* pkW, const float* s_w,
-                             int M, int N, int K, void* Y, int32_t* acc_dbg, cudaStream_t st) {
+static cudaError_t launch_tc(LinGroup grp, const void* Xq, const float* s_x, int M, int K, cudaStream_t st) {
   using C = TcCfg<BN, ACT_BITS>;
-  CUtensorMap tmW, tmX, tmY;
-  if (!make_map_bytes(&tmW, pkW, (uint64_t)K / 4, (uint64_t)N, TC_BK / 4, 128, CU_TENSOR_MAP_SWIZZLE_32B))
-    return cudaErrorInvalidValue;
+  TcMaps maps;                                     // copied into the launch's parameters
+  CUtensorMap tmX;
   const bool ok = ACT_BITS == 8
       ? make_map_bytes(&tmX, Xq, (uint64_t)K, (uint64_t)M, TC_BK, BN, CU_TENSOR_MAP_SWIZZLE_128B)
       : make_map_bytes(&tmX, Xq, (uint64_t)K / 2, (uint64_t)M, TC_BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
   // The output leaves through one TMA store per tile when rows are 16-byte
   // multiples; the diagnostics accumulators take the per-element path.
-  int use_tma_store = acc_dbg == nullptr && ((uint64_t)N * sizeof(TOut)) % 16 == 0;
-  if (use_tma_store && !make_map_2d(&tmY, Y, MapType<TOut>::v, (uint64_t)N, (uint64_t)M, (uint64_t)N * sizeof(TOut),
-                                     128, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
-    use_tma_store = 0;
-  if (!use_tma_store) tmY = tmX;                   // unused
+  int use_tma_store = 1;
+  for (int g = 0; g < grp.count; ++g)
+    if (grp.acc_dbg[g] != nullptr || ((uint64_t)grp.N[g] * sizeof(TOut)) % 16 != 0) use_tma_store = 0;
+  grp.first[0] = 0;
+  for (int g = 0; g < grp.count; ++g) {
+    if (!make_map_bytes(&maps.w[g], grp.pkW[g], (uint64_t)K / 4, (uint64_t)grp.N[g], TC_BK / 4, 128,
+                        CU_TENSOR_MAP_SWIZZLE_32B))
+      return cudaErrorInvalidValue;
+    if (use_tma_store && !make_map_2d(&maps.y[g], grp.Y[g], MapType<TOut>::v, (uint64_t)grp.N[g], (uint64_t)M,
+                                      (uint64_t)grp.N[g] * sizeof(TOut), 128, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    if (!use_tma_store) maps.y[g] = tmX;           // unused
+    grp.first[g + 1] = grp.first[g] + (grp.N[g] + 127) / 128;
+  }
+  for (int g = grp.count; g < GROUP_MAX; ++g) {
+    maps.w[g] = maps.w[0];
+    maps.y[g] = maps.y[0];
+    grp.first[g + 1] = grp.first[grp.count];
+  }
   // Split K across a cluster when the output tiles alone leave most SMs idle
   // (decode): each rank streams a K range, partial sums meet in the leader.
-  const int tiles = ((N + 127) / 128) * ((M + BN - 1) / BN);
+  const int ntiles = grp.first[grp.count];
+  const int tiles = ntiles * ((M + BN - 1) / BN);
   const int nk = K / TC_BK;
   int ksplit = 1;
   if (BN <= 32) {
@@ -522,18 +548,17 @@ static cudaError_t launch_tc(const void* Xq, const float* s_x, const uint8_t* pk
   auto kern = linear_tc_kernel<BN, ACT_BITS, TOut>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((N + 127) / 128, (M + BN - 1) / BN, ksplit);
-  return launch_pdl(kern, grid, dim3(TC_THREADS), smem, st, dim3(1, 1, ksplit), tmW, tmX, tmY, use_tma_store,
-                    s_x, s_w, M, N, K, ksplit, static_cast<TOut*>(Y), acc_dbg);
+  dim3 grid(ntiles, (M + BN - 1) / BN, ksplit);
+  return launch_pdl(kern, grid, dim3(TC_THREADS), smem, st, dim3(1, 1, ksplit), maps, tmX, grp, use_tma_store,
+                    s_x, M, K, ksplit);
 }
 
 template <int ACT_BITS, typename TOut>
-static cudaError_t dispatch_tc(const void* Xq, const float* s_x, const uint8_t* pkW, const float* s_w,
-                               int M, int N, int K, void* Y, int32_t* acc_dbg, cudaStream_t st) {
-  if (M <= 16) return launch_tc<16, ACT_BITS, TOut>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st);
-  if (M <= 32) return launch_tc<32, ACT_BITS, TOut>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st);
-  if (M <= 64) return launch_tc<64, ACT_BITS, TOut>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st);
-  return launch_tc<128, ACT_BITS, TOut>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st);
+static cudaError_t dispatch_tc(const LinGroup& grp, const void* Xq, const float* s_x, int M, int K, cudaStream_t st) {
+  if (M <= 16) return launch_tc<16, ACT_BITS, TOut>(grp, Xq, s_x, M, K, st);
+  if (M <= 32) return launch_tc<32, ACT_BITS, TOut>(grp, Xq, s_x, M, K, st);
+  if (M <= 64) return launch_tc<64, ACT_BITS, TOut>(grp, Xq, s_x, M, K, st);
+  return launch_tc<128, ACT_BITS, TOut>(grp, Xq, s_x, M, K, st);
 }
 
 template <int ACT_BITS, typename TOut>
@@ -550,24 +575,49 @@ bool tensor_map_encoder_available() { return get_encode() != nullptr; }
 bool decode_path_applies(int M, int K);
 cudaError_t run_linear_decode(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                               int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, cudaStream_t st);
+cudaError_t run_linear_decode_group(const LinGroup& grp, const void* Xq, int act_bits, const float* s_x, int M, int K,
+                                    int y_bf16, cudaStream_t st);
+
+cudaError_t run_linear_group(const LinGroup& grp, const void* Xq, int act_bits, const float* s_x, int M, int K,
+                             int y_bf16, int path, cudaStream_t st);
 
 // path: 0 = automatic, 1 = SIMT, 2 = tcgen05, 3 = warp-MMA decode kernel
 cudaError_t run_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                        int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, int path, cudaStream_t st) {
-  // up to 16 tokens: one pass over the weights with warp-level MMA
+  // up to 32 tokens: one pass over the weights with warp-level MMA
   if ((path == 0 || path == 3) && decode_path_applies(M, K))
     return run_linear_decode(Xq, act_bits, s_x, pkW, s_w, M, N, K, Y, y_bf16, acc_dbg, st);
   if (path == 3) return cudaErrorInvalidValue;
-  const bool tc = path != 1;          // the dp4a kernel is a diagnostics path (slower at every M)
-#define BN_LIN(BITS, T)                                                                  \
-  return tc ? dispatch_tc<BITS, T>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st)           \
-            : launch_simt<BITS, T>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st)
-  if (act_bits == 8) {
-    if (y_bf16) { BN_LIN(8, __nv_bfloat16); } else { BN_LIN(8, float); }
-  } else {
-    if (y_bf16) { BN_LIN(4, __nv_bfloat16); } else { BN_LIN(4, float); }
-  }
+  if (path == 1) {                    // the dp4a kernel is a diagnostics path (slower at every M)
+#define BN_LIN(BITS, T) return launch_simt<BITS, T>(Xq, s_x, pkW, s_w, M, N, K, Y, acc_dbg, st)
+    if (act_bits == 8) {
+      if (y_bf16) { BN_LIN(8, __nv_bfloat16); } else { BN_LIN(8, float); }
+    } else {
+      if (y_bf16) { BN_LIN(4, __nv_bfloat16); } else { BN_LIN(4, float); }
+    }
 #undef BN_LIN
+  }
+  LinGroup grp = {};
+  grp.pkW[0] = pkW;
+  grp.s_w[0] = s_w;
+  grp.Y[0] = Y;
+  grp.acc_dbg[0] = acc_dbg;
+  grp.N[0] = N;
+  grp.count = 1;
+  return run_linear_group(grp, Xq, act_bits, s_x, M, K, y_bf16, 2, st);
+}
+
+// Several weight matrices sharing Xq and s_x in one launch.  path: 0 = automatic,
+// 2 = tcgen05, 3 = warp-MMA decode kernel.
+cudaError_t run_linear_group(const LinGroup& grp, const void* Xq, int act_bits, const float* s_x, int M, int K,
+                             int y_bf16, int path, cudaStream_t st) {
+  if ((path == 0 || path == 3) && decode_path_applies(M, K))
+    return run_linear_decode_group(grp, Xq, act_bits, s_x, M, K, y_bf16, st);
+  if (path == 3) return cudaErrorInvalidValue;
+  if (act_bits == 8) {
+    return y_bf16 ? dispatch_tc<8, __nv_bfloat16>(grp, Xq, s_x, M, K, st) : dispatch_tc<8, float>(grp, Xq, s_x, M, K, st);
+  }
+  return y_bf16 ? dispatch_tc<4, __nv_bfloat16>(grp, Xq, s_x, M, K, st) : dispatch_tc<4, float>(grp, Xq, s_x, M, K, st);
 }
 
 }  // namespace bitnet

@@ -46,11 +46,12 @@ namespace bitnet {
 // onwards and tokens 8 * TG * (b % tsplit) onwards.  W5: pkW holds the weights
 // five per byte (trit5_row_bytes(K) bytes per row), rewritten into the 2-bit
 // slice layout in shared memory before the dependency wait.
+// A group of weight matrices sharing the activations runs in one launch: CTAs
+// grp.first[g] .. grp.first[g+1]-1 stream matrix g (see LinGroup).
 template <int ACT_BITS, int TG, int RG, typename TOut, bool W5>
 __global__ void __launch_bounds__(DEC_THREADS, 2)
-linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict__ Xq,
-                     const float* __restrict__ s_x, const float* __restrict__ s_w_ptr, int M, int N, int K,
-                     int tsplit, TOut* __restrict__ Y, int32_t* __restrict__ acc_dbg) {
+linear_decode_kernel(const __grid_constant__ LinGroup grp, const uint8_t* __restrict__ Xq,
+                     const float* __restrict__ s_x, int M, int K, int tsplit) {
   using C = DecCfg<TG>;
   constexpr int TOK = C::TOK, PB = C::PASS_BATCH;
   constexpr int ROWS = 16 * RG;
@@ -65,10 +66,17 @@ linear_decode_kernel(const uint8_t* __restrict__ pkW, const uint8_t* __restrict_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int nseg = K / 512;
-  const int n0 = (blockIdx.x / tsplit) * ROWS;
+  const int gi = group_of(grp, blockIdx.x);
+  const int blk = blockIdx.x - grp.first[gi];
+  const uint8_t* __restrict__ pkW = grp.pkW[gi];
+  const float* __restrict__ s_w_ptr = grp.s_w[gi];
+  TOut* __restrict__ Y = static_cast<TOut*>(grp.Y[gi]);
+  int32_t* __restrict__ acc_dbg = grp.acc_dbg[gi];
+  const int N = grp.N[gi];
+  const int n0 = (blk / tsplit) * ROWS;
   const size_t xrow = ACT_BITS == 8 ? (size_t)K : (size_t)K / 2;
   {
-    const int m0 = (blockIdx.x % tsplit) * TOK;     // this CTA's first token
+    const int m0 = (blk % tsplit) * TOK;            // this CTA's first token
     M = M - m0 < TOK ? M - m0 : TOK;
     Xq += (size_t)m0 * xrow;
     s_x += m0;
@@ -174,30 +182,35 @@ static size_t dec_smem_bytes(int K, bool w5) {
 }
 
 template <int ACT_BITS, int TG, int RG, typename TOut, bool W5>
-static cudaError_t launch_decode_rg(const void* Xq, const float* s_x, const uint8_t* pkW, const float* s_w, int M,
-                                    int N, int K, int tsplit, void* Y, int32_t* acc_dbg, cudaStream_t st) {
+static cudaError_t launch_decode_rg(LinGroup grp, const void* Xq, const float* s_x, int M, int K, int tsplit,
+                                    cudaStream_t st) {
   constexpr int ROWS = 16 * RG;
   const size_t smem = dec_smem_bytes<TG, RG>(K, W5);
   auto kern = linear_decode_kernel<ACT_BITS, TG, RG, TOut, W5>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)((N + ROWS - 1) / ROWS * tsplit));
-  return launch_pdl(kern, grid, dim3(DEC_THREADS), smem, st, 1u, pkW, static_cast<const uint8_t*>(Xq), s_x, s_w, M, N,
-                    K, tsplit, static_cast<TOut*>(Y), acc_dbg);
+  grp.first[0] = 0;
+  for (int g = 0; g < grp.count; ++g) grp.first[g + 1] = grp.first[g] + (grp.N[g] + ROWS - 1) / ROWS * tsplit;
+  for (int g = grp.count + 1; g <= GROUP_MAX; ++g) grp.first[g] = grp.first[grp.count];
+  const dim3 grid((unsigned)grp.first[grp.count]);
+  return launch_pdl(kern, grid, dim3(DEC_THREADS), smem, st, 1u, grp, static_cast<const uint8_t*>(Xq), s_x, M, K,
+                    tsplit);
 }
 
 template <int ACT_BITS, int TG, typename TOut, bool W5>
-static cudaError_t launch_decode_t(const void* Xq, const float* s_x, const uint8_t* pkW, const float* s_w, int M,
-                                   int N, int K, int tsplit, void* Y, int32_t* acc_dbg, cudaStream_t st) {
+static cudaError_t launch_decode_t(const LinGroup& grp, const void* Xq, const float* s_x, int M, int K, int tsplit,
+                                   cudaStream_t st) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int n_all = 0;
+  for (int g = 0; g < grp.count; ++g) n_all += grp.N[g];
   // one CTA per weight slice (up to 8 tokens): slices sized for two CTAs per
   // SM, which halves each warp's MMA chain (measured on B200: 8 tokens
   // 3.5 -> 2.9 us at N = 6912, K = 2560); with the token groups spread over
   // CTAs the grid already holds two per SM
-  const int rg = decode_rows(N, K, sms * (tsplit == 1 ? 2 : 1), DecCfg<TG>::MAX_ROWS) / 16;
-#define BN_RG(R) launch_decode_rg<ACT_BITS, TG, (R <= DecCfg<TG>::RG_MAX ? R : 1), TOut, W5>(Xq, s_x, pkW, s_w, M, N, K, tsplit, Y, acc_dbg, st)
+  const int rg = decode_rows(n_all, K, sms * (tsplit == 1 ? 2 : 1), DecCfg<TG>::MAX_ROWS) / 16;
+#define BN_RG(R) launch_decode_rg<ACT_BITS, TG, (R <= DecCfg<TG>::RG_MAX ? R : 1), TOut, W5>(grp, Xq, s_x, M, K, tsplit, st)
   switch (rg) {
     case 1: return BN_RG(1);
     case 2: return BN_RG(2);
@@ -208,15 +221,14 @@ static cudaError_t launch_decode_t(const void* Xq, const float* s_x, const uint8
 }
 
 template <bool W5>
-static cudaError_t dispatch_decode(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW,
-                                   const float* s_w, int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg,
-                                   cudaStream_t st) {
+static cudaError_t dispatch_decode(const LinGroup& grp, const void* Xq, int act_bits, const float* s_x, int M, int K,
+                                   int y_bf16, cudaStream_t st) {
   // up to 16 tokens: one token group per CTA (two CTAs per weight slice past
   // 8 tokens); up to 32: two token groups per CTA, two CTAs per slice
-#define BN_DEC(BITS, T)                                                                                   \
-  return M <= 8    ? launch_decode_t<BITS, 1, T, W5>(Xq, s_x, pkW, s_w, M, N, K, 1, Y, acc_dbg, st)      \
-         : M <= 16 ? launch_decode_t<BITS, 1, T, W5>(Xq, s_x, pkW, s_w, M, N, K, 2, Y, acc_dbg, st)      \
-                   : launch_decode_t<BITS, 2, T, W5>(Xq, s_x, pkW, s_w, M, N, K, (M + 15) / 16, Y, acc_dbg, st)
+#define BN_DEC(BITS, T)                                                                     \
+  return M <= 8    ? launch_decode_t<BITS, 1, T, W5>(grp, Xq, s_x, M, K, 1, st)            \
+         : M <= 16 ? launch_decode_t<BITS, 1, T, W5>(grp, Xq, s_x, M, K, 2, st)            \
+                   : launch_decode_t<BITS, 2, T, W5>(grp, Xq, s_x, M, K, (M + 15) / 16, st)
   if (act_bits == 8) {
     if (y_bf16) { BN_DEC(8, __nv_bfloat16); } else { BN_DEC(8, float); }
   } else {
@@ -225,9 +237,26 @@ static cudaError_t dispatch_decode(const void* Xq, int act_bits, const float* s_
 #undef BN_DEC
 }
 
+static LinGroup single_group(const uint8_t* pkW, const float* s_w, int N, void* Y, int32_t* acc_dbg) {
+  LinGroup g = {};
+  g.pkW[0] = pkW;
+  g.s_w[0] = s_w;
+  g.Y[0] = Y;
+  g.acc_dbg[0] = acc_dbg;
+  g.N[0] = N;
+  g.count = 1;
+  return g;
+}
+
 cudaError_t run_linear_decode(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                               int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, cudaStream_t st) {
-  return dispatch_decode<false>(Xq, act_bits, s_x, pkW, s_w, M, N, K, Y, y_bf16, acc_dbg, st);
+  return dispatch_decode<false>(single_group(pkW, s_w, N, Y, acc_dbg), Xq, act_bits, s_x, M, K, y_bf16, st);
+}
+
+// Several weight matrices that share the activations, in one launch.
+cudaError_t run_linear_decode_group(const LinGroup& grp, const void* Xq, int act_bits, const float* s_x, int M, int K,
+                                    int y_bf16, cudaStream_t st) {
+  return dispatch_decode<false>(grp, Xq, act_bits, s_x, M, K, y_bf16, st);
 }
 
 // Weights five per byte (trit5_row_bytes(K) bytes per row); same shapes as the
@@ -235,7 +264,7 @@ cudaError_t run_linear_decode(const void* Xq, int act_bits, const float* s_x, co
 cudaError_t run_linear_decode_trit5(const void* Xq, int act_bits, const float* s_x, const uint8_t* pk5,
                                     const float* s_w, int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg,
                                     cudaStream_t st) {
-  return dispatch_decode<true>(Xq, act_bits, s_x, pk5, s_w, M, N, K, Y, y_bf16, acc_dbg, st);
+  return dispatch_decode<true>(single_group(pk5, s_w, N, Y, acc_dbg), Xq, act_bits, s_x, M, K, y_bf16, st);
 }
 
 }  // namespace bitnet

@@ -195,6 +195,24 @@ BITNET_API int bitnet_linear(const void* Xq, int act_bits, const float* s_x, con
                   void* Y, int y_dtype, int32_t* acc_dbg, void* stream);
 
 /*
+ * Several ternary products that share one quantised activation tensor, in one
+ * launch: the Q, K and V projections of an attention block, or the up and gate
+ * projections of a gated FFN ("AI 혁신의 선두: 마이크로소프트의 1비트 LLM, BitNet
+ * b1.58 2B4T", 주요 아키텍처 혁신: every linear layer of attention and FFN is a
+ * BitLinear; P4 계산 패러다임 for the product itself).  For g < count,
+ *   Y[g] = bitnet_linear(Xq, act_bits, s_x, pkW[g], s_w[g], M, N[g], K),
+ * bit for bit.  One launch streams every matrix of the group, so its fixed
+ * costs (the wait on the previous kernel, the pipeline fill) are paid once.
+ * pkW, s_w, N, Y: HOST arrays of `count` entries holding device pointers and
+ *                 sizes; they are read during the call only.
+ * Limits: 1 <= count <= 4; M, K and each N[g] as for bitnet_linear; one
+ *         y_dtype for all outputs; no accumulator output.
+ */
+BITNET_API int bitnet_linear_group(const void* Xq, int act_bits, const float* s_x, int64_t M, int64_t K,
+                                   int count, const uint8_t* const* pkW, const float* const* s_w,
+                                   const int64_t* N, void* const* Y, int y_dtype, void* stream);
+
+/*
  * Denser weight storage: five ternary weights per byte as base-3 digits,
  * 1.6 bits per weight instead of 2 ("양자화(quantization) 1.58bit", section
  * "1.58비트는 어디서 나온거에요?": three states carry log2(3) = 1.58 bits).

@@ -143,6 +143,23 @@ def test_trit5_validation(L):
     assert lt(pk=MISALIGNED) == 3 and lt(s_w=ALIGNED + 2) == 3
 
 
+def test_linear_group_validation(L):
+    import ctypes
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+
+    def grp(count=2, N=(256, 128), pk=ALIGNED, Y=ALIGNED, sw=ALIGNED, M=4, K=512, bits=8, yt=0, Xq=ALIGNED,
+            n_arr=True):
+        ptrs = lambda v: (P * 4)(*([v] * 4))
+        Ns = (I64 * 4)(*(list(N) + [128] * (4 - len(N)))) if n_arr else None
+        return L.bitnet_linear_group(Xq, bits, ALIGNED, M, K, count, ptrs(pk), ptrs(sw), Ns, ptrs(Y), yt, None)
+    assert grp(bits=5) == 4 and grp(yt=2) == 4
+    assert grp(count=0) == 2 and grp(count=5) == 2
+    assert grp(K=100) == 2 and grp(N=(256, 0)) == 2 and grp(M=-1) == 2
+    assert grp(M=0) == 0
+    assert grp(n_arr=False) == 1 and grp(pk=None) == 1 and grp(Xq=None) == 1
+    assert grp(pk=MISALIGNED) == 3 and grp(Y=MISALIGNED) == 3 and grp(sw=ALIGNED + 2) == 3
+
+
 def test_kernel_choice_is_per_call(L):
     """The kernel family is an argument of the call (no process-wide switch):
     values outside the documented ones are refused before anything is enqueued."""

@@ -336,6 +336,43 @@ def test_linear_decode_full(M):
     assert np.array_equal(host(Y).view(np.uint32), y_o.view(np.uint32))
 
 
+@pytest.mark.parametrize("M,K,Ns,act_bits,out", [
+    (1, 2048, [2048, 2048, 2048], 8, "f32"),          # the chain's Q/K/V at one token
+    (16, 2560, [6912, 128], 8, "bf16"),
+    (32, 2048, [5632, 5632], 8, "f32"),               # up/gate at the chain's decode batch
+    (9, 1024, [200, 1000, 48, 16], 4, "f32"),         # ragged N, int4 activations, four matrices
+    (33, 512, [384, 130], 8, "f32"),                  # tensor-core kernel, ragged N
+    (130, 1024, [256, 520, 128], 4, "bf16"),
+    (512, 2048, [2048, 2048, 2048], 8, "f32"),        # the chain's Q/K/V at 512 tokens
+])
+def test_linear_group(M, K, Ns, act_bits, out):
+    """Several matrices sharing the activations in one launch: each output equals
+    the oracle's product bit for bit, and the separate bitnet_linear call."""
+    rng = np.random.default_rng(M * 7 + K + len(Ns))
+    lo, hi = (-128, 128) if act_bits == 8 else (-8, 8)
+    qx = rng.integers(lo, hi, size=(M, K)).astype(np.int8)
+    s_x = rng.uniform(0.5, 200, size=M).astype(np.float32)
+    xq = dev(qx) if act_bits == 8 else dev(O.pack_int4(qx))
+    mats, ws = [], []
+    for N in Ns:
+        qw = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+        s_w = np.float32(rng.uniform(5, 60))
+        mats.append((qw, s_w))
+        ws.append((dev(O.pack_ternary(qw)), dev(np.array([s_w], np.float32))))
+    od = torch.float32 if out == "f32" else torch.bfloat16
+    Ys = api.bitnet_linear_group(xq, act_bits, dev(s_x), ws, out_dtype=od)
+    torch.cuda.synchronize()
+    for (qw, s_w), Y, (pk, sw) in zip(mats, Ys, ws):
+        _, y_o = O.linear(qx, s_x, qw, s_w)
+        got = host(Y.float()) if out == "bf16" else host(Y)
+        if out == "f32":
+            assert np.array_equal(got.view(np.uint32), y_o.view(np.uint32))
+        else:
+            assert np.array_equal(host(Y.view(torch.int16)).view(np.uint16), O.bf16_round(y_o))
+        Y1, _ = api.bitnet_linear(xq, act_bits, dev(s_x), pk, sw, out_dtype=od)
+        assert torch.equal(Y1, Y)
+
+
 # ------------------------------------------------------- fused BitLinear ----
 
 def _check_bitlinear(M, N, K, dtype, use_gamma, out, path=0, seed=0):
