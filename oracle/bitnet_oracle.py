@@ -55,6 +55,10 @@ Readings where the pages are silent:
   byte = sum_i (w_{5g+i} + 1) * 3^i for i = 0..4 (3^5 = 243 <= 256), i.e. 1.6
   bits per weight.  Weights past K count as 0; each row is padded to a
   multiple of 16 bytes with bytes of five zero weights (121).
+* Attention core of the stacked layer (P2 names rotary position embedding;
+  the pages give no formula): plain float64 definitions.  RoPE turns the pair
+  (x[2i], x[2i+1]) of each head by p * 10000^(-2i/d); attention is per-head
+  softmax(q k^T / sqrt(d)) v over the keys at positions up to the query's.
 """
 from __future__ import annotations
 
@@ -391,3 +395,75 @@ def chain_layer(x: np.ndarray, layer: dict, eps: float = DEFAULT_EPS) -> np.ndar
     _, sd, cd, _ = hadamard_quant_act(a, None, eps)
     _, d = linear(cd, sd, *layer["down"])
     return h + d
+
+
+# ---------------------------------------------------------------------------
+# attention core of the stacked layer [P2 주요 아키텍처 혁신: rotary position
+# embedding; the BitLinear layers are the linear layers of a transformer's
+# attention and FFN blocks, P4 BitNet 아키텍처]
+#
+# Plain float64 definitions (the pages fix no precision for this part):
+#   RoPE: in each head of width d, the pair (x[2i], x[2i+1]) of a token at
+#   position p turns by the angle p * theta_i, theta_i = 10000^(-2i/d) (the
+#   rotary embedding's own pairing and base; the pages name the method only);
+#   attention: per head, softmax(q k^T / sqrt(d)) v over the keys a query may
+#   see (its own position and the earlier ones).
+# ---------------------------------------------------------------------------
+
+ROPE_BASE = 10000.0
+
+
+def rope_inv_freq(head_dim: int, base: float = ROPE_BASE) -> np.ndarray:
+    """theta_i = base^(-2i/d) for i < d/2, float64."""
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    return base ** (-2.0 * i / head_dim)
+
+
+def rope_f64(x: np.ndarray, positions, heads: int, base: float = ROPE_BASE) -> np.ndarray:
+    """Rotary position embedding of rows x [M, heads*d] at `positions` [M], float64:
+    (a, b) = (x[2i], x[2i+1]) -> (a cos t - b sin t, a sin t + b cos t), t = p * theta_i."""
+    x = np.asarray(x, dtype=np.float64)
+    M, HD = x.shape
+    d = HD // heads
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * rope_inv_freq(d, base)[None, :]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    v = x.reshape(M, heads, d // 2, 2)
+    a, b = v[..., 0], v[..., 1]
+    out = np.empty_like(v)
+    out[..., 0] = a * c - b * s
+    out[..., 1] = a * s + b * c
+    return out.reshape(M, HD)
+
+
+def attention_weights_f64(q: np.ndarray, k: np.ndarray, visible: np.ndarray) -> np.ndarray:
+    """Softmax weights of one head: p[i, j] = exp(s_ij - max_j s_ij) / sum_j(...) over
+    the visible keys, s_ij = (q_i . k_j) / sqrt(d); invisible keys get weight 0."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    d = q.shape[-1]
+    s = (q @ k.T) / math.sqrt(d)
+    s = np.where(visible, s, -np.inf)
+    m = np.max(s, axis=-1, keepdims=True)
+    e = np.where(visible, np.exp(s - m), 0.0)
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+def attention_f64(q: np.ndarray, k: np.ndarray, v: np.ndarray, heads: int, visible: np.ndarray) -> np.ndarray:
+    """Multi-head softmax attention, float64.  q [Mq, heads*d], k and v [Mk, heads*d],
+    visible [Mq, Mk] boolean.  Returns [Mq, heads*d]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    d = q.shape[-1] // heads
+    out = np.empty((q.shape[0], heads * d), dtype=np.float64)
+    for h in range(heads):
+        sl = slice(h * d, (h + 1) * d)
+        out[:, sl] = attention_weights_f64(q[:, sl], k[:, sl], visible) @ v[:, sl]
+    return out
+
+
+def causal_mask(n_query: int, n_key: int, first_query_pos: int) -> np.ndarray:
+    """Query r sits at position first_query_pos + r and sees keys 0 .. its own position."""
+    qpos = first_query_pos + np.arange(n_query)[:, None]
+    return np.arange(n_key)[None, :] <= qpos

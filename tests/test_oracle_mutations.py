@@ -4,6 +4,8 @@ Each mutation swaps one oracle function for a wrong variant — a dropped term,
 a wrong sign, index or constant, a transposed operand — and at least one
 check of tests/test_oracle_pins.py must then fail.
 """
+import math
+
 import numpy as np
 import pytest
 
@@ -181,6 +183,50 @@ def _bf16_ties_away(y):
     return ((u + 0x8000) >> 16).astype(np.uint16)
 
 
+def _rope_half_pairs(x, positions, heads, base=O.ROPE_BASE):
+    """Pairs (i, i + d/2) instead of (2i, 2i + 1)."""
+    x = np.asarray(x, np.float64)
+    M, HD = x.shape
+    d = HD // heads
+    perm = np.concatenate([np.arange(0, d, 2), np.arange(1, d, 2)])
+    inv = np.argsort(perm)
+    xs = x.reshape(M, heads, d)[:, :, inv].reshape(M, HD)
+    y = _orig["rope_f64"](xs, positions, heads, base)
+    return y.reshape(M, heads, d)[:, :, perm].reshape(M, HD)
+
+
+def _rope_turns_backwards(x, positions, heads, base=O.ROPE_BASE):
+    return _orig["rope_f64"](x, -np.asarray(positions), heads, base)
+
+
+def _rope_base_1e4_per_pair(head_dim, base=O.ROPE_BASE):
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    return base ** (-i / head_dim)
+
+
+def _attn_no_scale(q, k, visible):
+    d = np.asarray(q).shape[-1]
+    return _orig["attention_weights_f64"](np.asarray(q, np.float64) * math.sqrt(d), k, visible)
+
+
+def _attn_scale_1_over_d(q, k, visible):
+    d = np.asarray(q).shape[-1]
+    return _orig["attention_weights_f64"](np.asarray(q, np.float64) / math.sqrt(d), k, visible)
+
+
+def _attn_sees_future(q, k, visible):
+    return _orig["attention_weights_f64"](q, k, np.ones_like(visible))
+
+
+def _attn_normalises_keys(q, k, visible):
+    """Softmax taken over the queries instead of the keys."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    s = np.where(visible, (q @ k.T) / math.sqrt(q.shape[-1]), -np.inf)
+    e = np.where(visible, np.exp(s - np.max(s, axis=0, keepdims=True)), 0.0)
+    return e / np.sum(e, axis=0, keepdims=True)
+
+
 MUTATIONS = {
     "absmax_numerator_128": ("absmax_quantize", _absmax_128),
     "absmax_truncates": ("absmax_quantize", _absmax_no_rint),
@@ -207,6 +253,13 @@ MUTATIONS = {
     "chain_drops_residual": ("chain_layer", _chain_no_attention_residual),
     "bf16_truncates": ("bf16_round", _bf16_truncate),
     "bf16_ties_away": ("bf16_round", _bf16_ties_away),
+    "rope_half_pairs": ("rope_f64", _rope_half_pairs),
+    "rope_backwards": ("rope_f64", _rope_turns_backwards),
+    "rope_wrong_frequencies": ("rope_inv_freq", _rope_base_1e4_per_pair),
+    "attention_unscaled": ("attention_weights_f64", _attn_no_scale),
+    "attention_scale_1_over_d": ("attention_weights_f64", _attn_scale_1_over_d),
+    "attention_sees_future": ("attention_weights_f64", _attn_sees_future),
+    "attention_softmax_over_queries": ("attention_weights_f64", _attn_normalises_keys),
 }
 
 

@@ -375,6 +375,84 @@ def check_chain_layer_tiny_golden():
     assert np.max(np.abs(got[0] - want) / np.abs(want)) < 1e-5, (got, want)
 
 
+# -------------------------------------------------------------- attention ----
+
+def check_rope_golden():
+    for row in _golden("rope_worked_example.txt"):
+        lhs, rhs = row.split(";")
+        *x, pos = lhs.split()
+        want = np.array([float(v) for v in rhs.split()])
+        got = O.rope_f64(np.array([[float(v) for v in x]]), [int(pos)], heads=1)
+        assert np.max(np.abs(got[0] - want)) < 1e-12, (got, want)
+
+
+def check_rope_is_a_rotation():
+    """Each pair keeps its length; two rotated vectors' dot product depends only on
+    the distance of their positions; position 0 is the identity (any head count)."""
+    rng = np.random.default_rng(31)
+    q = rng.standard_normal((1, 4 * 128))
+    k = rng.standard_normal((1, 4 * 128))
+    rq = O.rope_f64(q, [37], heads=4)
+    pair = lambda a: np.sqrt((a.reshape(-1, 2) ** 2).sum(axis=1))
+    assert np.allclose(pair(rq), pair(q), rtol=1e-13)
+    dots = [float(O.rope_f64(q, [p + t], 4)[0] @ O.rope_f64(k, [s + t], 4)[0]) for p, s, t in
+            ((9, 4, 0), (9, 4, 100), (105, 100, 0))]
+    assert abs(dots[0] - dots[1]) < 1e-9 and abs(dots[0] - dots[2]) < 1e-9
+    assert np.array_equal(O.rope_f64(q, [0], 4), q)
+
+
+def check_attention_closed_form():
+    """Two keys whose scaled scores are ln 3 and 0: weights 3/4 and 1/4 exactly
+    (the scale is 1/sqrt(d), d = 4)."""
+    a = 2.0 * math.log(3.0)               # q . k1 = 2 ln 3, divided by sqrt(4) = ln 3
+    q = np.array([[1.0, 0, 0, 0]])
+    k = np.array([[a, 0, 0, 0], [0, 0, 0, 0]])
+    v = np.array([[4.0, 0, 0, 8], [0, 4, 0, -8]])
+    out = O.attention_f64(q, k, v, heads=1, visible=np.ones((1, 2), bool))
+    assert np.max(np.abs(out - np.array([[3.0, 1.0, 0.0, 4.0]]))) < 1e-12, out
+
+
+def check_attention_brute_force():
+    """Two heads, three queries, causal: explicit loops with math.exp."""
+    rng = np.random.default_rng(32)
+    H, d, n = 2, 8, 3
+    q, k, v = (rng.standard_normal((n, H * d)) for _ in range(3))
+    mask = O.causal_mask(n, n, 0)
+    got = O.attention_f64(q, k, v, H, mask)
+    for h in range(H):
+        sl = slice(h * d, (h + 1) * d)
+        for i in range(n):
+            sc = [sum(q[i, sl][t] * k[j, sl][t] for t in range(d)) / math.sqrt(d) for j in range(i + 1)]
+            mx = max(sc)
+            w = [math.exp(x - mx) for x in sc]
+            tot = sum(w)
+            ref = [sum(w[j] * v[j, sl][t] for j in range(i + 1)) / tot for t in range(d)]
+            assert np.max(np.abs(got[i, sl] - np.array(ref))) < 1e-12
+
+
+def check_attention_special_cases():
+    rng = np.random.default_rng(33)
+    q, k, v = (rng.standard_normal((5, 64)) for _ in range(3))
+    # one visible key: the output is that key's value (the one-token context)
+    one = O.attention_f64(q[:1], k[:1], v[:1], 2, np.ones((1, 1), bool))
+    assert np.allclose(one, v[:1], rtol=0, atol=1e-15)
+    # a zero query scores every key alike: the mean of the visible values
+    z = O.attention_f64(np.zeros((1, 64)), k, v, 2, np.ones((1, 5), bool))
+    assert np.allclose(z[0], v.mean(axis=0), atol=1e-14)
+    # softmax weights are non-negative and sum to one over the visible keys
+    w = O.attention_weights_f64(q[:, :32], k[:, :32], O.causal_mask(5, 5, 0))
+    assert np.all(w >= 0) and np.allclose(w.sum(axis=1), 1.0, atol=1e-14)
+    assert np.all(w[np.triu_indices(5, 1)] == 0)
+    # causality: a later key or value cannot change an earlier output
+    k2, v2 = k.copy(), v.copy()
+    k2[4] += 3.0
+    v2[4] -= 2.0
+    m = O.causal_mask(5, 5, 0)
+    assert np.array_equal(O.attention_f64(q, k, v, 2, m)[:4], O.attention_f64(q, k2, v2, 2, m)[:4])
+    # a query at position 2 of a cached context sees keys 0..2
+    assert np.array_equal(O.causal_mask(1, 5, 2)[0], [True, True, True, False, False])
+
+
 CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]
 
 
