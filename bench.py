@@ -72,9 +72,13 @@ WORKLOADS = {
     "prefill": lambda: wl.prefill(with_weights=False),
     "hbitlinear": lambda: wl.hbitlinear(with_weights=False),
 }
-CHAIN_WORKLOADS = {"chain_decode": 32, "chain_prefill": 512}    # tokens per step
+CHAIN_WORKLOADS = {"chain_decode": 32, "chain_prefill": 512,          # tokens per step
+                   "chain_decode_attn": 32, "chain_prefill_attn": 512}
+# with the attention core: (sequences, tokens per sequence, first position, cache rows)
+CHAIN_ATTENTION = {"chain_prefill_attn": (1, 512, 0, 512), "chain_decode_attn": (32, 1, 512, 513)}
 CHAIN_LAYERS = 24
-ORDER = ["tiny", "decode_m1", "decode_m4", "decode_m16", "prefill", "hbitlinear", "chain_decode", "chain_prefill"]
+ORDER = ["tiny", "decode_m1", "decode_m4", "decode_m16", "prefill", "hbitlinear", "chain_decode", "chain_decode_attn",
+         "chain_prefill_attn", "chain_prefill"]
 HEADLINE = "chain_prefill"
 
 
@@ -495,12 +499,27 @@ def run_chain(name, args, ctx):
             del w
         torch.cuda.synchronize()
         ctx["chain_layers"] = layers
-    ch = chain.BitLinearChain(layers, M, H, F, dev)
+    att = CHAIN_ATTENTION.get(name)
+    t0 = 0
+    if att is None:
+        ch = chain.BitLinearChain(layers, M, H, F, dev)
+    else:
+        B, L, t0, T_cap = att
+        ch = chain.BitLinearChain(layers, M, H, F, dev, attention=dict(B=B, L=L, T_cap=T_cap, heads=wl.CHAIN_HEADS))
+        if t0 > 0:
+            # the decode step continues B sequences whose first t0 tokens went through a prefill
+            pre = chain.BitLinearChain(layers, B * t0, H, F, dev,
+                                       attention=dict(B=B, L=t0, T_cap=T_cap, heads=wl.CHAIN_HEADS))
+            pre.kc, pre.vc = ch.kc, ch.vc
+            pre.forward(torch.from_numpy(wl.chain_input(B * t0, seed=9)).to(dev), stream, t0=0)
+            torch.cuda.synchronize()
+            del pre
+            torch.cuda.empty_cache()
     x = torch.from_numpy(wl.chain_input(M)).to(dev)
 
     warmup = max(3, args.warmup)
     for _ in range(warmup):
-        ch.forward(x, stream)
+        ch.forward(x, stream, t0=t0)
     torch.cuda.synchronize()
 
     def lin_only(i):                       # the chain's linear launches alone, same operands
@@ -510,8 +529,15 @@ def run_chain(name, args, ctx):
             api.bitnet_linear_group(ch.hq, 8, ch.sh, [w["up"], w["gate"]], Ys=[ch.up, ch.gate], stream=stream)
             api.bitnet_linear(ch.a4, 4, ch.sa, *w["down"], Y=ch.d, stream=stream)
 
-    t_step = timer.time(timer.graph(lambda i: ch.forward(x, stream)))
+    t_step = timer.time(timer.graph(lambda i: ch.forward(x, stream, t0=t0)))
     t_lin = timer.time(timer.graph(lin_only))
+    t_att = None
+    if att is not None:
+        def att_only(i):                   # rotary embedding, cache append and attention of every layer
+            for li in range(CHAIN_LAYERS):
+                api.bitnet_rope_append(ch.q, ch.k, ch.v, ch.kc[li], ch.vc[li], B, L, t0, ch.heads, stream=stream)
+                api.bitnet_attention(ch.q, ch.kc[li], ch.vc[li], B, L, t0, ch.heads, A=ch.att, stream=stream)
+        t_att = timer.time(timer.graph(att_only))
 
     # e2e: host input in, host output back, through the Python API
     x_pin = torch.empty((M, H), dtype=torch.float32).pin_memory()
@@ -520,7 +546,7 @@ def run_chain(name, args, ctx):
 
     def e2e_step(i):
         x.copy_(x_pin, non_blocking=True)
-        y_pin.copy_(ch.forward(x, stream), non_blocking=True)
+        y_pin.copy_(ch.forward(x, stream, t0=t0), non_blocking=True)
 
     for i in range(warmup):
         e2e_step(i)
@@ -546,8 +572,23 @@ def run_chain(name, args, ctx):
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     # whole-step view: the slower of the weight stream and the integer work, against the step time
     ideal = max((packed + act_bytes) / (peaks["hbm_gbs"] * 1e9), ops / (int8_peak(peaks) * 1e12))
+    extra = {}
+    if att is not None:
+        att_s = t_att["ms"] / 1e3
+        n_ctx = t0 + L
+        # per layer: the caches' keys and values each sequence's queries read (fp32), and the
+        # score and weighted-sum multiply-adds (causal: a query at position p reads p + 1 keys)
+        pairs = B * sum(t0 + l + 1 for l in range(L))
+        kv_bytes = CHAIN_LAYERS * B * n_ctx * H * 4 * 2
+        flops = CHAIN_LAYERS * 2 * 2 * pairs * H
+        extra["attention"] = {
+            "us_per_step": att_s * 1e6, "sequences": B, "tokens_per_sequence": L, "first_position": t0,
+            "cache_bytes_read_per_step": kv_bytes, "fp32_flops_per_step": flops,
+            "achieved_GBs": kv_bytes / att_s / 1e9, "achieved_TFLOPs": flops / att_s / 1e12,
+            "note": "rotary embedding + cache append + causal softmax attention of all 24 layers (fp32 CUDA cores)"}
     return {
-        "workload": f"bitlinear_chain_{CHAIN_LAYERS}layers_m{M}_hidden{H}_ffn{F}", "M_tokens": M,
+        "workload": (f"bitlinear_chain_{CHAIN_LAYERS}layers_m{M}_hidden{H}_ffn{F}" +
+                     ("" if att is None else f"_attention_{B}seq_ctx{t0 + L}")), "M_tokens": M,
         "layers": CHAIN_LAYERS, "hidden": H, "ffn": F,
         "l2": f"{packed / 1e6:.0f} MB of packed weights per step (> 2x L2)",
         "value": M * world / step_s, "unit": "tokens/s", "ms_per_step": t_step["ms"],
@@ -559,7 +600,8 @@ def run_chain(name, args, ctx):
         "e2e": {"value": M * world / t_e2e, "unit": "tokens/s",
                 "h2d_bytes_per_step": M * H * 4, "d2h_bytes_per_step": M * H * 4},
         "gpu_launches_per_step": ch.launches,
-        "clocks": ctx["clocks"].summary(t_step["window"][0], t_lin["window"][1]),
+        "clocks": ctx["clocks"].summary(t_step["window"][0], (t_att or t_lin)["window"][1]),
+        **extra,
     }
 
 
@@ -666,19 +708,28 @@ class ChainOracle:
                 lw[pn] = (q, s_w)
             self.layers.append(lw)
 
-    def step(self, x):
+    def step(self, x, context: int = 0):
+        """x [1, hidden] through all layers; with context > 0 the token sits at position
+        context - 1 and attends over a cache of that many keys (seeded values)."""
         y = x
         for l in range(CHAIN_LAYERS):
-            y = self.O.chain_layer(y, self.layers[l % 2])
+            if context:
+                rng = np.random.default_rng(l)
+                kc = rng.standard_normal((1, context, wl.CHAIN_HIDDEN)) * 0.6
+                vc = rng.standard_normal((1, context, wl.CHAIN_HIDDEN)) * 0.6
+                y = self.O.chain_layer_attention(y, self.layers[l % 2], kc, vc, context - 1, wl.CHAIN_HEADS)
+            else:
+                y = self.O.chain_layer(y, self.layers[l % 2])
         return len(x)
 
 
-def chain_cpu_baseline(budget_s=4.0, oracle=None):
+def chain_cpu_baseline(budget_s=4.0, oracle=None, context: int = 0):
     o = oracle or ChainOracle()
     x = wl.chain_input(1)
-    tokens, n, dt = _timed_loop(lambda: o.step(x), budget_s)
+    tokens, n, dt = _timed_loop(lambda: o.step(x, context), budget_s)
+    what = f"at position {context - 1} over a {context}-key cache " if context else ""
     return {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} passes of 1 token through all {CHAIN_LAYERS} layers of the numpy oracle "
+            "sample": f"{n} passes of 1 token {what}through all {CHAIN_LAYERS} layers of the numpy oracle "
                       f"(numpy, single thread)"}
 
 
@@ -731,7 +782,9 @@ def add_cpu_baselines(subs):
     for name, sub in subs.items():
         if name in CHAIN_WORKLOADS:
             chain_oracle = chain_oracle or ChainOracle()
-            sub["cpu_baseline"] = chain_cpu_baseline(oracle=chain_oracle)
+            att = CHAIN_ATTENTION.get(name)
+            sub["cpu_baseline"] = chain_cpu_baseline(oracle=chain_oracle,
+                                                     context=0 if att is None else att[2] + att[1])
             continue
         c = WORKLOADS[name]()
         sub["cpu_baseline"] = cpu_baseline(c)

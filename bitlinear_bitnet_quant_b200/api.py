@@ -61,6 +61,10 @@ _SIGNATURES = {
                                            ctypes.POINTER(_c_void_p), ctypes.POINTER(_c_void_p),
                                            ctypes.POINTER(_i64), ctypes.POINTER(_c_void_p), ctypes.c_int,
                                            _c_void_p]),
+    "bitnet_rope_append": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_double, _c_void_p, _c_void_p, _i64, _c_void_p]),
+    "bitnet_attention": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64, ctypes.c_int,
+                                        ctypes.c_int, _i64, _c_void_p, _c_void_p]),
     "bitnet_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
 }
 
@@ -317,6 +321,30 @@ def bitnet_relu2_glu(gate: torch.Tensor, up: torch.Tensor, out=None, stream=None
     _check("bitnet_relu2_glu", lib().bitnet_relu2_glu(_ptr(gate), _ptr(up), _ptr(out), gate.numel(),
                                                       _stream(stream)))
     return out
+
+
+def bitnet_rope_append(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, Kc: torch.Tensor, Vc: torch.Tensor,
+                       B: int, L: int, t0: int, heads: int, base: float = 10000.0, stream=None):
+    """Rotary embedding of Q (in place) and K; rotated K and V rows written into
+    the caches Kc, Vc [B, T_cap, heads*d] at positions t0 .. t0+L-1."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (Kc, "Kc"), (Vc, "Vc")):
+        _require(t, n)
+    d = Q.shape[1] // heads
+    _check("bitnet_rope_append", lib().bitnet_rope_append(
+        _ptr(Q), _ptr(K), _ptr(V), B, L, t0, heads, d, float(base), _ptr(Kc), _ptr(Vc), Kc.shape[1],
+        _stream(stream)))
+
+
+def bitnet_attention(Q: torch.Tensor, Kc: torch.Tensor, Vc: torch.Tensor, B: int, L: int, t0: int, heads: int,
+                     A=None, stream=None):
+    """Causal softmax attention of the rows Q [B*L, heads*d] over the caches.  Returns A."""
+    for t, n in ((Q, "Q"), (Kc, "Kc"), (Vc, "Vc")):
+        _require(t, n)
+    A = torch.empty_like(Q) if A is None else A
+    d = Q.shape[1] // heads
+    _check("bitnet_attention", lib().bitnet_attention(
+        _ptr(Q), _ptr(Kc), _ptr(Vc), B, L, t0, heads, d, Kc.shape[1], _ptr(A), _stream(stream)))
+    return A
 
 
 def bitnet_device_error() -> int:

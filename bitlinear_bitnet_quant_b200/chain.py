@@ -7,8 +7,10 @@ Per layer, with fp32 residuals:
 
     q, k, v = BitLinear(x)                      (one int8 quantisation of x,
                                                  one launch for the three)
-    o = H-BitLinear(v)                          (attention over a one-token
-                                                 context returns V)
+    o = H-BitLinear(attention(q, k, v))         (rotary embedding, key/value
+                                                 cache, causal softmax; without
+                                                 a cache, a one-token context,
+                                                 which returns V)
     h = x + o
     up, gate = BitLinear(h)                     (one int8 quantisation of h,
                                                  one launch for the two)
@@ -37,11 +39,28 @@ def quantize_layer(weights: dict, stream=None) -> dict:
 
 
 class BitLinearChain:
-    """Runs a list of quantised layers on a batch of M tokens of width `hidden`."""
+    """Runs a list of quantised layers on a batch of M tokens of width `hidden`.
 
-    def __init__(self, layers: list, M: int, hidden: int, ffn: int, device, eps: float = 1e-6):
+    attention=None: the attention core over a one-token context (O's input is V).
+    attention=dict(B=..., L=..., T_cap=..., heads=...): the M = B*L rows are B
+    sequences of L tokens each; every layer keeps a key/value cache
+    [B, T_cap, hidden] (allocated here) and runs rotary embedding, the cache
+    append and causal softmax attention; forward(x, t0) places the step's
+    tokens at positions t0 .. t0+L-1."""
+
+    def __init__(self, layers: list, M: int, hidden: int, ffn: int, device, eps: float = 1e-6, attention=None):
         self.layers = layers
         self.M, self.hidden, self.ffn, self.eps = M, hidden, ffn, eps
+        self.attention = attention
+        if attention is not None:
+            B, L, T_cap = attention["B"], attention["L"], attention["T_cap"]
+            assert B * L == M and L <= T_cap
+            self.heads = attention.get("heads", 16)
+            self.rope_base = attention.get("base", 10000.0)
+            self.kc = [torch.empty((B, T_cap, hidden), dtype=torch.float32, device=device) for _ in layers]
+            self.vc = [torch.empty((B, T_cap, hidden), dtype=torch.float32, device=device) for _ in layers]
+            self.att = torch.empty((M, hidden), dtype=torch.float32, device=device)
+        self.t0 = 0
         f32 = dict(dtype=torch.float32, device=device)
         e = lambda *shape: torch.empty(shape, **f32)
         self.x = [e(M, hidden), e(M, hidden)]          # layer input, chain output
@@ -56,7 +75,7 @@ class BitLinearChain:
         self.a4 = torch.empty((M, ffn // 2), dtype=torch.uint8, device=device)
         self.sa = e(M)
 
-    def layer(self, x_parts, w: dict, stream=None):
+    def layer(self, x_parts, w: dict, stream=None, index: int = 0):
         """One layer.  x_parts: (x,) or (h_prev, d_prev), whose sum is the
         layer input.  Returns (h, d), whose sum is the layer output.  Buffers
         are reused from layer to layer: every kernel waits for the one before
@@ -69,7 +88,15 @@ class BitLinearChain:
             x = self.x[0]
             A.bitnet_add_quant_act(x_parts[0], x_parts[1], None, self.eps, H=x, Xq=self.xq, s_x=self.sx, stream=s)
         A.bitnet_linear_group(self.xq, 8, self.sx, [w["q"], w["k"], w["v"]], Ys=[self.q, self.k, self.v], stream=s)
-        A.bitnet_hadamard_quant_act(self.v, None, self.eps, 0, Xq4=self.v4, s_x=self.sv, stream=s)
+        if self.attention is None:
+            att = self.v                                   # a one-token context returns V
+        else:
+            B, L = self.attention["B"], self.attention["L"]
+            A.bitnet_rope_append(self.q, self.k, self.v, self.kc[index], self.vc[index], B, L, self.t0, self.heads,
+                                 self.rope_base, stream=s)
+            att = A.bitnet_attention(self.q, self.kc[index], self.vc[index], B, L, self.t0, self.heads, A=self.att,
+                                     stream=s)
+        A.bitnet_hadamard_quant_act(att, None, self.eps, 0, Xq4=self.v4, s_x=self.sv, stream=s)
         A.bitnet_linear(self.v4, 4, self.sv, *w["o"], Y=self.o, stream=s)
         A.bitnet_add_quant_act(x, self.o, None, self.eps, H=self.h, Xq=self.hq, s_x=self.sh, stream=s)
         A.bitnet_linear_group(self.hq, 8, self.sh, [w["up"], w["gate"]], Ys=[self.up, self.gate], stream=s)
@@ -77,12 +104,14 @@ class BitLinearChain:
         A.bitnet_linear(self.a4, 4, self.sa, *w["down"], Y=self.d, stream=s)
         return self.h, self.d
 
-    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, stream=None, t0: int = 0) -> torch.Tensor:
         """x: [M, hidden] fp32 on the device; returns the last layer's output
-        (one of the chain's own buffers)."""
+        (one of the chain's own buffers).  t0: position of each sequence's first
+        token in this step (with attention)."""
+        self.t0 = t0
         parts = (x,)
-        for w in self.layers:
-            parts = self.layer(parts, w, stream)
+        for i, w in enumerate(self.layers):
+            parts = self.layer(parts, w, stream, i)
         api.bitnet_add(parts[0], parts[1], out=self.x[1], stream=stream)
         return self.x[1]
 
@@ -93,7 +122,7 @@ class BitLinearChain:
     # the last layer
     @property
     def launches(self) -> int:
-        return 8 * len(self.layers) + 1
+        return (8 if self.attention is None else 10) * len(self.layers) + 1
 
     def packed_bytes(self) -> int:
         return sum(pk.numel() for w in self.layers for pk, _ in w.values())

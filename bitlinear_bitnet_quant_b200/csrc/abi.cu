@@ -39,6 +39,10 @@ cudaError_t run_linear_decode_trit5(const void* Xq, int act_bits, const float* s
                                     const float* s_w, int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg,
                                     cudaStream_t st);
 cudaError_t run_relu2_glu(const float* gate, const float* up, float* out, size_t n, cudaStream_t st);
+cudaError_t run_rope_append(float* Q, const float* K, const float* V, int B, int L, int t0, int heads, int d,
+                            double base, float* Kc, float* Vc, int T_cap, cudaStream_t st);
+cudaError_t run_attention(const float* Q, const float* Kc, const float* Vc, int B, int L, int t0, int heads, int d,
+                          int T_cap, float* A, cudaStream_t st);
 }  // namespace bitnet
 
 namespace {
@@ -338,6 +342,42 @@ int bitnet_relu2_glu(const float* gate, const float* up, float* out, int64_t n, 
   const int c = elementwise_check(gate, up, out, n);
   if (c != BITNET_OK) return c < 0 ? BITNET_OK : c;
   return cuda_status(bitnet::run_relu2_glu(gate, up, out, (size_t)n, static_cast<cudaStream_t>(stream)));
+}
+
+static int attention_shape(int64_t B, int64_t L, int64_t t0, int heads, int head_dim, int64_t T_cap) {
+  if (head_dim != 128 || heads < 1 || heads > 256) return BITNET_ERR_SHAPE;
+  if (B < 0 || L < 0 || t0 < 0 || T_cap < 1 || T_cap > (int64_t(1) << 24) || t0 + L > T_cap) return BITNET_ERR_SHAPE;
+  if (B * T_cap * heads * head_dim >= (int64_t(1) << 40) || B * L >= (int64_t(1) << 30) || B > 65535)
+    return BITNET_ERR_SHAPE;
+  return BITNET_OK;
+}
+
+int bitnet_rope_append(float* Q, const float* K, const float* V, int64_t B, int64_t L, int64_t t0, int heads,
+                       int head_dim, double base, float* Kc, float* Vc, int64_t T_cap, void* stream) {
+  const int sh = attention_shape(B, L, t0, heads, head_dim, T_cap);
+  if (sh != BITNET_OK) return sh;
+  if (!(base > 1.0) || !(base < 1e300)) return BITNET_ERR_SHAPE;
+  if (B == 0 || L == 0) return BITNET_OK;
+  if (!Q || !K || !V || !Kc || !Vc) return BITNET_ERR_NULL;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(Kc) || !aligned16(Vc)) return BITNET_ERR_ALIGN;
+  int d = check_device();
+  if (d != BITNET_OK) return d;
+  return cuda_status(bitnet::run_rope_append(Q, K, V, (int)B, (int)L, (int)t0, heads, head_dim, base, Kc, Vc,
+                                             (int)T_cap, static_cast<cudaStream_t>(stream)));
+}
+
+int bitnet_attention(const float* Q, const float* Kc, const float* Vc, int64_t B, int64_t L, int64_t t0, int heads,
+                     int head_dim, int64_t T_cap, float* A, void* stream) {
+  const int sh = attention_shape(B, L, t0, heads, head_dim, T_cap);
+  if (sh != BITNET_OK) return sh;
+  if (heads > 65535) return BITNET_ERR_SHAPE;
+  if (B == 0 || L == 0) return BITNET_OK;
+  if (!Q || !Kc || !Vc || !A) return BITNET_ERR_NULL;
+  if (!aligned16(Q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(A)) return BITNET_ERR_ALIGN;
+  int d = check_device();
+  if (d != BITNET_OK) return d;
+  return cuda_status(bitnet::run_attention(Q, Kc, Vc, (int)B, (int)L, (int)t0, heads, head_dim, (int)T_cap, A,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 int bitnet_device_error(int* code_out) {

@@ -126,6 +126,7 @@ def hbitlinear(seed: int = 0, M: int = 2048, with_weights: bool = True) -> dict:
 # Layer shapes of the stacked BitLinear chain (hidden 2048, FFN 5632).
 CHAIN_HIDDEN = 2048
 CHAIN_FFN = 5632
+CHAIN_HEADS = 16
 CHAIN_PROJ = (  # name, N (out), K (in), activation bits of its input
     ("q", 2048, 2048, 8), ("k", 2048, 2048, 8), ("v", 2048, 2048, 8),
     ("o", 2048, 2048, 4), ("up", 5632, 2048, 8), ("gate", 5632, 2048, 8),

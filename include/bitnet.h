@@ -295,6 +295,32 @@ BITNET_API int bitnet_bitlinear_kernel(const void* X, int x_dtype, int64_t M, in
                                        int y_dtype, int8_t* Xq, float* s_x, int kernel, void* stream);
 
 /*
+ * Attention core of a stacked layer: rotary position embedding, a key/value
+ * cache, and causal softmax attention ("AI 혁신의 선두: 마이크로소프트의 1비트 LLM,
+ * BitNet b1.58 2B4T", 주요 아키텍처 혁신: rotary position embedding; the Q/K/V/O
+ * projections around it are BitLinear).  The pages give no formula; the
+ * definitions are the methods' own:
+ *   RoPE: in each head of width d, the pair (x[2i], x[2i+1]) of a token at
+ *         position p turns by the angle p * theta_i, theta_i = base^(-2i/d)
+ *         (computed in fp64, rounded once to fp32);
+ *   attention: per head, softmax(q k^T / sqrt(d)) v over the keys at
+ *         positions 0 .. the query's own (fp32 arithmetic).
+ * Layout: token rows [B*L][heads*d] fp32, where sequence b's L tokens sit at
+ * positions t0 .. t0+L-1; caches Kc, Vc [B][T_cap][heads*d] fp32 whose row t
+ * holds position t (rotated key; value).
+ * bitnet_rope_append: rotates Q in place; writes the rotated K rows and the V
+ *   rows into the caches at positions t0 .. t0+L-1.
+ * bitnet_attention: A [B*L][heads*d] = attention of every query row over its
+ *   sequence's cached keys 0 .. t0+l (the caches must hold them already).
+ * Limits: head_dim == 128; t0 + L <= T_cap; base > 1; B, L >= 0 (0 is a no-op).
+ */
+BITNET_API int bitnet_rope_append(float* Q, const float* K, const float* V, int64_t B, int64_t L, int64_t t0,
+                                  int heads, int head_dim, double base, float* Kc, float* Vc, int64_t T_cap,
+                                  void* stream);
+BITNET_API int bitnet_attention(const float* Q, const float* Kc, const float* Vc, int64_t B, int64_t L, int64_t t0,
+                                int heads, int head_dim, int64_t T_cap, float* A, void* stream);
+
+/*
  * Reads and clears the library's device-side error flag on the current
  * device (synchronises the device).  A kernel that waited more than ~2 s on
  * a pipeline barrier gives up, records a nonzero code here and returns; 0

@@ -467,3 +467,39 @@ def causal_mask(n_query: int, n_key: int, first_query_pos: int) -> np.ndarray:
     """Query r sits at position first_query_pos + r and sees keys 0 .. its own position."""
     qpos = first_query_pos + np.arange(n_query)[:, None]
     return np.arange(n_key)[None, :] <= qpos
+
+
+def chain_layer_attention(x: np.ndarray, layer: dict, k_cache: np.ndarray, v_cache: np.ndarray, t0: int,
+                          heads: int = 16, eps: float = DEFAULT_EPS) -> np.ndarray:
+    """One stacked layer with the attention core.  x [B*L, hidden] fp32 holds B
+    sequences of L tokens at positions t0 .. t0+L-1; k_cache, v_cache
+    [B, T_cap, hidden] float64 receive this step's rotated keys and values.
+    The attention output enters the O projection's quantiser as fp32.  With one
+    token per sequence at position 0 this is chain_layer (the one-token context)."""
+    x = np.asarray(x, dtype=np.float32)
+    B = k_cache.shape[0]
+    L = x.shape[0] // B
+    qx, sx = quant_act(x, None, eps)
+    _, q = linear(qx, sx, *layer["q"])
+    _, k = linear(qx, sx, *layer["k"])
+    _, v = linear(qx, sx, *layer["v"])
+    pos = np.tile(t0 + np.arange(L), B)
+    q_r = rope_f64(q, pos, heads)
+    k_r = rope_f64(k, pos, heads)
+    att = np.empty(q.shape, dtype=np.float64)
+    for b in range(B):
+        rows = slice(b * L, (b + 1) * L)
+        k_cache[b, t0:t0 + L] = k_r[rows]
+        v_cache[b, t0:t0 + L] = v[rows]
+        att[rows] = attention_f64(q_r[rows], k_cache[b, :t0 + L], v_cache[b, :t0 + L], heads,
+                                  causal_mask(L, t0 + L, t0))
+    _, so, co, _ = hadamard_quant_act(att.astype(np.float32), None, eps)
+    _, o = linear(co, so, *layer["o"])
+    h = x + o
+    qh, sh = quant_act(h, None, eps)
+    _, up = linear(qh, sh, *layer["up"])
+    _, gate = linear(qh, sh, *layer["gate"])
+    a = squared_relu_glu(gate, up)
+    _, sd, cd, _ = hadamard_quant_act(a, None, eps)
+    _, d = linear(cd, sd, *layer["down"])
+    return h + d

@@ -453,6 +453,26 @@ def check_attention_special_cases():
     assert np.array_equal(O.causal_mask(1, 5, 2)[0], [True, True, True, False, False])
 
 
+def check_layer_attention_reduces_to_one_token_context():
+    """A layer whose every sequence holds one token at position 0 attends over that
+    token alone, so it equals the one-token-context layer bit for bit; with more
+    tokens the attention changes the output."""
+    layer = _tiny_chain_layer()
+    x = np.random.default_rng(34).standard_normal((3, 16)).astype(np.float32)
+    kc, vc = np.zeros((3, 4, 16)), np.zeros((3, 4, 16))
+    got = O.chain_layer_attention(x, layer, kc, vc, 0, heads=1)
+    assert np.array_equal(got, O.chain_layer(x, layer))
+    rng = np.random.default_rng(35)
+    rand = {n: (rng.integers(-1, 2, size=w.shape).astype(np.int8), np.float32(rng.uniform(20, 60)))
+            for n, (w, _) in layer.items()}
+    kc, vc = np.zeros((3, 4, 16)), np.zeros((3, 4, 16))
+    assert np.array_equal(O.chain_layer_attention(x, rand, kc, vc, 0, heads=2), O.chain_layer(x, rand))
+    kc, vc = np.zeros((1, 4, 16)), np.zeros((1, 4, 16))
+    seq = O.chain_layer_attention(x, rand, kc, vc, 0, heads=2)       # one sequence of three tokens
+    ref = O.chain_layer(x, rand)
+    assert np.array_equal(seq[0], ref[0]) and not np.array_equal(seq[1:], ref[1:])
+
+
 CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]
 
 

@@ -565,3 +565,142 @@ def test_elementwise_glue():
     assert np.array_equal(s, a + b)
     g = host(api.bitnet_relu2_glu(dev(a), dev(b)))
     assert np.array_equal(g, O.squared_relu_glu(a, b))
+
+
+# -------------------------------------------------------------- attention -----
+#
+# Rotary embedding and softmax attention decide no integer code; they are
+# compared with the oracle's float64 definitions within the bound the fp32
+# arithmetic allows (u = 2^-24):
+#   rotation, computed in fp64 and rounded once: |error| <= u * |pair|;
+#   attention: each score q.k/sqrt(d) is a 128-term fp32 dot product, off by at
+#   most E_j = (128 + 3) u sqrt(1/d) sum_i |q_i k_ji| (accumulation, scaling and
+#   the rounding of the rotated inputs); the softmax weights then move by a
+#   relative 2E (E = max_j E_j), expf by 2 ulp and the running rescaling by
+#   about 2 u per key, so each output is within (2E + (8 + 2n) u) max_j |v_j|.
+
+U32 = 2.0 ** -24
+
+
+def _attention_tol(q, k, v, mask, heads):
+    """Per (query, head) bound of the fp32 attention against float64."""
+    d = q.shape[1] // heads
+    tol = np.zeros((q.shape[0], heads))
+    for h in range(heads):
+        sl = slice(h * d, (h + 1) * d)
+        mag = np.abs(q[:, sl]).astype(np.float64) @ np.abs(k[:, sl]).astype(np.float64).T / math.sqrt(d)
+        mag = np.where(mask, mag, 0.0)
+        E = 131 * U32 * mag.max(axis=1)
+        n = mask.sum(axis=1)
+        vmax = np.array([np.abs(v[mask[i]][:, sl]).max() for i in range(q.shape[0])])
+        tol[:, h] = (2 * E + (8 + 2 * n) * U32) * vmax * 1.05 + 1e-30
+    return tol
+
+
+def _check_attention(got, ref, tol, heads):
+    d = got.shape[1] // heads
+    err = np.abs(got.astype(np.float64) - ref).reshape(got.shape[0], heads, d).max(axis=2)
+    assert np.all(err <= tol), (err / tol).max()
+
+
+def _rand_rows(rng, n, HD, scale=0.6):
+    return (rng.standard_normal((n, HD)) * scale).astype(np.float32)
+
+
+@pytest.mark.parametrize("B,L,t0,heads", [(1, 64, 0, 16), (2, 40, 0, 16), (3, 20, 37, 2), (32, 1, 512, 16),
+                                          (4, 5, 100, 4), (2, 1, 0, 16)])
+def test_rope_append_and_attention(B, L, t0, heads):
+    """RoPE of Q and K, the cache append, and causal attention over the cache,
+    on the prefill kernel (16 or more queries per sequence) and the decode
+    kernel (fewer)."""
+    rng = np.random.default_rng(B * 1000 + L * 10 + t0)
+    HD = heads * 128
+    T_cap = t0 + L + 3
+    q, k, v = (_rand_rows(rng, B * L, HD) for _ in range(3))
+    # earlier positions of the caches: already rotated keys and values
+    kc0 = _rand_rows(rng, B * T_cap, HD).reshape(B, T_cap, HD)
+    vc0 = _rand_rows(rng, B * T_cap, HD).reshape(B, T_cap, HD)
+    Qd, Kd, Vd = dev(q), dev(k), dev(v)
+    Kc, Vc = dev(kc0), dev(vc0)
+    api.bitnet_rope_append(Qd, Kd, Vd, Kc, Vc, B, L, t0, heads)
+    A = api.bitnet_attention(Qd, Kc, Vc, B, L, t0, heads)
+    torch.cuda.synchronize()
+    qr, kcg, vcg, a = host(Qd), host(Kc), host(Vc), host(A)
+    pos = np.tile(t0 + np.arange(L), B)
+    q_ref = O.rope_f64(q, pos, heads)
+    k_ref = O.rope_f64(k, pos, heads)
+    pair = lambda x: np.repeat(np.sqrt((x.astype(np.float64).reshape(x.shape[0], -1, 2) ** 2).sum(-1)), 2, axis=1)
+    assert np.all(np.abs(qr - q_ref) <= U32 * pair(q) * 1.001 + 1e-38)
+    for b in range(B):
+        rows = slice(t0, t0 + L)
+        kg = kcg[b, rows]
+        assert np.all(np.abs(kg - k_ref[b * L:(b + 1) * L]) <= U32 * pair(k[b * L:(b + 1) * L]) * 1.001 + 1e-38)
+        assert np.array_equal(vcg[b, rows], v[b * L:(b + 1) * L])
+        # rows outside the step are untouched
+        assert np.array_equal(kcg[b, :t0], kc0[b, :t0]) and np.array_equal(kcg[b, t0 + L:], kc0[b, t0 + L:])
+        mask = O.causal_mask(L, t0 + L, t0)
+        ref = O.attention_f64(qr[b * L:(b + 1) * L], kcg[b, :t0 + L], vcg[b, :t0 + L], heads, mask)
+        tol = _attention_tol(qr[b * L:(b + 1) * L], kcg[b, :t0 + L], vcg[b, :t0 + L], mask, heads)
+        _check_attention(a[b * L:(b + 1) * L], ref, tol, heads)
+    if t0 == 0 and L == 1:
+        assert np.array_equal(a, v)                 # one visible key: its value, exactly
+
+
+def test_chain_with_attention_prefill_then_decode():
+    """Two full-width layers (hidden 2048, 16 heads, FFN 5632) with the attention
+    core: a 24-token prefill of 2 sequences, then one decode step.  Layer by
+    layer, the GPU's own layer input goes to the oracle: K and V bit-exact; the
+    rotation and attention within their fp32 bounds; and from the GPU's
+    attention output on, everything bit-exact (O, residual, up/gate, gated
+    unit, down)."""
+    from bitlinear_bitnet_quant_b200 import chain
+    gpu_w, ora_w = _chain_weights(2)
+    B, L, H, heads = 2, 24, wl.CHAIN_HIDDEN, 16
+    T_cap = L + 1
+    x_pre = wl.chain_input(B * L, seed=5)
+    x_dec = wl.chain_input(B, seed=6)
+    pre = chain.BitLinearChain(gpu_w, B * L, H, wl.CHAIN_FFN, torch.device("cuda"),
+                               attention=dict(B=B, L=L, T_cap=T_cap, heads=heads))
+    dec = chain.BitLinearChain(gpu_w, B, H, wl.CHAIN_FFN, torch.device("cuda"),
+                               attention=dict(B=B, L=1, T_cap=T_cap, heads=heads))
+    dec.kc, dec.vc = pre.kc, pre.vc                  # the decode step continues the prefill's caches
+    ora_k = [np.zeros((B, T_cap, H)) for _ in range(2)]
+    ora_v = [np.zeros((B, T_cap, H)) for _ in range(2)]
+    for ch, x0, t0, Ls in ((pre, x_pre, 0, L), (dec, x_dec, L, 1)):
+        ch.t0 = t0
+        parts = (dev(x0),)
+        x_in = x0
+        for li, (w, lw) in enumerate(zip(gpu_w, ora_w)):
+            h, d = ch.layer(parts, w, None, li)
+            torch.cuda.synchronize()
+            qx, sx = O.quant_act(x_in, None, 1e-6)
+            _, q = O.linear(qx, sx, *lw["q"])
+            _, k = O.linear(qx, sx, *lw["k"])
+            _, v = O.linear(qx, sx, *lw["v"])
+            assert np.array_equal(host(ch.k), k) and np.array_equal(host(ch.v), v)
+            pos = np.tile(t0 + np.arange(Ls), B)
+            q_r, k_r = O.rope_f64(q, pos, heads), O.rope_f64(k, pos, heads)
+            for b in range(B):
+                ora_k[li][b, t0:t0 + Ls] = k_r[b * Ls:(b + 1) * Ls]
+                ora_v[li][b, t0:t0 + Ls] = v[b * Ls:(b + 1) * Ls]
+            att_g = host(ch.att)
+            qg = host(ch.q)
+            kcg, vcg = host(ch.kc[li]), host(ch.vc[li])
+            for b in range(B):
+                sl = slice(b * Ls, (b + 1) * Ls)
+                mask = O.causal_mask(Ls, t0 + Ls, t0)
+                ref = O.attention_f64(q_r[sl], ora_k[li][b, :t0 + Ls], ora_v[li][b, :t0 + Ls], heads, mask)
+                tol = _attention_tol(qg[sl], kcg[b, :t0 + Ls], vcg[b, :t0 + Ls], mask, heads)
+                _check_attention(att_g[sl], ref, tol, heads)
+            # from the GPU's attention output on, the oracle follows bit for bit
+            _, so, co, _ = O.hadamard_quant_act(att_g, None, 1e-6)
+            _, o = O.linear(co, so, *lw["o"])
+            hh = x_in + o
+            qh, sh = O.quant_act(hh, None, 1e-6)
+            _, up = O.linear(qh, sh, *lw["up"])
+            _, gate = O.linear(qh, sh, *lw["gate"])
+            _, sd, cd, _ = O.hadamard_quant_act(O.squared_relu_glu(gate, up), None, 1e-6)
+            _, dd = O.linear(cd, sd, *lw["down"])
+            assert np.array_equal(host(h), hh) and np.array_equal(host(d), dd)
+            x_in = hh + dd
+            parts = (h, d)
