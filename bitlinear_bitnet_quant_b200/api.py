@@ -9,6 +9,7 @@ If the library is missing, loading raises instead of falling back.
 from __future__ import annotations
 
 import ctypes
+import glob
 import os
 import re
 
@@ -66,6 +67,8 @@ _SIGNATURES = {
     "bitnet_attention": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64, ctypes.c_int,
                                         ctypes.c_int, _i64, _c_void_p, _c_void_p]),
     "bitnet_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
+    "bitnet_measure_i8_mma": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_void_p, _c_void_p,
+                                             _c_void_p]),
 }
 
 
@@ -76,10 +79,12 @@ class BitnetError(RuntimeError):
 
 
 def header_functions() -> list[str]:
-    """Names of the functions include/bitnet.h declares."""
-    with open(os.path.join(build_lib.INCLUDE, "bitnet.h")) as f:
-        text = f.read()
-    return re.findall(r"^BITNET_API\s+[\w\s\*]+?\b(bitnet_\w+)\s*\(", text, flags=re.M)
+    """Names of the functions the headers under include/ declare."""
+    names = []
+    for h in sorted(glob.glob(os.path.join(build_lib.INCLUDE, "*.h"))):
+        with open(h) as f:
+            names += re.findall(r"^BITNET_API\s+[\w\s\*]+?\b(bitnet_\w+)\s*\(", f.read(), flags=re.M)
+    return names
 
 
 def lib() -> ctypes.CDLL:
@@ -345,6 +350,16 @@ def bitnet_attention(Q: torch.Tensor, Kc: torch.Tensor, Vc: torch.Tensor, B: int
     _check("bitnet_attention", lib().bitnet_attention(
         _ptr(Q), _ptr(Kc), _ptr(Vc), B, L, t0, heads, d, Kc.shape[1], _ptr(A), _stream(stream)))
     return A
+
+
+def bitnet_measure_i8_mma(n_mma: int, bn: int, ctas: int, stream=None):
+    """Enqueues the int8 tensor-core throughput measurement; returns the (cycles,
+    nanoseconds) device tensors [ctas] it fills."""
+    cyc = torch.zeros((ctas,), dtype=torch.int64, device="cuda")
+    ns = torch.zeros((ctas,), dtype=torch.int64, device="cuda")
+    _check("bitnet_measure_i8_mma", lib().bitnet_measure_i8_mma(int(n_mma), int(bn), int(ctas), _ptr(cyc), _ptr(ns),
+                                                                _stream(stream)))
+    return cyc, ns
 
 
 def bitnet_device_error() -> int:

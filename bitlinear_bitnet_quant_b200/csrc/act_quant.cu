@@ -521,6 +521,154 @@ hadamard_quant_i4_row_kernel(const TIn* __restrict__ X, const float* __restrict_
 // ---------------------------------------------------------------------------
 // host launchers (called from abi.cu after validation)
 // ---------------------------------------------------------------------------
+// ---------------------------------------------------------------------------
+// RMSNorm + Hadamard + int4, one token per CTA of T = K / 32 threads (K =
+// 4096, 8192 or 16384: W = log2(T / 32) = 2, 3 or 4 warp bits), 32 elements per
+// thread, for blocks of b = 2^L >= 1024.  The element index bits are handled in
+// three groups, each while a thread holds all 32 elements the group's stages
+// pair up (stages always in the order stride 1, 2, ..., b/2):
+//   mapping A: thread t holds elements 32t .. 32t+31 (bits 0-4 in-thread):
+//              coalesced loads, the sum of squares (in-thread tree, lanes,
+//              warps in order), the norm, stages 0-4;
+//   mapping B: in-thread bits 5-9, thread = (bits 10.. << 5) | bits 0-4:
+//              stages 5-9;
+//   mapping C: in-thread bits 10..10+W-1 and 0..4-W, thread = bits 5-W .. 9:
+//              stages 10 .. L-1, the normalisation c_b, the absmax and the
+//              codes (bit 0 is in-thread, so codes pair into bytes there).
+// The row goes through shared memory between mappings with one pad word per
+// 32 (every access pattern is conflict-free).  Fewer registers per thread
+// than the 128-element kernel, so more warps keep the SM busy; every value is
+// the one the other Hadamard kernels produce.
+// ---------------------------------------------------------------------------
+BN_DEV int hsidx(int e) { return e + (e >> 5); }
+
+template <int W>
+BN_DEV int map_b(int t, int c) { return ((t >> 5) << 10) | (c << 5) | (t & 31); }
+
+template <int W>
+BN_DEV int map_c(int t, int c) {
+  constexpr int LOW = 5 - W;                       // low in-thread bits
+  return ((c >> LOW) << 10) | (t << LOW) | (c & ((1 << LOW) - 1));
+}
+
+// Radix-2 stages s = S0 .. S1-1 (stride 2^s) on 32 in-thread values whose
+// in-thread index bit (s - SHIFT) is element bit s.
+template <int S0, int S1, int SHIFT>
+BN_DEV void fwht32(float (&v)[32]) {
+#pragma unroll
+  for (int st = S0; st < S1; ++st) {
+    const int h = 1 << (st - SHIFT);
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      if ((c & h) == 0) {
+        const float a = v[c], b = v[c + h];
+        v[c] = __fadd_rn(a, b);
+        v[c + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+}
+
+template <typename TIn, int L, int W, int PRE>
+__global__ void __launch_bounds__(32 << W, (32 << W) == 256 ? 4 : (32 << W) == 128 ? 8 : 2)
+hadamard_quant_i4_split_kernel(const TIn* __restrict__ X, const float* __restrict__ B, int K,
+                               const float* __restrict__ gamma, float eps, float cb, uint8_t* __restrict__ Xq4,
+                               float* __restrict__ s_x, float* __restrict__ T_dbg) {
+  constexpr int T = 32 << W, NW = 1 << W, LOW = 5 - W;
+  static_assert(L >= 10 && L <= 10 + W, "block of 2^10 .. K");
+  extern __shared__ float hs[];
+  uint8_t* bytes = reinterpret_cast<uint8_t*>(hs + (K + K / 32));
+  __shared__ float red[NW];
+  pdl_launch_dependents();
+  pdl_wait();                                // X may come from, and Xq4 may still be read by, the previous kernel
+  const int m = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+
+  float v[32];
+  {
+    const size_t off = (size_t)m * K + (size_t)t * 32;
+    constexpr int E = InVec<TIn>::E;
+#pragma unroll
+    for (int q = 0; q < 32 / E; ++q) {
+      float tmp[E];
+      load_chunk<PRE, TIn, E>(X + off + q * E, B + off + q * E, nullptr, tmp);
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[q * E + e] = tmp[e];
+    }
+  }
+  // ---- sum of squares: in-thread tree (first level fused), lanes, warps in order ----
+  float part;
+  {
+    float sq[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) sq[c] = __fadd_rn(__fmul_rn(v[2 * c], v[2 * c]), __fmul_rn(v[2 * c + 1], v[2 * c + 1]));
+    part = warp_tree_sum(tree_sum<16>(sq));
+  }
+  if (lane == 0) red[warp] = part;
+  __syncthreads();
+  float w[NW];
+#pragma unroll
+  for (int i = 0; i < NW; ++i) w[i] = red[i];
+  const float ss = tree_sum<NW>(w);
+  const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)K), eps)));
+  if (gamma != nullptr) {
+    const float* gp = gamma + (size_t)t * 32;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] = __fmul_rn(__fmul_rn(v[c], r), __ldg(gp + c));
+  } else {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] = __fmul_rn(v[c], r);
+  }
+  // ---- stages 0-4 (mapping A) ----
+  fwht32<0, 5, 0>(v);
+#pragma unroll
+  for (int c = 0; c < 32; ++c) hs[hsidx(32 * t + c)] = v[c];
+  __syncthreads();
+  // ---- stages 5-9 (mapping B) ----
+#pragma unroll
+  for (int c = 0; c < 32; ++c) v[c] = hs[hsidx(map_b<W>(t, c))];
+  fwht32<5, 10, 5>(v);
+#pragma unroll
+  for (int c = 0; c < 32; ++c) hs[hsidx(map_b<W>(t, c))] = v[c];
+  __syncthreads();
+  // ---- stages 10 .. L-1 (mapping C), normalisation, absmax ----
+#pragma unroll
+  for (int c = 0; c < 32; ++c) v[c] = hs[hsidx(map_c<W>(t, c))];
+  fwht32<10, L, 10 - LOW>(v);
+  float amax = 0.f;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    v[c] = __fmul_rn(v[c], cb);
+    amax = fmaxf(amax, fabsf(v[c]));
+  }
+  amax = warp_max(amax);
+  __syncthreads();                           // every thread has read red[] (the sum of squares)
+  if (lane == 0) red[warp] = amax;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < NW; ++i) amax = fmaxf(amax, red[i]);
+  const float sc = __fdiv_rn(7.0f, fmaxf(amax, 1e-5f));
+  if (T_dbg != nullptr) {
+    float* dst = T_dbg + (size_t)m * K;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) dst[map_c<W>(t, c)] = v[c];
+  }
+  // ---- codes, two per byte (element pairs differ in bit 0, held in-thread) ----
+#pragma unroll
+  for (int hh = 0; hh < NW; ++hh) {
+    const int e0 = map_c<W>(t, hh << LOW);           // first element of this run of 2^LOW
+#pragma unroll
+    for (int j = 0; j < (1 << LOW); j += 2) {
+      const int c = (hh << LOW) + j;
+      bytes[(e0 + j) >> 1] = (uint8_t)pair_nibbles(nib(v[c], sc), nib(v[c + 1], sc));
+    }
+  }
+  __syncthreads();
+  const uint4* src = reinterpret_cast<const uint4*>(bytes);
+  uint4* dst = reinterpret_cast<uint4*>(Xq4 + (size_t)m * (K / 2));
+  for (int q = t; q < K / 32; q += T) dst[q] = src[q];
+  if (t == 0) s_x[m] = sc;
+}
+
 template <typename TIn, int NT, int IT, int PRE>
 static cudaError_t launch_q8(const void* X, const float* B, float* H, int M, int K, const float* gamma, float eps,
                              int8_t* Xq, float* s_x, cudaStream_t st) {
@@ -583,6 +731,28 @@ static cudaError_t launch_h4(const void* X, const float* B, int M, int K, const 
     if (e != cudaSuccess) return e;
     return launch_pdl(rk, dim3(M), dim3(HR_THREADS), rsmem, st, 1u, static_cast<const TIn*>(X), B, K, gamma, eps, cb,
                       Xq4, s_x, T_dbg);
+  }
+  // Many tokens, K = 4096 / 8192 / 16384, blocks of 1024 or more: one token per
+  // CTA of K / 32 threads, 32 elements per thread.
+  if constexpr (L >= 10) {
+    const int W = K == 4096 ? 2 : K == 8192 ? 3 : K == 16384 ? 4 : 0;
+    if (W != 0 && L <= 10 + W) {
+      const size_t ssmem = (size_t)(K + K / 32) * sizeof(float) + (size_t)K / 2;
+#define BN_HS(WW)                                                                                           \
+  do {                                                                                                      \
+    if constexpr (L <= 10 + WW) {                                                                           \
+      auto sk = hadamard_quant_i4_split_kernel<TIn, L, WW, PRE>;                                            \
+      cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(sk), ssmem);                          \
+      if (e != cudaSuccess) return e;                                                                       \
+      return launch_pdl(sk, dim3(M), dim3(32 << WW), ssmem, st, 1u, static_cast<const TIn*>(X), B, K,       \
+                        gamma, eps, cb, Xq4, s_x, T_dbg);                                                   \
+    }                                                                                                       \
+  } while (0)
+      if (W == 2) BN_HS(2);
+      if (W == 3) BN_HS(3);
+      if (W == 4) BN_HS(4);
+#undef BN_HS
+    }
   }
   const size_t smem = (size_t)TPB * ((K + 2 * (K >> 7) + 3) & ~3) * sizeof(float) + (size_t)TPB * 4 * sizeof(float);
   auto kern = hadamard_quant_i4_kernel<TIn, L, PRE>;

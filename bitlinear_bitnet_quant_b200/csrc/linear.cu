@@ -120,25 +120,34 @@ linear_simt_kernel(const uint8_t* __restrict__ Xq, const float* __restrict__ s_x
 constexpr int TC_THREADS = 320;
 constexpr int TC_CONV_THREADS = 256;
 constexpr int TC_BK = 128;
-constexpr int TC_WBYTES = 128 * TC_BK / 4;       // packed W tile: 128 rows x 32 B
 
-template <int BN, int ACT_BITS>
+// MB = 128 or 256 weight rows per CTA.  With 256, two M = 128 MMAs (two
+// accumulators, two A slices in tensor memory) share every activation tile:
+// half the activation bytes per MMA, at one CTA per SM (all 512 columns).
+// On B200 a CTA's TMA stream delivers about 27 bytes per clock (measured with
+// 16 KB tiles, whatever their layout), below the 80 bytes per clock that a
+// 128 x 128 tile needs at the int8 MMA rate: the activation bytes per MMA set
+// the GEMM's speed.
+template <int BN, int ACT_BITS, int MB = 128>
 struct TcCfg {
+  static constexpr int RB = MB / 128;                          // row blocks = accumulators
   static constexpr int XBYTES = BN * 128;                      // int8 operand tile
   static constexpr int XRAW = ACT_BITS == 4 ? BN * 64 : 0;     // packed int4 tile
-  static constexpr int STAGE = XBYTES + XRAW + TC_WBYTES;
-  // One accumulator: measured on B200, rotating tcgen05.mma over several
-  // accumulators costs ~3x more per instruction than chaining into one.
-  static constexpr int DCOLS = BN;                             // accumulator columns
+  static constexpr int WBYTES = MB * TC_BK / 4;                // packed W tile: MB rows x 32 B
+  static constexpr int STAGE = XBYTES + XRAW + WBYTES;
+  // One accumulator per row block: measured on B200, rotating tcgen05.mma over
+  // several accumulators costs ~3x more per instruction than chaining into one.
+  static constexpr int DCOLS = BN * RB;                        // accumulator columns
+  static constexpr int ACOLS = 32 * RB;                        // A columns per stage
   // 256 columns: two CTAs share an SM, so one CTA's prologue and epilogue
-  // overlap the other's MMAs (a 256-token tile needs all 512 columns)
-  static constexpr int TMEM_BUDGET = BN <= 128 ? 256 : 512;
+  // overlap the other's MMAs (a 256-token or 256-row tile needs all 512 columns)
+  static constexpr int TMEM_BUDGET = (BN <= 128 && RB == 1) ? 256 : 512;
   static constexpr int SMEM_BUDGET = TMEM_BUDGET == 256 ? 108 * 1024 : 200 * 1024;
   static constexpr int S_SMEM = SMEM_BUDGET / STAGE;
-  static constexpr int S_TMEM = (TMEM_BUDGET - DCOLS) / 32;
+  static constexpr int S_TMEM = (TMEM_BUDGET - DCOLS) / ACOLS;
   static constexpr int S0 = S_SMEM < S_TMEM ? S_SMEM : S_TMEM;
   static constexpr int S = S0 > 6 ? 6 : S0;
-  static constexpr int COLS_NEEDED = DCOLS + 32 * S;
+  static constexpr int COLS_NEEDED = DCOLS + ACOLS * S;
   static constexpr int TMEM_COLS = COLS_NEEDED <= 32 ? 32 : COLS_NEEDED <= 64 ? 64 :
                                    COLS_NEEDED <= 128 ? 128 : COLS_NEEDED <= 256 ? 256 : 512;
   static constexpr size_t SMEM = (size_t)S * STAGE + 1024;
@@ -171,12 +180,13 @@ struct TcMaps {
   CUtensorMap y[GROUP_MAX];
 };
 
-template <int BN, int ACT_BITS, typename TOut>
-__global__ void __launch_bounds__(TC_THREADS, BN <= 128 ? 2 : 1)
+template <int BN, int ACT_BITS, typename TOut, int MB>
+__global__ void __launch_bounds__(TC_THREADS, (BN <= 128 && MB == 128) ? 2 : 1)
 linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CUtensorMap tmX,
                  const __grid_constant__ LinGroup grp, int use_tma_store, const float* __restrict__ s_x,
                  int M, int K, int ksplit) {
-  using C = TcCfg<BN, ACT_BITS>;
+  using C = TcCfg<BN, ACT_BITS, MB>;
+  constexpr int RB = C::RB;
   constexpr int S = C::S;
   constexpr uint32_t XTX = ACT_BITS == 8 ? BN * 128 : BN * 64;      // activation bytes per stage
   constexpr uint32_t PART_BYTES = 128u * BN * 4u;                    // one split-K partial tile
@@ -195,7 +205,7 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
   auto xs = [&](int s) { return base + (size_t)s * C::XBYTES; };                          // 1024-aligned
   auto xraw = [&](int s) { return base + (size_t)S * C::XBYTES + (size_t)s * C::XRAW; };
-  auto ws = [&](int s) { return base + (size_t)S * (C::XBYTES + C::XRAW) + (size_t)s * TC_WBYTES; };
+  auto ws = [&](int s) { return base + (size_t)S * (C::XBYTES + C::XRAW) + (size_t)s * C::WBYTES; };
   // split-K partial sums, [slot][column][row] int32: in the leader, slot r-1 receives rank r;
   // in the other ranks, slot 0 stages the outgoing partial
   int32_t* red = reinterpret_cast<int32_t*>(base + (size_t)S * C::STAGE);
@@ -211,7 +221,7 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
   TOut* __restrict__ Y = static_cast<TOut*>(grp.Y[gi]);
   int32_t* __restrict__ acc_dbg = grp.acc_dbg[gi];
   const int N = grp.N[gi];
-  const int n0 = (blockIdx.x - grp.first[gi]) * 128;
+  const int n0 = (blockIdx.x - grp.first[gi]) * MB;
   const int m0 = blockIdx.y * BN;
   const int kr = blockIdx.z;                    // rank inside the cluster (cluster = 1 x 1 x ksplit)
   const int nk_all = K / TC_BK;
@@ -253,7 +263,7 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
     if (lane == 0) {
       // weights do not depend on the previous kernel: start streaming them now
       for (int i = 0; i < pre; ++i) {
-        mbar_arrive_expect_tx(&bar_wfull[i], TC_WBYTES);
+        mbar_arrive_expect_tx(&bar_wfull[i], C::WBYTES);
         tma_load_2d(ws(i), tmW, &bar_wfull[i], (kb + i) * (TC_BK / 4), n0);
       }
     }
@@ -282,7 +292,7 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
       for (int i = pre; i < nk; ++i) {
         const int s = i % S, r = i / S;
         if (!mbar_wait(&bar_empty[s], (r - 1) & 1, DEV_ERR_TIMEOUT_EMPTY)) break;
-        mbar_arrive_expect_tx(&bar_wfull[s], TC_WBYTES);
+        mbar_arrive_expect_tx(&bar_wfull[s], C::WBYTES);
         tma_load_2d(ws(s), tmW, &bar_wfull[s], (kb + i) * (TC_BK / 4), n0);
         load_x(i);
         issued = i + 1;
@@ -307,8 +317,11 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
 #pragma unroll
         for (int kk = 0; kk < TC_BK / 32; ++kk) {
           const uint64_t bdesc = smem_desc_k_sw128(xaddr + kk * 32);
-          const uint32_t aaddr = tmem + (uint32_t)(C::DCOLS + 32 * s + 8 * kk);
-          mma_i8_ts(tmem, aaddr, bdesc, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int rb = 0; rb < RB; ++rb) {
+            const uint32_t aaddr = tmem + (uint32_t)(C::DCOLS + C::ACOLS * s + 32 * rb + 8 * kk);
+            mma_i8_ts(tmem + (uint32_t)(BN * rb), aaddr, bdesc, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         if (i + S < nk) mma_commit(&bar_empty[s]);   // only stages that are refilled need releasing
       }
@@ -327,23 +340,29 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
       const int s = i % S, r = i / S;
       if (!mbar_wait_warp(&bar_wfull[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
       tc_fence_after();
-      // 64 weights of this row -> 16 tensor-memory columns
+      // 64 weights of this row (of each row block) -> 16 tensor-memory columns
       // the tile arrives with the 32-byte swizzle: the two 16-byte halves of
       // row r are swapped when bit 2 of r is set, so the eight rows a
       // quarter-warp reads fall on distinct banks
-      const uint4 w = *reinterpret_cast<const uint4*>(ws(s) + 32 * row + 16 * (h ^ ((row >> 2) & 1)));
+      uint4 w[RB];
+#pragma unroll
+      for (int rb = 0; rb < RB; ++rb)
+        w[rb] = *reinterpret_cast<const uint4*>(ws(s) + 32 * (row + 128 * rb) + 16 * (h ^ ((row >> 2) & 1)));
       if constexpr (ACT_BITS == 8) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_empty[s]);   // packed tile consumed
       }
-      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-      uint32_t a[16];
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
+      for (int rb = 0; rb < RB; ++rb) {
+        const uint32_t wv[4] = {w[rb].x, w[rb].y, w[rb].z, w[rb].w};
+        uint32_t a[16];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) a[4 * g + jj] = unpack4(wv[g], jj);
+        for (int g = 0; g < 4; ++g) {
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) a[4 * g + jj] = unpack4(wv[g], jj);
+        }
+        tmem_st16(lane_base + (uint32_t)(C::DCOLS + C::ACOLS * s + 32 * rb + 16 * h), a);
       }
-      tmem_st16(lane_base + (uint32_t)(C::DCOLS + 32 * s + 16 * h), a);
       if constexpr (ACT_BITS == 4) {
         // int4 activation tile: widen to int8 (16*x) in the 128-byte-swizzled layout
         if (!mbar_wait_warp(&bar_xfull[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
@@ -400,11 +419,17 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
       const bool sdq_ok = mbar_wait_warp(&bar_sdq, 0, DEV_ERR_TIMEOUT_ACC);
       const bool red_ok = ksplit == 1 || mbar_wait_cluster(&bar_red, 0, DEV_ERR_TIMEOUT_CLUSTER);
       const bool ok = acc_ok && red_ok && sdq_ok;
-      const int n = n0 + row;
+#pragma unroll 1
+      for (int rb = 0; rb < RB; ++rb) {
+      const int n = n0 + 128 * rb + row;
+      if (rb > 0 && use_tma_store) {
+        // the thread that stored the previous row block waited for its copy
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+      }
 #pragma unroll 1
       for (int g0 = 0; g0 < NCH; g0 += G) {
         uint32_t v[G][16];
-        load_cols<NC, G>(lane_base + (uint32_t)(cbeg + g0 * NC), v);
+        load_cols<NC, G>(lane_base + (uint32_t)(BN * rb + cbeg + g0 * NC), v);
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const int c0 = cbeg + (g0 + g) * NC;
@@ -439,9 +464,10 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
         fence_proxy_async_smem();
         asm volatile("bar.sync 1, 256;" ::: "memory");
         if (ct == 0 && ok) {
-          tma_store_2d(tmY, ostage, n0, m0);
+          tma_store_2d(tmY, ostage, n0 + 128 * rb, m0);
           bulk_wait_all();
         }
+      }
       }
     }
   }
@@ -497,9 +523,9 @@ template <typename T> struct MapType;
 template <> struct MapType<float> { static constexpr CUtensorMapDataType v = CU_TENSOR_MAP_DATA_TYPE_FLOAT32; };
 template <> struct MapType<__nv_bfloat16> { static constexpr CUtensorMapDataType v = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; };
 
-template <int BN, int ACT_BITS, typename TOut>
+template <int BN, int ACT_BITS, typename TOut, int MB>
 static cudaError_t launch_tc(LinGroup grp, const void* Xq, const float* s_x, int M, int K, cudaStream_t st) {
-  using C = TcCfg<BN, ACT_BITS>;
+  using C = TcCfg<BN, ACT_BITS, MB>;
   TcMaps maps;                                     // copied into the launch's parameters
   CUtensorMap tmX;
   const bool ok = ACT_BITS == 8
@@ -513,14 +539,14 @@ static cudaError_t launch_tc(LinGroup grp, const void* Xq, const float* s_x, int
     if (grp.acc_dbg[g] != nullptr || ((uint64_t)grp.N[g] * sizeof(TOut)) % 16 != 0) use_tma_store = 0;
   grp.first[0] = 0;
   for (int g = 0; g < grp.count; ++g) {
-    if (!make_map_bytes(&maps.w[g], grp.pkW[g], (uint64_t)K / 4, (uint64_t)grp.N[g], TC_BK / 4, 128,
+    if (!make_map_bytes(&maps.w[g], grp.pkW[g], (uint64_t)K / 4, (uint64_t)grp.N[g], TC_BK / 4, MB,
                         CU_TENSOR_MAP_SWIZZLE_32B))
       return cudaErrorInvalidValue;
     if (use_tma_store && !make_map_2d(&maps.y[g], grp.Y[g], MapType<TOut>::v, (uint64_t)grp.N[g], (uint64_t)M,
                                       (uint64_t)grp.N[g] * sizeof(TOut), 128, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
     if (!use_tma_store) maps.y[g] = tmX;           // unused
-    grp.first[g + 1] = grp.first[g] + (grp.N[g] + 127) / 128;
+    grp.first[g + 1] = grp.first[g] + (grp.N[g] + MB - 1) / MB;
   }
   for (int g = grp.count; g < GROUP_MAX; ++g) {
     maps.w[g] = maps.w[0];
@@ -533,7 +559,7 @@ static cudaError_t launch_tc(LinGroup grp, const void* Xq, const float* s_x, int
   const int tiles = ntiles * ((M + BN - 1) / BN);
   const int nk = K / TC_BK;
   int ksplit = 1;
-  if (BN <= 32) {
+  if (BN <= 32 && MB == 128) {
     int sms = 148, dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -545,7 +571,7 @@ static cudaError_t launch_tc(LinGroup grp, const void* Xq, const float* s_x, int
   // barrier would never run.  Shared memory (228 KB per SM) enforces the bound.
   const size_t min_smem = (size_t)(228 * 1024) / (512 / C::TMEM_COLS + 1) + 1024;
   if (smem < min_smem) smem = min_smem;
-  auto kern = linear_tc_kernel<BN, ACT_BITS, TOut>;
+  auto kern = linear_tc_kernel<BN, ACT_BITS, TOut, MB>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   dim3 grid(ntiles, (M + BN - 1) / BN, ksplit);
@@ -555,10 +581,26 @@ static cudaError_t launch_tc(LinGroup grp, const void* Xq, const float* s_x, int
 
 template <int ACT_BITS, typename TOut>
 static cudaError_t dispatch_tc(const LinGroup& grp, const void* Xq, const float* s_x, int M, int K, cudaStream_t st) {
-  if (M <= 16) return launch_tc<16, ACT_BITS, TOut>(grp, Xq, s_x, M, K, st);
-  if (M <= 32) return launch_tc<32, ACT_BITS, TOut>(grp, Xq, s_x, M, K, st);
-  if (M <= 64) return launch_tc<64, ACT_BITS, TOut>(grp, Xq, s_x, M, K, st);
-  return launch_tc<128, ACT_BITS, TOut>(grp, Xq, s_x, M, K, st);
+  if (M <= 16) return launch_tc<16, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
+  if (M <= 32) return launch_tc<32, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
+  if (M <= 64) return launch_tc<64, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
+  // 256 weight rows per CTA halve the activation bytes per MMA but hold a
+  // whole SM: only when the tiles fill at least two such waves
+  int sms = 148, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int tiles256 = 0;
+  for (int g = 0; g < grp.count; ++g) tiles256 += (grp.N[g] + 255) / 256;
+  tiles256 *= (M + 127) / 128;
+  if (tiles256 >= 2 * sms) return launch_tc<128, ACT_BITS, TOut, 256>(grp, Xq, s_x, M, K, st);
+  return launch_tc<128, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
+}
+
+// The 256-row tile with any number of tokens above 64 (tests of the tile itself).
+template <int ACT_BITS, typename TOut>
+static cudaError_t dispatch_tc256(const LinGroup& grp, const void* Xq, const float* s_x, int M, int K,
+                                  cudaStream_t st) {
+  return launch_tc<128, ACT_BITS, TOut, 256>(grp, Xq, s_x, M, K, st);
 }
 
 template <int ACT_BITS, typename TOut>

@@ -179,6 +179,21 @@ def test_hadamard_quant_many_tokens(M, K, b, dtype):
     _check_hadamard(x, dtype, b)
 
 
+@pytest.mark.parametrize("M,K,b,dtype,use_gamma", [(640, 4096, 0, "bf16", False), (600, 8192, 1024, "f32", False),
+                                                   (700, 16384, 8192, "bf16", True), (620, 8192, 0, "f32", True),
+                                                   (900, 4096, 2048, "f32", False)])
+def test_hadamard_quant_split_kernel(M, K, b, dtype, use_gamma):
+    """Many tokens at K = 4096 / 8192 / 16384 with blocks of 1024 or more: the
+    kernel that spreads a token over K/32 threads (three index-bit groups)."""
+    rng = np.random.default_rng(M + K + b)
+    x = wl.add_channel_outliers(rng, wl.student_t(rng, (M, K)), 0.005, 50.0)
+    x[0] = 0
+    x[1] = 0
+    x[1, K // 3] = 3.0
+    gamma = rng.uniform(0.5, 1.5, K).astype(np.float32) if use_gamma else None
+    _check_hadamard(x, dtype, b, gamma)
+
+
 def test_hadamard_gamma_and_edges():
     rng = np.random.default_rng(3)
     x = rng.standard_normal((6, 1024)).astype(np.float32)
@@ -704,3 +719,19 @@ def test_chain_with_attention_prefill_then_decode():
             assert np.array_equal(host(h), hh) and np.array_equal(host(d), dd)
             x_in = hh + dd
             parts = (h, d)
+
+
+# ------------------------------------------------------------ measurement -----
+
+def test_measure_i8_mma_runs():
+    """The int8 tensor-core throughput measurement completes on every SM, and its
+    cycle count is plausible: at least half the cycles that 128 x bn x 32 MACs
+    per MMA take at 8192 MACs per clock and SM (about the nominal dense rate)."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for bn in (128, 256):
+        cyc, ns = api.bitnet_measure_i8_mma(2048, bn, sms)
+        torch.cuda.synchronize()
+        c, t = host(cyc), host(ns)
+        assert np.all(c > 0) and np.all(t > 0)
+        assert np.all(c >= 2048 * (128 * bn * 32 // 8192) * 0.5)
+    assert api.bitnet_device_error() == 0
