@@ -579,8 +579,11 @@ static cudaError_t launch_tc(LinGroup grp, const void* Xq, const float* s_x, int
                     s_x, M, K, ksplit);
 }
 
+// rows: 0 = choose the weight rows per CTA, 128 or 256 = that tile.
 template <int ACT_BITS, typename TOut>
-static cudaError_t dispatch_tc(const LinGroup& grp, const void* Xq, const float* s_x, int M, int K, cudaStream_t st) {
+static cudaError_t dispatch_tc(const LinGroup& grp, const void* Xq, const float* s_x, int M, int K, int rows,
+                               cudaStream_t st) {
+  if (rows == 256) return launch_tc<128, ACT_BITS, TOut, 256>(grp, Xq, s_x, M, K, st);
   if (M <= 16) return launch_tc<16, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
   if (M <= 32) return launch_tc<32, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
   if (M <= 64) return launch_tc<64, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
@@ -592,15 +595,8 @@ static cudaError_t dispatch_tc(const LinGroup& grp, const void* Xq, const float*
   int tiles256 = 0;
   for (int g = 0; g < grp.count; ++g) tiles256 += (grp.N[g] + 255) / 256;
   tiles256 *= (M + 127) / 128;
-  if (tiles256 >= 2 * sms) return launch_tc<128, ACT_BITS, TOut, 256>(grp, Xq, s_x, M, K, st);
+  if (rows == 0 && tiles256 >= 2 * sms) return launch_tc<128, ACT_BITS, TOut, 256>(grp, Xq, s_x, M, K, st);
   return launch_tc<128, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
-}
-
-// The 256-row tile with any number of tokens above 64 (tests of the tile itself).
-template <int ACT_BITS, typename TOut>
-static cudaError_t dispatch_tc256(const LinGroup& grp, const void* Xq, const float* s_x, int M, int K,
-                                  cudaStream_t st) {
-  return launch_tc<128, ACT_BITS, TOut, 256>(grp, Xq, s_x, M, K, st);
 }
 
 template <int ACT_BITS, typename TOut>
@@ -623,7 +619,8 @@ cudaError_t run_linear_decode_group(const LinGroup& grp, const void* Xq, int act
 cudaError_t run_linear_group(const LinGroup& grp, const void* Xq, int act_bits, const float* s_x, int M, int K,
                              int y_bf16, int path, cudaStream_t st);
 
-// path: 0 = automatic, 1 = SIMT, 2 = tcgen05, 3 = warp-MMA decode kernel
+// path: 0 = automatic, 1 = SIMT, 2 = tcgen05, 3 = warp-MMA decode kernel, 4 = tcgen05 with
+// 256 weight rows per CTA
 cudaError_t run_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                        int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, int path, cudaStream_t st) {
   // up to 32 tokens: one pass over the weights with warp-level MMA
@@ -646,20 +643,24 @@ cudaError_t run_linear(const void* Xq, int act_bits, const float* s_x, const uin
   grp.acc_dbg[0] = acc_dbg;
   grp.N[0] = N;
   grp.count = 1;
-  return run_linear_group(grp, Xq, act_bits, s_x, M, K, y_bf16, 2, st);
+  return run_linear_group(grp, Xq, act_bits, s_x, M, K, y_bf16, path, st);
 }
 
 // Several weight matrices sharing Xq and s_x in one launch.  path: 0 = automatic,
-// 2 = tcgen05, 3 = warp-MMA decode kernel.
+// 2 = tcgen05 with 128 weight rows per CTA, 3 = warp-MMA decode kernel, 4 =
+// tcgen05 with 256 weight rows per CTA.
 cudaError_t run_linear_group(const LinGroup& grp, const void* Xq, int act_bits, const float* s_x, int M, int K,
                              int y_bf16, int path, cudaStream_t st) {
   if ((path == 0 || path == 3) && decode_path_applies(M, K))
     return run_linear_decode_group(grp, Xq, act_bits, s_x, M, K, y_bf16, st);
   if (path == 3) return cudaErrorInvalidValue;
+  const int rows = path == 2 ? 128 : path == 4 ? 256 : 0;
   if (act_bits == 8) {
-    return y_bf16 ? dispatch_tc<8, __nv_bfloat16>(grp, Xq, s_x, M, K, st) : dispatch_tc<8, float>(grp, Xq, s_x, M, K, st);
+    return y_bf16 ? dispatch_tc<8, __nv_bfloat16>(grp, Xq, s_x, M, K, rows, st)
+                  : dispatch_tc<8, float>(grp, Xq, s_x, M, K, rows, st);
   }
-  return y_bf16 ? dispatch_tc<4, __nv_bfloat16>(grp, Xq, s_x, M, K, st) : dispatch_tc<4, float>(grp, Xq, s_x, M, K, st);
+  return y_bf16 ? dispatch_tc<4, __nv_bfloat16>(grp, Xq, s_x, M, K, rows, st)
+                : dispatch_tc<4, float>(grp, Xq, s_x, M, K, rows, st);
 }
 
 }  // namespace bitnet

@@ -278,10 +278,13 @@ BITNET_API int bitnet_relu2_glu(const float* gate, const float* up, float* out, 
  * chosen per call instead of automatically; every choice computes the same
  * bit-exact result.  Arguments as for the plain calls, plus `kernel`:
  *   bitnet_linear_kernel:    0 = automatic (as bitnet_linear), 1 = CUDA-core
- *                            dp4a kernel, 2 = tcgen05 tensor-core kernel,
+ *                            dp4a kernel, 2 = tcgen05 tensor-core kernel
+ *                            with 128 weight rows per CTA,
  *                            3 = warp-MMA decode kernel (BITNET_ERR_SHAPE for
  *                            shapes it does not cover: M > 32, K % 512 != 0 or
- *                            K > 16384).
+ *                            K > 16384), 4 = tcgen05 kernel with 256 weight
+ *                            rows per CTA (the automatic choice for large
+ *                            products, forced here at any shape).
  *   bitnet_bitlinear_kernel: 0-3 = the int8 quantiser, then that linear
  *                            kernel; 4 = the fused single kernel described at
  *                            bitnet_bitlinear (BITNET_ERR_SHAPE outside its range).

@@ -388,6 +388,16 @@ def test_linear_group(M, K, Ns, act_bits, out):
         assert torch.equal(Y1, Y)
 
 
+@pytest.mark.parametrize("M,N,K,act_bits,out", [(130, 520, 512, 8, "f32"), (33, 300, 1024, 4, "bf16"),
+                                              (256, 768, 2048, 8, "bf16"), (200, 260, 384, 4, "f32"),
+                                              (5, 256, 256, 8, "f32")])
+def test_linear_256_row_tile(M, N, K, act_bits, out):
+    """The tcgen05 kernel with two accumulators (256 weight rows per CTA), forced
+    at small and ragged shapes: bit-exact accumulators and outputs."""
+    qx, qw, s_x, s_w = _random_codes(M, N, K, act_bits, seed=M + N + K)
+    _check_linear(qx, qw, s_x, s_w, act_bits, out, path=4)
+
+
 # ------------------------------------------------------- fused BitLinear ----
 
 def _check_bitlinear(M, N, K, dtype, use_gamma, out, path=0, seed=0):
@@ -453,6 +463,35 @@ def test_linear_prefill_sampled():
     acc_o, y_o = O.linear(q_o, s_o, qw_o, s_wo)
     assert np.array_equal(host(acc)[rows], acc_o)
     assert np.array_equal(O.bf16_round(host(Y.float())[rows]), O.bf16_round(y_o))
+    # the launch the bench times (no accumulator output: 256-row tiles and the
+    # tensor-store epilogue) gives the same bits everywhere
+    Y2, _ = api.bitnet_linear(q, 8, s, pk, s_w, out_dtype=torch.bfloat16)
+    assert torch.equal(Y2.view(torch.int16), Y.view(torch.int16))
+    assert np.array_equal(O.bf16_round(host(Y2.float())[rows]), O.bf16_round(y_o))
+
+
+@pytest.mark.parametrize("M,N,K,out", [(2048, 4736, 512, "f32"), (2100, 4800, 1024, "bf16")])
+def test_linear_256_row_tile_store_path(M, N, K, out):
+    """Enough tiles for the automatic 256-row choice, with the tensor-store
+    epilogue (no accumulator output), including a ragged last row block and
+    token tile: sampled rows against the oracle, and every element against
+    the 128-row tile."""
+    qx, qw, s_x, s_w = _random_codes(M, N, K, 8, seed=M + N)
+    od = torch.float32 if out == "f32" else torch.bfloat16
+    args = (dev(qx), 8, dev(s_x), dev(O.pack_ternary(qw)), dev(np.array([s_w], np.float32)))
+    Y, _ = api.bitnet_linear(*args, out_dtype=od)
+    Y2, _ = api.bitnet_linear(*args, out_dtype=od, kernel=2)
+    rows = np.concatenate([np.random.default_rng(2).choice(M, size=10, replace=False), [0, M - 1]])
+    _, y_o = O.linear(qx[rows], s_x[rows], qw, s_w)
+    got = host(Y.float())[rows]
+    if out == "f32":
+        assert np.array_equal(got.view(np.uint32), y_o.view(np.uint32))
+    else:
+        assert np.array_equal(O.bf16_round(got), O.bf16_round(y_o))
+    Y3, _ = api.bitnet_linear(*args, out_dtype=od, kernel=4)
+    assert torch.equal(Y.view(torch.int16) if out == "bf16" else Y, Y3.view(torch.int16) if out == "bf16" else Y3)
+    # the 128-row kernel on the same operands (its own launch shape)
+    assert torch.equal(Y.float(), Y2.float())
 
 
 def test_hbitlinear_sampled():
