@@ -102,9 +102,41 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def int8_peak(peaks) -> float:
-    """Dense int8 peak in TOPS: the measured bf16 burst x the nominal int8 : bf16 ratio (4.5 : 2.25)."""
+def int8_peak_from_bf16(peaks) -> float:
+    """Dense int8 TOPS derived from the measured bf16 burst x the nominal int8 : bf16 ratio (4.5 : 2.25)."""
     return 2.0 * float(peaks["bf16_tflops"])
+
+
+def measure_int8_peak(api, stream, sms: int) -> dict:
+    """Dense int8 tensor-core throughput measured here: back-to-back tcgen05 kind::i8
+    MMAs (128 x 128 x 32, the GEMM's instruction form) on every SM, between CUDA
+    events; the SM clock over the run comes from the kernel's own cycle and
+    nanosecond counters."""
+    import torch
+    n_mma = 65536
+    best = None
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cyc, ns = api.bitnet_measure_i8_mma(n_mma, 128, sms, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        tops = 2.0 * 128 * 128 * 32 * n_mma * sms / (ms * 1e-3) / 1e12
+        mhz = float((cyc.double() / ns.double()).median().item() * 1e3)
+        if best is None or tops > best["tops"]:
+            best = {"tops": tops, "sm_mhz": mhz, "ms": ms}
+    return {"value": best["tops"], "unit": "TOPS", "sm_mhz_during": best["sm_mhz"],
+            "method": f"bitnet_measure_i8_mma: {n_mma} back-to-back 128x128x32 kind::i8 MMAs per SM on {sms} SMs, "
+                      "CUDA events (best of 3)"}
+
+
+def tensor_peak(ctx) -> tuple:
+    """(peak TOPS, source) for the int8 tensor-core rooflines: this run's measurement."""
+    m = ctx.get("int8_peak")
+    if m is not None:
+        return m["value"], "measured in this run (bitnet_measure_i8_mma)"
+    return int8_peak_from_bf16(ctx["peaks"][0]), "2 x bf16 burst (nominal int8 : bf16 ratio)"
 
 
 def profiled_traffic(kernel_tag: str):
@@ -385,13 +417,16 @@ def run_layer(name, args, ctx):
                 "algorithmic_bytes_per_launch": alg_bytes}
     else:
         ops = 2.0 * M * N * K
-        roof = {"bound": "tensor", "achieved": ops / lin_s / 1e12, "peak": int8_peak(peaks), "unit": "TOPS",
+        tp, tsrc = tensor_peak(ctx)
+        roof = {"bound": "tensor", "achieved": ops / lin_s / 1e12, "peak": tp, "unit": "TOPS",
                 "kernel": "bitnet_linear (tcgen05 kind::i8)", "algorithmic_ops_per_launch": ops,
-                "peak_note": "2 x measured bf16 burst (nominal int8 : bf16 ratio)",
+                "peak_note": tsrc,
+                "frac_of_bf16_derived_peak": ops / lin_s / 1e12 / int8_peak_from_bf16(peaks),
                 "frac_of_nominal_4500_tops": ops / lin_s / 1e12 / NOMINAL_INT8_TOPS}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = profiled_traffic(f"linear_{name}")
-    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    if roof["bound"] == "hbm":
+        roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     quant_bytes = x_in_bytes + xq_bytes + 4 * M
     sub.update({
         "value": M * world / step_s, "unit": "tokens/s", "ms_per_step": t_step["ms"],
@@ -563,15 +598,18 @@ def run_chain(name, args, ctx):
                 "unit": "GB/s", "kernel": f"bitnet_linear(_group), all {4 * CHAIN_LAYERS} launches of a step",
                 "algorithmic_bytes_per_step": packed + act_bytes}
     else:
-        roof = {"bound": "tensor", "achieved": ops / lin_s / 1e12, "peak": int8_peak(peaks),
+        tp, tsrc = tensor_peak(ctx)
+        roof = {"bound": "tensor", "achieved": ops / lin_s / 1e12, "peak": tp,
                 "unit": "TOPS", "kernel": f"bitnet_linear(_group), all {4 * CHAIN_LAYERS} launches of a step",
-                "algorithmic_ops_per_step": ops, "peak_note": "2 x measured bf16 burst (nominal int8 : bf16 ratio)",
+                "algorithmic_ops_per_step": ops, "peak_note": tsrc,
+                "frac_of_bf16_derived_peak": ops / lin_s / 1e12 / int8_peak_from_bf16(peaks),
                 "frac_of_nominal_4500_tops": ops / lin_s / 1e12 / NOMINAL_INT8_TOPS}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = profiled_traffic(f"linear_{name}")
-    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    if roof["bound"] == "hbm":
+        roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     # whole-step view: the slower of the weight stream and the integer work, against the step time
-    ideal = max((packed + act_bytes) / (peaks["hbm_gbs"] * 1e9), ops / (int8_peak(peaks) * 1e12))
+    ideal = max((packed + act_bytes) / (peaks["hbm_gbs"] * 1e9), ops / (tensor_peak(ctx)[0] * 1e12))
     extra = {}
     if att is not None:
         att_s = t_att["ms"] / 1e3
@@ -813,6 +851,7 @@ def run_ours(args, rank, world, local_rank):
     timer = Timer(stream, world, dev, args.steps, args.min_time, clocks)
     ctx = {"api": api, "rank": rank, "world": world, "dev": dev, "stream": stream, "timer": timer,
            "clocks": clocks, "peaks": load_peaks()}
+    ctx["int8_peak"] = measure_int8_peak(api, stream, torch.cuda.get_device_properties(dev).multi_processor_count)
     names = ORDER if args.workload == "all" else [args.workload]
     subs = {}
     try:
@@ -852,10 +891,12 @@ def run_ours(args, rank, world, local_rank):
     line["config"]["timing"] = ("R replays of a CUDA graph of K steps between a barrier and a device synchronise "
                                 "on both sides; CUDA events around each replay on the launching stream; median")
     line["config"]["parallelism"] = f"dp{world} (independent batches per rank)"
-    for k in ("step_roofline", "cpu_baseline", "cpu_baseline_all_cores"):
+    for k in ("step_roofline", "cpu_baseline", "cpu_baseline_all_cores", "attention", "quant_roofline",
+              "decode_variants", "weights_quant"):
         if k in head:
             line[k] = head[k]
     line["configs"] = {n: s for n, s in subs.items() if n != head_name}
+    line["int8_peak_measured"] = ctx["int8_peak"]
     line["clocks_whole_run"] = overall
     return line
 
