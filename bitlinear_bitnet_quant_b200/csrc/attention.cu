@@ -132,115 +132,135 @@ attention_decode_kernel(const float* __restrict__ Q, const float* __restrict__ K
 }
 
 // ---------------------------------------------------------------------------
-// many queries per sequence (prefill): one CTA per (block of 16 queries, head,
-// sequence).  Key blocks of 64 keys (and their values) are staged in shared
-// memory; 256 threads compute the 16 x 64 scores (4 each), update the running
-// softmax of their query row, then accumulate P V (8 output dimensions each).
+// many queries per sequence (prefill): one CTA per (block of 32 queries, head,
+// sequence).  Key blocks of 32 keys and their values are double-buffered in
+// shared memory by 16-byte asynchronous copies (the next block streams in
+// while this one is used).  Thread (r, g) of the 256 (r = query row, g < 8)
+// computes the scores of keys g, g+8, g+16, g+24 of the block (128-term dot
+// products from float4 reads that are broadcasts or conflict-free), updates
+// its row's running softmax with the 8 threads of the row (shuffles), then
+// accumulates P V for dimensions 32 i + 4 g .. + 3, i < 4.
 // ---------------------------------------------------------------------------
-constexpr int ATP_QB = 16;
-constexpr int ATP_KB = 64;
-constexpr int ATP_PITCH = ATT_D + 4;               // floats per staged row (conflict-free float4 reads)
-constexpr size_t ATP_SMEM = (size_t)(ATP_QB + 2 * ATP_KB) * ATP_PITCH * 4 + (size_t)ATP_QB * ATP_KB * 4;
+constexpr int ATP_QB = 32;
+constexpr int ATP_KB = 32;
+constexpr int ATP_PITCH = ATT_D + 4;               // floats per staged row
+constexpr size_t ATP_SMEM = (size_t)(ATP_QB + 4 * ATP_KB) * ATP_PITCH * 4 + (size_t)ATP_QB * (ATP_KB + 1) * 4;
+
+// 16-byte asynchronous copies of key/value rows j0 .. j0+31 (rows past nk zero).
+BN_DEV void att_stage_kv(const float* kbase, const float* vbase, int HD, int j0, int nk, float* ks, float* vs) {
+  for (int e = threadIdx.x; e < ATP_KB * (ATT_D / 4); e += 256) {
+    const int rr = e / (ATT_D / 4), cc = e - rr * (ATT_D / 4);
+    const bool in = rr < nk;
+    const size_t off = in ? (size_t)(j0 + rr) * HD + 4 * cc : 0;
+    cp_async_16(smem_u32(ks + rr * ATP_PITCH + 4 * cc), kbase + off, in ? 16u : 0u);
+    cp_async_16(smem_u32(vs + rr * ATP_PITCH + 4 * cc), vbase + off, in ? 16u : 0u);
+  }
+  cp_async_commit();
+}
 
 __global__ void __launch_bounds__(256, 2)
 attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ Kc, const float* __restrict__ Vc,
                          int L, int t0, int HD, int T_cap, float scale, float* __restrict__ A) {
   extern __shared__ float atp[];
-  float* qs = atp;                                  // [16][PITCH]
-  float* ks = qs + ATP_QB * ATP_PITCH;              // [64][PITCH]
-  float* vs = ks + ATP_KB * ATP_PITCH;              // [64][PITCH]
-  float* ps = vs + ATP_KB * ATP_PITCH;              // [16][64] probabilities of the current block
+  float* qs = atp;                                  // [32][PITCH]
+  float* kbuf = qs + ATP_QB * ATP_PITCH;            // [2][32][PITCH]
+  float* vbuf = kbuf + 2 * ATP_KB * ATP_PITCH;      // [2][32][PITCH]
+  float* ps = vbuf + 2 * ATP_KB * ATP_PITCH;        // [32][33] probabilities of the current block
   pdl_launch_dependents();
   pdl_wait();
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int l0 = qb * ATP_QB;
   const int nq = L - l0 < ATP_QB ? L - l0 : ATP_QB;
   const int tid = threadIdx.x;
-  const int row = tid >> 4, c16 = tid & 15;         // query row; column slot
-  // queries
+  const int row = tid >> 3, g = tid & 7;
+  const float* kbase = Kc + (size_t)b * T_cap * HD + h * ATT_D;
+  const float* vbase = Vc + (size_t)b * T_cap * HD + h * ATT_D;
+  const int kend = t0 + l0 + nq;                     // keys 0 .. kend-1 are needed by the block
+  const int nblk = (kend + ATP_KB - 1) / ATP_KB;
+  att_stage_kv(kbase, vbase, HD, 0, kend < ATP_KB ? kend : ATP_KB, kbuf, vbuf);
   for (int e = tid; e < ATP_QB * (ATT_D / 4); e += 256) {
     const int rr = e / (ATT_D / 4), cc = e - rr * (ATT_D / 4);
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (rr < nq) v = *reinterpret_cast<const float4*>(Q + ((size_t)b * L + l0 + rr) * HD + h * ATT_D + 4 * cc);
     *reinterpret_cast<float4*>(qs + rr * ATP_PITCH + 4 * cc) = v;
   }
-  const int qpos = t0 + l0 + row;                    // this thread's query position
-  const int kend = t0 + l0 + nq;                     // keys 0 .. kend-1 are needed by the block
+  const int qpos = t0 + l0 + row;
   float m = -INFINITY, sum = 0.f;
-  float o[8];
+  float o[4][4];
 #pragma unroll
-  for (int t = 0; t < 8; ++t) o[t] = 0.f;
-  const float* kbase = Kc + (size_t)b * T_cap * HD + h * ATT_D;
-  const float* vbase = Vc + (size_t)b * T_cap * HD + h * ATT_D;
-  for (int j0 = 0; j0 < kend; j0 += ATP_KB) {
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) o[i][c] = 0.f;
+  for (int blk = 0; blk < nblk; ++blk) {
+    const int j0 = blk * ATP_KB;
     const int nk = kend - j0 < ATP_KB ? kend - j0 : ATP_KB;
-    __syncthreads();                                 // the previous block's K, V, P are consumed
-    for (int e = tid; e < ATP_KB * (ATT_D / 4); e += 256) {
-      const int rr = e / (ATT_D / 4), cc = e - rr * (ATT_D / 4);
-      float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
-      if (rr < nk) {
-        kv = *reinterpret_cast<const float4*>(kbase + (size_t)(j0 + rr) * HD + 4 * cc);
-        vv = *reinterpret_cast<const float4*>(vbase + (size_t)(j0 + rr) * HD + 4 * cc);
-      }
-      *reinterpret_cast<float4*>(ks + rr * ATP_PITCH + 4 * cc) = kv;
-      *reinterpret_cast<float4*>(vs + rr * ATP_PITCH + 4 * cc) = vv;
+    if (blk + 1 < nblk) {
+      const int j1 = j0 + ATP_KB;
+      att_stage_kv(kbase, vbase, HD, j1, kend - j1 < ATP_KB ? kend - j1 : ATP_KB,
+                   kbuf + ((blk + 1) & 1) * ATP_KB * ATP_PITCH, vbuf + ((blk + 1) & 1) * ATP_KB * ATP_PITCH);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      cp_async_wait_all();
     }
-    __syncthreads();
-    // scores of keys c16 + 16 u for this thread's query row
-    float s[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) s[u] = 0.f;
+    __syncthreads();                                 // this block's K, V (and the queries) are in place
+    const float* ks = kbuf + (blk & 1) * ATP_KB * ATP_PITCH;
+    const float* vs = vbuf + (blk & 1) * ATP_KB * ATP_PITCH;
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
     const float* qr = qs + row * ATP_PITCH;
 #pragma unroll 8
     for (int dd = 0; dd < ATT_D; dd += 4) {
       const float4 qv = *reinterpret_cast<const float4*>(qr + dd);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const float4 kv = *reinterpret_cast<const float4*>(ks + (c16 + 16 * u) * ATP_PITCH + dd);
+        const float4 kv = *reinterpret_cast<const float4*>(ks + (g + 8 * u) * ATP_PITCH + dd);
         s[u] += qv.x * kv.x + qv.y * kv.y + qv.z * kv.z + qv.w * kv.w;
       }
     }
     float bm = -INFINITY;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int j = j0 + c16 + 16 * u;
-      s[u] = (c16 + 16 * u < nk && j <= qpos) ? s[u] * scale : -INFINITY;
+      const int jj = g + 8 * u;
+      s[u] = (jj < nk && j0 + jj <= qpos) ? s[u] * scale : -INFINITY;
       bm = fmaxf(bm, s[u]);
     }
 #pragma unroll
-    for (int off = 8; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+    for (int off = 4; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
     const float mn = fmaxf(m, bm);
     // a query row whose keys in this block are all masked keeps its state
     const float corr = mn == -INFINITY ? 1.f : expf(m - mn);
-    float ps_sum = 0.f;
+    float psum = 0.f;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const float p = s[u] == -INFINITY ? 0.f : expf(s[u] - mn);
-      ps[row * ATP_KB + c16 + 16 * u] = p;
-      ps_sum += p;
+      ps[row * (ATP_KB + 1) + g + 8 * u] = p;
+      psum += p;
     }
 #pragma unroll
-    for (int off = 8; off > 0; off >>= 1) ps_sum += __shfl_xor_sync(0xffffffffu, ps_sum, off);
-    sum = sum * corr + ps_sum;
+    for (int off = 4; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
+    sum = sum * corr + psum;
     m = mn;
 #pragma unroll
-    for (int t = 0; t < 8; ++t) o[t] *= corr;
-    __syncwarp();
-    // P V for dimensions 8 c16 .. 8 c16 + 7 of this query row
-    const float* pr = ps + row * ATP_KB;
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) o[i][c] *= corr;
+    __syncwarp();                                    // the row's probabilities come from its 8 lanes
+    const float* pr = ps + row * (ATP_KB + 1);
     for (int j = 0; j < nk; ++j) {
       const float p = pr[j];
-      const float4 v0 = *reinterpret_cast<const float4*>(vs + j * ATP_PITCH + 8 * c16);
-      const float4 v1 = *reinterpret_cast<const float4*>(vs + j * ATP_PITCH + 8 * c16 + 4);
-      o[0] += p * v0.x; o[1] += p * v0.y; o[2] += p * v0.z; o[3] += p * v0.w;
-      o[4] += p * v1.x; o[5] += p * v1.y; o[6] += p * v1.z; o[7] += p * v1.w;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = *reinterpret_cast<const float4*>(vs + j * ATP_PITCH + 32 * i + 4 * g);
+        o[i][0] += p * v.x; o[i][1] += p * v.y; o[i][2] += p * v.z; o[i][3] += p * v.w;
+      }
     }
+    __syncthreads();                                 // every thread is done with this block's buffers
   }
   if (row < nq) {
     const float inv = 1.0f / sum;
-    float* dst = A + ((size_t)b * L + l0 + row) * HD + h * ATT_D + 8 * c16;
-    *reinterpret_cast<float4*>(dst) = make_float4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
-    *reinterpret_cast<float4*>(dst + 4) = make_float4(o[4] * inv, o[5] * inv, o[6] * inv, o[7] * inv);
+    float* dst = A + ((size_t)b * L + l0 + row) * HD + h * ATT_D + 4 * g;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<float4*>(dst + 32 * i) = make_float4(o[i][0] * inv, o[i][1] * inv, o[i][2] * inv, o[i][3] * inv);
   }
 }
 
@@ -260,7 +280,7 @@ cudaError_t run_attention(const float* Q, const float* Kc, const float* Vc, int 
                           int T_cap, float* A, cudaStream_t st) {
   const int HD = heads * d;
   const float scale = (float)(1.0 / sqrt((double)d));
-  if (L < ATP_QB) {
+  if (L < 16) {
     return launch_pdl(attention_decode_kernel, dim3((unsigned)(B * L), (unsigned)heads), dim3(32 * ATD_WARPS), 0, st,
                       1u, Q, Kc, Vc, L, t0, HD, T_cap, scale, A);
   }
