@@ -558,12 +558,18 @@ static cudaError_t launch_tc(LinGroup grp, const void* Xq, const float* s_x, int
   const int ntiles = grp.first[grp.count];
   const int tiles = ntiles * ((M + BN - 1) / BN);
   const int nk = K / TC_BK;
+  // With 64 or 128 tokens per tile the partial tiles (32 or 64 KB) take shared
+  // memory, so a split tile holds an SM alone; it pays when the tiles would
+  // otherwise leave SMs idle (the N = 2048 layers of a 512-token batch), and a
+  // CTA alone on its SM also gets the SM's whole load bandwidth.
   int ksplit = 1;
-  if (BN <= 32 && MB == 128) {
+  if (MB == 128) {
     int sms = 148, dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    while (ksplit < 8 && tiles * ksplit * 2 <= 2 * sms && ksplit * 2 <= nk) ksplit *= 2;
+    const int kmax = BN <= 32 ? 8 : BN == 64 ? 4 : 2;
+    const int per_sm = BN <= 32 ? 2 : 1;
+    while (ksplit < kmax && tiles * ksplit * 2 <= per_sm * sms && ksplit * 2 <= nk) ksplit *= 2;
   }
   size_t smem = C::SMEM + (size_t)(ksplit - 1) * 128 * BN * sizeof(int32_t);
   // Never more CTAs per SM than tensor memory can serve at once (512 columns):

@@ -388,6 +388,25 @@ def test_linear_group(M, K, Ns, act_bits, out):
         assert torch.equal(Y1, Y)
 
 
+@pytest.mark.parametrize("M,N,K,act_bits,out", [(128, 2048, 2048, 8, "f32"), (512, 2048, 5632, 4, "f32"),
+                                              (100, 384, 1024, 8, "bf16"), (64, 640, 4096, 4, "f32")])
+def test_linear_split_k_wide_tiles(M, N, K, act_bits, out):
+    """Few 64- or 128-token tiles: K split over a cluster, partial sums meeting in
+    the leader's shared memory; bit-exact like every other launch shape."""
+    qx, qw, s_x, s_w = _random_codes(M, N, K, act_bits, seed=M * 3 + N + K)
+    _check_linear(qx, qw, s_x, s_w, act_bits, out, path=2)
+    # and through the tensor-store epilogue (no accumulator output)
+    od = torch.float32 if out == "f32" else torch.bfloat16
+    xq = dev(qx) if act_bits == 8 else dev(O.pack_int4(qx))
+    Y, _ = api.bitnet_linear(xq, act_bits, dev(s_x), dev(O.pack_ternary(qw)), dev(np.array([s_w], np.float32)),
+                             out_dtype=od)
+    _, y_o = O.linear(qx, s_x, qw, s_w)
+    if out == "f32":
+        assert np.array_equal(host(Y).view(np.uint32), y_o.view(np.uint32))
+    else:
+        assert np.array_equal(O.bf16_round(host(Y.float())), O.bf16_round(y_o))
+
+
 @pytest.mark.parametrize("M,N,K,act_bits,out", [(130, 520, 512, 8, "f32"), (33, 300, 1024, 4, "bf16"),
                                               (256, 768, 2048, 8, "bf16"), (200, 260, 384, 4, "f32"),
                                               (5, 256, 256, 8, "f32")])
