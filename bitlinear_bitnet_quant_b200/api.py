@@ -69,6 +69,7 @@ _SIGNATURES = {
     "bitnet_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
     "bitnet_measure_i8_mma": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_void_p, _c_void_p,
                                              _c_void_p]),
+    "bitnet_selftest_wait_timeout": (ctypes.c_int, [_c_void_p]),
 }
 
 
@@ -360,6 +361,11 @@ def bitnet_measure_i8_mma(n_mma: int, bn: int, ctas: int, stream=None):
     _check("bitnet_measure_i8_mma", lib().bitnet_measure_i8_mma(int(n_mma), int(bn), int(ctas), _ptr(cyc), _ptr(ns),
                                                                 _stream(stream)))
     return cyc, ns
+
+
+def bitnet_selftest_wait_timeout(stream=None) -> None:
+    """Enqueues the bounded-wait self-test (a wait that runs out after ~2 s)."""
+    _check("bitnet_selftest_wait_timeout", lib().bitnet_selftest_wait_timeout(_stream(stream)))
 
 
 def bitnet_device_error() -> int:

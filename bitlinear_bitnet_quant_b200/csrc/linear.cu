@@ -124,10 +124,10 @@ constexpr int TC_BK = 128;
 // MB = 128 or 256 weight rows per CTA.  With 256, two M = 128 MMAs (two
 // accumulators, two A slices in tensor memory) share every activation tile:
 // half the activation bytes per MMA, at one CTA per SM (all 512 columns).
-// On B200 a CTA's TMA stream delivers about 27 bytes per clock (measured with
-// 16 KB tiles, whatever their layout), below the 80 bytes per clock that a
-// 128 x 128 tile needs at the int8 MMA rate: the activation bytes per MMA set
-// the GEMM's speed.
+// On B200 an SM takes in about 47-50 bytes per clock (measured with 16 KB
+// transfers, whatever the method), below the 80 bytes per clock that a
+// 128 x 128 tile needs at the int8 MMA rate: the bytes per MMA set the speed
+// of the 128-row tile.
 template <int BN, int ACT_BITS, int MB = 128>
 struct TcCfg {
   static constexpr int RB = MB / 128;                          // row blocks = accumulators
@@ -145,14 +145,20 @@ struct TcCfg {
   static constexpr int SMEM_BUDGET = TMEM_BUDGET == 256 ? 108 * 1024 : 200 * 1024;
   static constexpr int S_SMEM = SMEM_BUDGET / STAGE;
   static constexpr int S_TMEM = (TMEM_BUDGET - DCOLS) / ACOLS;
+  // 128-row tile: one ring of stages (shared-memory stage s and tensor-memory
+  // A slot s go together; two CTAs per SM keep enough steps in flight).
+  // 256-row tile: one CTA per SM, so the shared-memory ring runs deeper than
+  // the four A slots tensor memory has room for; each A slot is released by
+  // its own MMA commit.
   static constexpr int S0 = S_SMEM < S_TMEM ? S_SMEM : S_TMEM;
-  static constexpr int S = S0 > 6 ? 6 : S0;
-  static constexpr int COLS_NEEDED = DCOLS + ACOLS * S;
+  static constexpr int S = RB == 1 ? (S0 > 6 ? 6 : S0) : (S_SMEM > 8 ? 8 : S_SMEM);   // shared-memory stages
+  static constexpr int ST = RB == 1 ? S : S_TMEM;                                      // tensor-memory A slots
+  static constexpr int COLS_NEEDED = DCOLS + ACOLS * ST;
   static constexpr int TMEM_COLS = COLS_NEEDED <= 32 ? 32 : COLS_NEEDED <= 64 ? 64 :
                                    COLS_NEEDED <= 128 ? 128 : COLS_NEEDED <= 256 ? 256 : 512;
   static constexpr size_t SMEM = (size_t)S * STAGE + 1024;
   static constexpr int HALF = BN / 2;                          // token columns per epilogue warp
-  static_assert(S >= 2, "pipeline needs two stages");
+  static_assert(S >= 2 && ST >= 2 && ST <= S, "pipeline needs two stages");
   static_assert((size_t)BN * 128 * 4 <= (size_t)S * STAGE, "output staging fits in the operand stages");
 };
 
@@ -187,7 +193,7 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
                  int M, int K, int ksplit) {
   using C = TcCfg<BN, ACT_BITS, MB>;
   constexpr int RB = C::RB;
-  constexpr int S = C::S;
+  constexpr int S = C::S, ST = C::ST;
   constexpr uint32_t XTX = ACT_BITS == 8 ? BN * 128 : BN * 64;      // activation bytes per stage
   constexpr uint32_t PART_BYTES = 128u * BN * 4u;                    // one split-K partial tile
   constexpr int NC = C::HALF < 16 ? C::HALF : 16;                    // epilogue column chunk
@@ -197,7 +203,8 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
   // wfull: weight tile landed; xfull: activation tile landed; conv: weights in TMEM (and, for
   // int4, activations widened); empty: stage free; acc: all MMAs done; sdq: scales ready;
   // red: split-K partials of the other ranks landed (leader only)
-  __shared__ __align__(8) uint64_t bar_wfull[S], bar_xfull[S], bar_empty[S], bar_conv[S];
+  // afree: the A slot's MMAs are done (used only when the A ring is shorter than the stage ring)
+  __shared__ __align__(8) uint64_t bar_wfull[S], bar_xfull[S], bar_empty[S], bar_conv[ST], bar_afree[ST];
   __shared__ __align__(8) uint64_t bar_acc, bar_sdq, bar_red;
   __shared__ uint32_t tmem_base_sh;
   __shared__ float sdq[BN];
@@ -233,7 +240,10 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
       mbar_init(&bar_wfull[s], 1);
       mbar_init(&bar_xfull[s], 1);
       mbar_init(&bar_empty[s], 1 + 8);
-      mbar_init(&bar_conv[s], 8);
+    }
+    for (int a = 0; a < ST; ++a) {
+      mbar_init(&bar_conv[a], 8);
+      mbar_init(&bar_afree[a], 1);
     }
     mbar_init(&bar_acc, 1);
     mbar_init(&bar_sdq, 1);
@@ -310,8 +320,9 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
       constexpr uint32_t IDESC = idesc_i8(128, BN);
       for (int i = 0; i < nk; ++i) {
         const int s = i % S, r = i / S;
+        const int a = i % ST, ra = i / ST;
         if (!mbar_wait(&bar_xfull[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
-        if (!mbar_wait(&bar_conv[s], r & 1, DEV_ERR_TIMEOUT_A)) break;
+        if (!mbar_wait(&bar_conv[a], ra & 1, DEV_ERR_TIMEOUT_A)) break;
         tc_fence_after();
         const uint32_t xaddr = smem_u32(xs(s));
 #pragma unroll
@@ -319,11 +330,12 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
           const uint64_t bdesc = smem_desc_k_sw128(xaddr + kk * 32);
 #pragma unroll
           for (int rb = 0; rb < RB; ++rb) {
-            const uint32_t aaddr = tmem + (uint32_t)(C::DCOLS + C::ACOLS * s + 32 * rb + 8 * kk);
+            const uint32_t aaddr = tmem + (uint32_t)(C::DCOLS + C::ACOLS * a + 32 * rb + 8 * kk);
             mma_i8_ts(tmem + (uint32_t)(BN * rb), aaddr, bdesc, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
           }
         }
         if (i + S < nk) mma_commit(&bar_empty[s]);   // only stages that are refilled need releasing
+        if (ST < S && i + ST < nk) mma_commit(&bar_afree[a]);
       }
       mma_commit(&bar_acc);
       mbar_wait(&bar_acc, 0, DEV_ERR_TIMEOUT_ACC, false);   // no MMA in flight at teardown
@@ -338,6 +350,7 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
 
     for (int i = 0; i < nk; ++i) {
       const int s = i % S, r = i / S;
+      const int a = i % ST, ra = i / ST;
       if (!mbar_wait_warp(&bar_wfull[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
       tc_fence_after();
       // 64 weights of this row (of each row block) -> 16 tensor-memory columns
@@ -352,16 +365,21 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_empty[s]);   // packed tile consumed
       }
+      if constexpr (ST < S) {
+        // the A slot is free once the MMAs of step i - ST are done
+        if (i >= ST && !mbar_wait_warp(&bar_afree[a], (ra - 1) & 1, DEV_ERR_TIMEOUT_A)) break;
+        tc_fence_after();
+      }
 #pragma unroll
       for (int rb = 0; rb < RB; ++rb) {
         const uint32_t wv[4] = {w[rb].x, w[rb].y, w[rb].z, w[rb].w};
-        uint32_t a[16];
+        uint32_t av[16];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) a[4 * g + jj] = unpack4(wv[g], jj);
+          for (int jj = 0; jj < 4; ++jj) av[4 * g + jj] = unpack4(wv[g], jj);
         }
-        tmem_st16(lane_base + (uint32_t)(C::DCOLS + C::ACOLS * s + 32 * rb + 16 * h), a);
+        tmem_st16(lane_base + (uint32_t)(C::DCOLS + C::ACOLS * a + 32 * rb + 16 * h), av);
       }
       if constexpr (ACT_BITS == 4) {
         // int4 activation tile: widen to int8 (16*x) in the 128-byte-swizzled layout
@@ -386,7 +404,7 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_conv[s]);
+      if (lane == 0) mbar_arrive(&bar_conv[a]);
     }
 
     // ------------------------------------------------------------ epilogue

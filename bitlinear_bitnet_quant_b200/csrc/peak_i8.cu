@@ -65,7 +65,32 @@ peak_i8_kernel(int n_mma, unsigned long long* __restrict__ cycles, unsigned long
   }
 }
 
+// Self-test of the bounded waits: one thread waits on an mbarrier that nothing
+// will ever complete, through the same mbar_wait every pipeline uses.  After
+// its time limit (about two seconds) the wait gives up, records the code in
+// g_device_error and returns; the kernel then exits normally.
+__global__ void wait_timeout_selftest_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  mbar_wait(&bar, 0, DEV_ERR_TIMEOUT_FULL, false);
+}
+
 }  // namespace bitnet
+
+extern "C" int bitnet_selftest_wait_timeout(void* stream) {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return BITNET_ERR_CUDA;
+  }
+  if (major != 10) return BITNET_ERR_UNSUPPORTED;
+  bitnet::wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  if (cudaGetLastError() != cudaSuccess) return BITNET_ERR_CUDA;
+  return BITNET_OK;
+}
 
 extern "C" int bitnet_measure_i8_mma(int n_mma, int bn, int ctas, unsigned long long* cycles,
                                      unsigned long long* nanos, void* stream) {

@@ -1,9 +1,9 @@
 /*
- * bitnet_measure.h - measurement entry points of libbitnet.so.
+ * bitnet_measure.h - measurement and self-test entry points of libbitnet.so.
  *
  * These are not steps of the BitLinear method: they measure the hardware the
  * method's kernels run on, so that roofline fractions use a measured
- * denominator.  Same conventions as bitnet.h (device pointers owned by the
+ * denominator, and exercise the library's failure path.  Same conventions as bitnet.h (device pointers owned by the
  * caller, asynchronous on `stream`, host-side validation, bitnet_status codes).
  */
 #ifndef BITNET_B200_MEASURE_H
@@ -30,6 +30,16 @@ extern "C" {
  */
 BITNET_API int bitnet_measure_i8_mma(int n_mma, int bn, int ctas, unsigned long long* cycles,
                                      unsigned long long* nanos, void* stream);
+
+/*
+ * Self-test of the failure path of the pipelines' bounded waits.  Enqueues one
+ * kernel whose single thread waits on a barrier that nothing completes, with
+ * the wait every kernel of the library uses: after about two seconds it gives
+ * up, records a nonzero code in the device error flag (read it with
+ * bitnet_device_error) and the kernel exits normally.  No fault, trap or
+ * endless loop is involved; the CUDA context stays usable.
+ */
+BITNET_API int bitnet_selftest_wait_timeout(void* stream);
 
 #ifdef __cplusplus
 }

@@ -793,3 +793,16 @@ def test_measure_i8_mma_runs():
         assert np.all(c > 0) and np.all(t > 0)
         assert np.all(c >= 2048 * (128 * bn * 32 // 8192) * 0.5)
     assert api.bitnet_device_error() == 0
+
+
+def test_bounded_wait_gives_up_and_reports():
+    """A pipeline wait that nothing completes gives up after its time limit,
+    records a code in the device error flag and lets the kernel exit: the
+    context stays usable and the next call computes correctly."""
+    assert api.bitnet_device_error() == 0
+    api.bitnet_selftest_wait_timeout()
+    torch.cuda.synchronize()
+    assert api.bitnet_device_error() == 1          # the code of a timed-out "full" wait
+    assert api.bitnet_device_error() == 0          # reading clears it
+    qx, qw, s_x, s_w = _random_codes(40, 256, 512, 8, seed=77)
+    _check_linear(qx, qw, s_x, s_w, 8, "f32", path=2)
