@@ -669,6 +669,123 @@ hadamard_quant_i4_split_kernel(const TIn* __restrict__ X, const float* __restric
   if (t == 0) s_x[m] = sc;
 }
 
+// ---------------------------------------------------------------------------
+// RMSNorm + Hadamard + int4 for blocks of b = 2^L <= 512 elements, one warp per
+// block and one CTA per token (K / b <= 32 warps; e.g. K = 5632 in 11 blocks of
+// 512, the down projection's input).  Lane j holds the E = b / 32 consecutive
+// elements b w + E j .. of block w: stages of stride < E run in registers, the
+// five stages of stride E .. b/2 pair lanes (xor shuffles: the lower lane keeps
+// a + c, the upper a - c).  The sum of squares follows the fixed tree: in-lane,
+// lanes, then the warps' block sums in order, padded with zero subtrees.  Every
+// value is the one the other Hadamard kernels produce.
+// ---------------------------------------------------------------------------
+template <typename TIn, int L, int PRE>
+__global__ void __launch_bounds__(1024)
+hadamard_quant_i4_warp_kernel(const TIn* __restrict__ X, const float* __restrict__ B, int K,
+                              const float* __restrict__ gamma, float eps, float cb, uint8_t* __restrict__ Xq4,
+                              float* __restrict__ s_x, float* __restrict__ T_dbg) {
+  constexpr int E = 1 << (L - 5);
+  static_assert(L >= 6 && L <= 9, "2 to 16 elements per lane");
+  __shared__ float red[32];
+  pdl_launch_dependents();
+  pdl_wait();                                // X may come from, and Xq4 may still be read by, the previous kernel
+  const int m = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const size_t e0 = (size_t)warp * (E * 32) + (size_t)lane * E;      // first element of this lane
+  float v[E];
+  {
+    constexpr int EV = InVec<TIn>::E;
+    const size_t off = (size_t)m * K + e0;
+    if constexpr (E >= EV) {
+#pragma unroll
+      for (int q = 0; q < E / EV; ++q) {
+        float tmp[EV];
+        load_chunk<PRE, TIn, EV>(X + off + q * EV, B + off + q * EV, nullptr, tmp);
+#pragma unroll
+        for (int e = 0; e < EV; ++e) v[q * EV + e] = tmp[e];
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        float x;
+        if constexpr (sizeof(TIn) == 4) x = reinterpret_cast<const float*>(X)[off + e];
+        else x = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(X)[off + e] << 16);
+        if constexpr (PRE == PRE_GLU) x = relu2_times(x, B[off + e]);
+        v[e] = x;
+      }
+    }
+  }
+  // ---- sum of squares: in-lane tree, lanes, warps (zero-padded to 32) in order ----
+  float sq[E];
+#pragma unroll
+  for (int c = 0; c < E; ++c) sq[c] = __fmul_rn(v[c], v[c]);
+  float part = warp_tree_sum(tree_sum<E>(sq));
+  if (lane == 0) red[warp] = part;
+  __syncthreads();
+  float wsum[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) wsum[i] = i < nw ? red[i] : 0.f;
+  const float ss = tree_sum<32>(wsum);
+  const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)K), eps)));
+  if (gamma != nullptr) {
+#pragma unroll
+    for (int c = 0; c < E; ++c) v[c] = __fmul_rn(__fmul_rn(v[c], r), __ldg(gamma + e0 + c));
+  } else {
+#pragma unroll
+    for (int c = 0; c < E; ++c) v[c] = __fmul_rn(v[c], r);
+  }
+  // ---- stages of stride 1 .. E/2 in registers, then E .. b/2 across lanes ----
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+    for (int c = 0; c < E; ++c) {
+      if ((c & h) == 0) {
+        const float a = v[c], b = v[c + h];
+        v[c] = __fadd_rn(a, b);
+        v[c + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int lb = 1; lb < 32; lb <<= 1) {
+    const bool upper = (lane & lb) != 0;
+#pragma unroll
+    for (int c = 0; c < E; ++c) {
+      const float other = __shfl_xor_sync(0xffffffffu, v[c], lb);
+      v[c] = upper ? __fsub_rn(other, v[c]) : __fadd_rn(v[c], other);
+    }
+  }
+  // ---- normalise, absmax over the token ----
+  float amax = 0.f;
+#pragma unroll
+  for (int c = 0; c < E; ++c) {
+    v[c] = __fmul_rn(v[c], cb);
+    amax = fmaxf(amax, fabsf(v[c]));
+  }
+  amax = warp_max(amax);
+  __syncthreads();                           // every warp has read red[] (the sum of squares)
+  if (lane == 0) red[warp] = amax;
+  __syncthreads();
+  for (int i = 0; i < nw; ++i) amax = fmaxf(amax, red[i]);
+  const float sc = __fdiv_rn(7.0f, fmaxf(amax, 1e-5f));
+  if (T_dbg != nullptr) {
+#pragma unroll
+    for (int c = 0; c < E; ++c) T_dbg[(size_t)m * K + e0 + c] = v[c];
+  }
+  // ---- E / 2 bytes of codes per lane, contiguous ----
+  uint8_t* dst = Xq4 + (size_t)m * (K / 2) + e0 / 2;
+  if constexpr (E >= 8) {
+    uint32_t w[E / 8];
+#pragma unroll
+    for (int q = 0; q < E / 8; ++q) w[q] = pack_nibbles8(v + 8 * q, sc);
+    if constexpr (E == 16) *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+    else *reinterpret_cast<uint32_t*>(dst) = w[0];
+  } else {
+#pragma unroll
+    for (int c = 0; c < E; c += 2) dst[c / 2] = (uint8_t)pair_nibbles(nib(v[c], sc), nib(v[c + 1], sc));
+  }
+  if (threadIdx.x == 0) s_x[m] = sc;
+}
+
 template <typename TIn, int NT, int IT, int PRE>
 static cudaError_t launch_q8(const void* X, const float* B, float* H, int M, int K, const float* gamma, float eps,
                              int8_t* Xq, float* s_x, cudaStream_t st) {
@@ -720,6 +837,15 @@ static cudaError_t launch_h4(const void* X, const float* B, int M, int K, const 
   const int TPB = GP >= 128 ? 1 : 128 / GP;
   const int threads = TPB * GP;
   const float cb = (float)(1.0 / sqrt((double)(1 << L)));
+  // Blocks of 64 .. 512 elements and at most 32 of them: one warp per block.
+  if constexpr (L >= 6 && L <= 9) {
+    if (K / (1 << L) <= 32) {
+      auto wk = hadamard_quant_i4_warp_kernel<TIn, L, PRE>;
+      const float cbw = (float)(1.0 / sqrt((double)(1 << L)));
+      return launch_pdl(wk, dim3(M), dim3(32 * (K >> L)), 0, st, 1u, static_cast<const TIn*>(X), B, K, gamma, eps,
+                        cbw, Xq4, s_x, T_dbg);
+    }
+  }
   // Few tokens: the register kernel would leave most SMs idle; one CTA per token instead.
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

@@ -325,11 +325,13 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
         if (!mbar_wait(&bar_conv[a], ra & 1, DEV_ERR_TIMEOUT_A)) break;
         tc_fence_after();
         const uint32_t xaddr = smem_u32(xs(s));
+        // all of one accumulator's MMAs of the step, then the other's: switching the
+        // accumulator between consecutive MMAs costs about three times the MMA
 #pragma unroll
-        for (int kk = 0; kk < TC_BK / 32; ++kk) {
-          const uint64_t bdesc = smem_desc_k_sw128(xaddr + kk * 32);
+        for (int rb = 0; rb < RB; ++rb) {
 #pragma unroll
-          for (int rb = 0; rb < RB; ++rb) {
+          for (int kk = 0; kk < TC_BK / 32; ++kk) {
+            const uint64_t bdesc = smem_desc_k_sw128(xaddr + kk * 32);
             const uint32_t aaddr = tmem + (uint32_t)(C::DCOLS + C::ACOLS * a + 32 * rb + 8 * kk);
             mma_i8_ts(tmem + (uint32_t)(BN * rb), aaddr, bdesc, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
           }
