@@ -274,7 +274,9 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
       // weights do not depend on the previous kernel: start streaming them now
       for (int i = 0; i < pre; ++i) {
         mbar_arrive_expect_tx(&bar_wfull[i], C::WBYTES);
-        tma_load_2d(ws(i), tmW, &bar_wfull[i], (kb + i) * (TC_BK / 4), n0);
+#pragma unroll
+        for (int rb = 0; rb < RB; ++rb)
+          tma_load_2d(ws(i) + rb * (C::WBYTES / RB), tmW, &bar_wfull[i], (kb + i) * (TC_BK / 4), n0 + 128 * rb);
       }
     }
     __syncwarp();
@@ -303,7 +305,9 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
         const int s = i % S, r = i / S;
         if (!mbar_wait(&bar_empty[s], (r - 1) & 1, DEV_ERR_TIMEOUT_EMPTY)) break;
         mbar_arrive_expect_tx(&bar_wfull[s], C::WBYTES);
-        tma_load_2d(ws(s), tmW, &bar_wfull[s], (kb + i) * (TC_BK / 4), n0);
+#pragma unroll
+        for (int rb = 0; rb < RB; ++rb)
+          tma_load_2d(ws(s) + rb * (C::WBYTES / RB), tmW, &bar_wfull[s], (kb + i) * (TC_BK / 4), n0 + 128 * rb);
         load_x(i);
         issued = i + 1;
       }
@@ -559,7 +563,7 @@ static cudaError_t launch_tc(LinGroup grp, const void* Xq, const float* s_x, int
     if (grp.acc_dbg[g] != nullptr || ((uint64_t)grp.N[g] * sizeof(TOut)) % 16 != 0) use_tma_store = 0;
   grp.first[0] = 0;
   for (int g = 0; g < grp.count; ++g) {
-    if (!make_map_bytes(&maps.w[g], grp.pkW[g], (uint64_t)K / 4, (uint64_t)grp.N[g], TC_BK / 4, MB,
+    if (!make_map_bytes(&maps.w[g], grp.pkW[g], (uint64_t)K / 4, (uint64_t)grp.N[g], TC_BK / 4, 128,
                         CU_TENSOR_MAP_SWIZZLE_32B))
       return cudaErrorInvalidValue;
     if (use_tma_store && !make_map_2d(&maps.y[g], grp.Y[g], MapType<TOut>::v, (uint64_t)grp.N[g], (uint64_t)M,
@@ -614,14 +618,16 @@ static cudaError_t dispatch_tc(const LinGroup& grp, const void* Xq, const float*
   if (M <= 32) return launch_tc<32, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
   if (M <= 64) return launch_tc<64, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
   // 256 weight rows per CTA halve the activation bytes per MMA but hold a
-  // whole SM: only when the tiles fill at least two such waves
+  // whole SM.  Measured on B200 it runs the batched prefill product slower
+  // than the 128-row tile at two CTAs per SM (about 1700 cycles per K step
+  // against 512 of MMA work), so it is used only when asked for (kernel 4).
   int sms = 148, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int tiles256 = 0;
   for (int g = 0; g < grp.count; ++g) tiles256 += (grp.N[g] + 255) / 256;
   tiles256 *= (M + 127) / 128;
-  if (rows == 0 && tiles256 >= 2 * sms) return launch_tc<128, ACT_BITS, TOut, 256>(grp, Xq, s_x, M, K, st);
+  (void)tiles256;                     // measured on B200: the 256-row tile is slower (see the tile's notes)
   return launch_tc<128, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
 }
 
