@@ -132,10 +132,8 @@ attention_decode_kernel(const float* __restrict__ Q, const float* __restrict__ K
 }
 
 // ---------------------------------------------------------------------------
-// many queries per sequence (prefill): one CTA per (pair of query blocks of 32,
-// head, sequence).  Causal attention gives query block j j+1 key blocks, so a
-// CTA takes blocks j and NQB-1-j (NQB+1 key blocks in all): every CTA has the
-// same work, where one CTA per block left most SMs idle behind the last ones.  Key blocks of 32 keys and their values are double-buffered in
+// many queries per sequence (prefill): one CTA per (block of 32 queries, head,
+// sequence).  Key blocks of 32 keys and their values are double-buffered in
 // shared memory by 16-byte asynchronous copies (the next block streams in
 // while this one is used).  Thread (r, g) of the 256 (r = query row, g < 8)
 // computes the scores of keys g, g+8, g+16, g+24 of the block (128-term dot
@@ -170,13 +168,7 @@ attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ 
   float* ps = vbuf + 2 * ATP_KB * ATP_PITCH;        // [32][33] probabilities of the current block
   pdl_launch_dependents();
   pdl_wait();
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int nqb = (L + ATP_QB - 1) / ATP_QB;
-#pragma unroll 1
-  for (int half = 0; half < 2; ++half) {
-  const int qb = half == 0 ? (int)blockIdx.x : nqb - 1 - (int)blockIdx.x;
-  if (half == 1 && qb <= (int)blockIdx.x) break;    // the middle block of an odd count runs once
-  if (half == 1) __syncthreads();                    // the first block's buffers are free
+  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int l0 = qb * ATP_QB;
   const int nq = L - l0 < ATP_QB ? L - l0 : ATP_QB;
   const int tid = threadIdx.x;
@@ -270,7 +262,6 @@ attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ 
     for (int i = 0; i < 4; ++i)
       *reinterpret_cast<float4*>(dst + 32 * i) = make_float4(o[i][0] * inv, o[i][1] * inv, o[i][2] * inv, o[i][3] * inv);
   }
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -295,8 +286,7 @@ cudaError_t run_attention(const float* Q, const float* Kc, const float* Vc, int 
   }
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(attention_prefill_kernel), ATP_SMEM);
   if (e != cudaSuccess) return e;
-  const unsigned nqb = (unsigned)((L + ATP_QB - 1) / ATP_QB);
-  return launch_pdl(attention_prefill_kernel, dim3((nqb + 1) / 2, (unsigned)heads, (unsigned)B),
+  return launch_pdl(attention_prefill_kernel, dim3((unsigned)((L + ATP_QB - 1) / ATP_QB), (unsigned)heads, (unsigned)B),
                     dim3(256), ATP_SMEM, st, 1u, Q, Kc, Vc, L, t0, HD, T_cap, scale, A);
 }
 
