@@ -523,8 +523,8 @@ hadamard_quant_i4_row_kernel(const TIn* __restrict__ X, const float* __restrict_
 // ---------------------------------------------------------------------------
 // ---------------------------------------------------------------------------
 // RMSNorm + Hadamard + int4, one token per CTA of T = K / 32 threads (K =
-// 4096, 8192 or 16384: W = log2(T / 32) = 2, 3 or 4 warp bits), 32 elements per
-// thread, for blocks of b = 2^L >= 1024.  The element index bits are handled in
+// 2048, 4096, 8192 or 16384: W = log2(T / 32) = 1 .. 4 warp bits), 32 elements
+// per thread, for blocks of b = 2^L >= 1024.  The element index bits are handled in
 // three groups, each while a thread holds all 32 elements the group's stages
 // pair up (stages always in the order stride 1, 2, ..., b/2):
 //   mapping A: thread t holds elements 32t .. 32t+31 (bits 0-4 in-thread):
@@ -575,7 +575,7 @@ BN_DEV void fwht32(float (&v)[32]) {
 // one, so the load latency is hidden.  A thread reads back only what it copied
 // itself, so the staging needs no barrier.
 template <typename TIn, int L, int W, int PRE, bool PF>
-__global__ void __launch_bounds__(32 << W, (32 << W) == 256 ? 4 : (32 << W) == 128 ? 8 : 2)
+__global__ void __launch_bounds__(32 << W, (32 << W) == 512 ? 2 : (32 << W) == 256 ? 4 : (32 << W) == 128 ? 8 : 16)
 hadamard_quant_i4_split_kernel(const TIn* __restrict__ X, const float* __restrict__ B, int M, int K,
                                const float* __restrict__ gamma, float eps, float cb, uint8_t* __restrict__ Xq4,
                                float* __restrict__ s_x, float* __restrict__ T_dbg) {
@@ -880,22 +880,13 @@ static cudaError_t launch_h4(const void* X, const float* B, int M, int K, const 
                         cbw, Xq4, s_x, T_dbg);
     }
   }
-  // Few tokens: the register kernel would leave most SMs idle; one CTA per token instead.
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if ((M + TPB - 1) / TPB < 2 * sms) {
-    auto rk = hadamard_quant_i4_row_kernel<TIn, L, PRE>;
-    const size_t rsmem = (size_t)(K + K / 8) * sizeof(float);
-    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(rk), rsmem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(rk, dim3(M), dim3(HR_THREADS), rsmem, st, 1u, static_cast<const TIn*>(X), B, K, gamma, eps, cb,
-                      Xq4, s_x, T_dbg);
-  }
-  // Many tokens, K = 4096 / 8192 / 16384, blocks of 1024 or more: one token per
-  // CTA of K / 32 threads, 32 elements per thread.
+  // K = 2048 / 4096 / 8192 / 16384, blocks of 1024 or more: one token per CTA
+  // of K / 32 threads, 32 elements per thread.
   if constexpr (L >= 10) {
-    const int W = K == 4096 ? 2 : K == 8192 ? 3 : K == 16384 ? 4 : 0;
+    const int W = K == 2048 ? 1 : K == 4096 ? 2 : K == 8192 ? 3 : K == 16384 ? 4 : 0;
     if (W != 0 && L <= 10 + W) {
       constexpr bool PF = sizeof(TIn) == 2 && PRE == PRE_NONE;
       const size_t ssmem = (size_t)(K + K / 32) * sizeof(float) + (size_t)K / 2 + (PF ? (size_t)K * 2 : 0);
@@ -911,11 +902,21 @@ static cudaError_t launch_h4(const void* X, const float* B, int M, int K, const 
                         gamma, eps, cb, Xq4, s_x, T_dbg);                                                   \
     }                                                                                                       \
   } while (0)
+      if (W == 1) BN_HS(1);
       if (W == 2) BN_HS(2);
       if (W == 3) BN_HS(3);
       if (W == 4) BN_HS(4);
 #undef BN_HS
     }
+  }
+  // Few tokens: the register kernel would leave most SMs idle; one CTA per token instead.
+  if ((M + TPB - 1) / TPB < 2 * sms) {
+    auto rk = hadamard_quant_i4_row_kernel<TIn, L, PRE>;
+    const size_t rsmem = (size_t)(K + K / 8) * sizeof(float);
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(rk), rsmem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(rk, dim3(M), dim3(HR_THREADS), rsmem, st, 1u, static_cast<const TIn*>(X), B, K, gamma, eps, cb,
+                      Xq4, s_x, T_dbg);
   }
   const size_t smem = (size_t)TPB * ((K + 2 * (K >> 7) + 3) & ~3) * sizeof(float) + (size_t)TPB * 4 * sizeof(float);
   auto kern = hadamard_quant_i4_kernel<TIn, L, PRE>;
