@@ -569,54 +569,21 @@ BN_DEV void fwht32(float (&v)[32]) {
   }
 }
 
-// PF (bf16 input, no prologue): the CTA is persistent and loops over tokens
-// m = blockIdx.x, + gridDim.x, ...; each thread copies its 64 input bytes of
-// the next token into shared memory (cp.async) while it works on the current
-// one, so the load latency is hidden.  A thread reads back only what it copied
-// itself, so the staging needs no barrier.
-template <typename TIn, int L, int W, int PRE, bool PF>
+template <typename TIn, int L, int W, int PRE>
 __global__ void __launch_bounds__(32 << W, (32 << W) == 512 ? 2 : (32 << W) == 256 ? 4 : (32 << W) == 128 ? 8 : 16)
-hadamard_quant_i4_split_kernel(const TIn* __restrict__ X, const float* __restrict__ B, int M, int K,
+hadamard_quant_i4_split_kernel(const TIn* __restrict__ X, const float* __restrict__ B, int K,
                                const float* __restrict__ gamma, float eps, float cb, uint8_t* __restrict__ Xq4,
                                float* __restrict__ s_x, float* __restrict__ T_dbg) {
   constexpr int T = 32 << W, NW = 1 << W, LOW = 5 - W;
   static_assert(L >= 10 && L <= 10 + W, "block of 2^10 .. K");
-  static_assert(!PF || (sizeof(TIn) == 2 && PRE == PRE_NONE), "staging of bf16 rows");
   extern __shared__ float hs[];
   uint8_t* bytes = reinterpret_cast<uint8_t*>(hs + (K + K / 32));
-  uint8_t* stage = bytes + K / 2;                  // PF: this thread's 64 bytes at 64 t
   __shared__ float red[NW];
   pdl_launch_dependents();
   pdl_wait();                                // X may come from, and Xq4 may still be read by, the previous kernel
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  if constexpr (PF) {
-    if ((int)blockIdx.x < M) {
-      const uint8_t* src = reinterpret_cast<const uint8_t*>(X + (size_t)blockIdx.x * K + (size_t)t * 32);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) cp_async_16(smem_u32(stage + 64 * t + 16 * q), src + 16 * q, 16u);
-    }
-    cp_async_commit();
-  }
-#pragma unroll 1
-  for (int m = blockIdx.x; m < M; m += PF ? gridDim.x : M) {
+  const int m = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   float v[32];
-  if constexpr (PF) {
-    cp_async_wait_all();                       // this thread's bytes of token m
-    const uint4* mine = reinterpret_cast<const uint4*>(stage + 64 * t);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 u = mine[q];
-      v[8 * q + 0] = bf16lo(u.x); v[8 * q + 1] = bf16hi(u.x); v[8 * q + 2] = bf16lo(u.y); v[8 * q + 3] = bf16hi(u.y);
-      v[8 * q + 4] = bf16lo(u.z); v[8 * q + 5] = bf16hi(u.z); v[8 * q + 6] = bf16lo(u.w); v[8 * q + 7] = bf16hi(u.w);
-    }
-    const int mn = m + gridDim.x;              // the next token's bytes stream in meanwhile
-    if (mn < M) {
-      const uint8_t* src = reinterpret_cast<const uint8_t*>(X + (size_t)mn * K + (size_t)t * 32);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) cp_async_16(smem_u32(stage + 64 * t + 16 * q), src + 16 * q, 16u);
-    }
-    cp_async_commit();
-  } else {
+  {
     const size_t off = (size_t)m * K + (size_t)t * 32;
     constexpr int E = InVec<TIn>::E;
 #pragma unroll
@@ -635,7 +602,6 @@ hadamard_quant_i4_split_kernel(const TIn* __restrict__ X, const float* __restric
     for (int c = 0; c < 16; ++c) sq[c] = __fadd_rn(__fmul_rn(v[2 * c], v[2 * c]), __fmul_rn(v[2 * c + 1], v[2 * c + 1]));
     part = warp_tree_sum(tree_sum<16>(sq));
   }
-  if (PF) __syncthreads();                   // the previous token's codes have left shared memory
   if (lane == 0) red[warp] = part;
   __syncthreads();
   float w[NW];
@@ -700,7 +666,6 @@ hadamard_quant_i4_split_kernel(const TIn* __restrict__ X, const float* __restric
   uint4* dst = reinterpret_cast<uint4*>(Xq4 + (size_t)m * (K / 2));
   for (int q = t; q < K / 32; q += T) dst[q] = src[q];
   if (t == 0) s_x[m] = sc;
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -887,18 +852,18 @@ static cudaError_t launch_h4(const void* X, const float* B, int M, int K, const 
   // of K / 32 threads, 32 elements per thread.
   if constexpr (L >= 10) {
     const int W = K == 2048 ? 1 : K == 4096 ? 2 : K == 8192 ? 3 : K == 16384 ? 4 : 0;
-    if (W != 0 && L <= 10 + W) {
-      constexpr bool PF = sizeof(TIn) == 2 && PRE == PRE_NONE;
-      const size_t ssmem = (size_t)(K + K / 32) * sizeof(float) + (size_t)K / 2 + (PF ? (size_t)K * 2 : 0);
-      // persistent CTAs (PF): as many as can be resident, each looping over tokens
-      const unsigned grid = PF ? (unsigned)(M < 4 * sms ? M : 4 * sms) : (unsigned)M;
+    // 64 or 128 threads per token only with enough tokens to fill the SMs (a few
+    // tokens go faster on the one-CTA-per-token kernel's 256 threads)
+    if (W != 0 && L <= 10 + W && (W >= 3 || M >= sms)) {
+      const size_t ssmem = (size_t)(K + K / 32) * sizeof(float) + (size_t)K / 2;
+      const unsigned grid = (unsigned)M;
 #define BN_HS(WW)                                                                                           \
   do {                                                                                                      \
     if constexpr (L <= 10 + WW) {                                                                           \
-      auto sk = hadamard_quant_i4_split_kernel<TIn, L, WW, PRE, PF>;                                        \
+      auto sk = hadamard_quant_i4_split_kernel<TIn, L, WW, PRE>;                                            \
       cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(sk), ssmem);                          \
       if (e != cudaSuccess) return e;                                                                       \
-      return launch_pdl(sk, dim3(grid), dim3(32 << WW), ssmem, st, 1u, static_cast<const TIn*>(X), B, M, K, \
+      return launch_pdl(sk, dim3(grid), dim3(32 << WW), ssmem, st, 1u, static_cast<const TIn*>(X), B, K,    \
                         gamma, eps, cb, Xq4, s_x, T_dbg);                                                   \
     }                                                                                                       \
   } while (0)

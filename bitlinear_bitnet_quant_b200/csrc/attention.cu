@@ -132,23 +132,25 @@ attention_decode_kernel(const float* __restrict__ Q, const float* __restrict__ K
 }
 
 // ---------------------------------------------------------------------------
-// many queries per sequence (prefill): one CTA per (block of 32 queries, head,
-// sequence).  Key blocks of 32 keys and their values are double-buffered in
-// shared memory by 16-byte asynchronous copies (the next block streams in
-// while this one is used).  Thread (r, g) of the 256 (r = query row, g < 8)
-// computes the scores of keys g, g+8, g+16, g+24 of the block (128-term dot
-// products from float4 reads that are broadcasts or conflict-free), updates
-// its row's running softmax with the 8 threads of the row (shuffles), then
-// accumulates P V for dimensions 32 i + 4 g .. + 3, i < 4.
+// many queries per sequence (prefill): one CTA of 128 threads per (block of 64
+// queries, head, sequence).  Key blocks of 32 keys and their values are double-
+// buffered in shared memory by 16-byte asynchronous copies.  Register blocking:
+// thread (q, k) (q < 16, k < 8) computes the scores of queries q + 16 r and keys
+// k + 8 c (r, c < 4) as outer products of float4 reads (8 reads per 64 multiply-
+// adds, all broadcast or conflict-free), keeps the running softmax of its four
+// query rows with the row's 8 lanes (shuffles), and accumulates P V for its four
+// queries and 16 dimensions 32 i + 4 k .. + 3 (i < 4).
 // ---------------------------------------------------------------------------
-constexpr int ATP_QB = 32;
+constexpr int ATP_QB = 64;
 constexpr int ATP_KB = 32;
+constexpr int ATP_THREADS = 128;
 constexpr int ATP_PITCH = ATT_D + 4;               // floats per staged row
-constexpr size_t ATP_SMEM = (size_t)(ATP_QB + 4 * ATP_KB) * ATP_PITCH * 4 + (size_t)ATP_QB * (ATP_KB + 1) * 4;
+constexpr int ATP_PPITCH = ATP_QB + 4;             // probabilities, [key][query]
+constexpr size_t ATP_SMEM = (size_t)(ATP_QB + 4 * ATP_KB) * ATP_PITCH * 4 + (size_t)ATP_KB * ATP_PPITCH * 4;
 
 // 16-byte asynchronous copies of key/value rows j0 .. j0+31 (rows past nk zero).
 BN_DEV void att_stage_kv(const float* kbase, const float* vbase, int HD, int j0, int nk, float* ks, float* vs) {
-  for (int e = threadIdx.x; e < ATP_KB * (ATT_D / 4); e += 256) {
+  for (int e = threadIdx.x; e < ATP_KB * (ATT_D / 4); e += ATP_THREADS) {
     const int rr = e / (ATT_D / 4), cc = e - rr * (ATT_D / 4);
     const bool in = rr < nk;
     const size_t off = in ? (size_t)(j0 + rr) * HD + 4 * cc : 0;
@@ -158,39 +160,43 @@ BN_DEV void att_stage_kv(const float* kbase, const float* vbase, int HD, int j0,
   cp_async_commit();
 }
 
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(ATP_THREADS, 2)
 attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ Kc, const float* __restrict__ Vc,
                          int L, int t0, int HD, int T_cap, float scale, float* __restrict__ A) {
   extern __shared__ float atp[];
-  float* qs = atp;                                  // [32][PITCH]
+  float* qs = atp;                                  // [64][PITCH]
   float* kbuf = qs + ATP_QB * ATP_PITCH;            // [2][32][PITCH]
   float* vbuf = kbuf + 2 * ATP_KB * ATP_PITCH;      // [2][32][PITCH]
-  float* ps = vbuf + 2 * ATP_KB * ATP_PITCH;        // [32][33] probabilities of the current block
+  float* pt = vbuf + 2 * ATP_KB * ATP_PITCH;        // [32][PPITCH] probabilities of the current block
   pdl_launch_dependents();
   pdl_wait();
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int l0 = qb * ATP_QB;
   const int nq = L - l0 < ATP_QB ? L - l0 : ATP_QB;
   const int tid = threadIdx.x;
-  const int row = tid >> 3, g = tid & 7;
+  const int tq = tid >> 3, tk = tid & 7;
   const float* kbase = Kc + (size_t)b * T_cap * HD + h * ATT_D;
   const float* vbase = Vc + (size_t)b * T_cap * HD + h * ATT_D;
   const int kend = t0 + l0 + nq;                     // keys 0 .. kend-1 are needed by the block
   const int nblk = (kend + ATP_KB - 1) / ATP_KB;
   att_stage_kv(kbase, vbase, HD, 0, kend < ATP_KB ? kend : ATP_KB, kbuf, vbuf);
-  for (int e = tid; e < ATP_QB * (ATT_D / 4); e += 256) {
+  for (int e = tid; e < ATP_QB * (ATT_D / 4); e += ATP_THREADS) {
     const int rr = e / (ATT_D / 4), cc = e - rr * (ATT_D / 4);
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (rr < nq) v = *reinterpret_cast<const float4*>(Q + ((size_t)b * L + l0 + rr) * HD + h * ATT_D + 4 * cc);
     *reinterpret_cast<float4*>(qs + rr * ATP_PITCH + 4 * cc) = v;
   }
-  const int qpos = t0 + l0 + row;
-  float m = -INFINITY, sum = 0.f;
-  float o[4][4];
+  float m[4], sum[4];
+  float o[4][4][4];                                  // [query r][dimension group i][4]
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int r = 0; r < 4; ++r) {
+    m[r] = -INFINITY;
+    sum[r] = 0.f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) o[i][c] = 0.f;
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) o[r][i][c] = 0.f;
+  }
   for (int blk = 0; blk < nblk; ++blk) {
     const int j0 = blk * ATP_KB;
     const int nk = kend - j0 < ATP_KB ? kend - j0 : ATP_KB;
@@ -205,62 +211,86 @@ attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ 
     __syncthreads();                                 // this block's K, V (and the queries) are in place
     const float* ks = kbuf + (blk & 1) * ATP_KB * ATP_PITCH;
     const float* vs = vbuf + (blk & 1) * ATP_KB * ATP_PITCH;
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* qr = qs + row * ATP_PITCH;
-#pragma unroll 8
+    // ---- scores of queries tq + 16 r and keys tk + 8 c ----
+    float s[4][4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) s[r][c] = 0.f;
+#pragma unroll 4
     for (int dd = 0; dd < ATT_D; dd += 4) {
-      const float4 qv = *reinterpret_cast<const float4*>(qr + dd);
+      float4 qv[4], kv[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float4 kv = *reinterpret_cast<const float4*>(ks + (g + 8 * u) * ATP_PITCH + dd);
-        s[u] += qv.x * kv.x + qv.y * kv.y + qv.z * kv.z + qv.w * kv.w;
+      for (int r = 0; r < 4; ++r) qv[r] = *reinterpret_cast<const float4*>(qs + (tq + 16 * r) * ATP_PITCH + dd);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) kv[c] = *reinterpret_cast<const float4*>(ks + (tk + 8 * c) * ATP_PITCH + dd);
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          s[r][c] += qv[r].x * kv[c].x + qv[r].y * kv[c].y + qv[r].z * kv[c].z + qv[r].w * kv[c].w;
+    }
+    // ---- running softmax of the four query rows (the row's 8 lanes: xor 1, 2, 4) ----
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int qpos = t0 + l0 + tq + 16 * r;
+      float bm = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int jj = tk + 8 * c;
+        s[r][c] = (jj < nk && j0 + jj <= qpos) ? s[r][c] * scale : -INFINITY;
+        bm = fmaxf(bm, s[r][c]);
       }
+#pragma unroll
+      for (int off = 4; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+      const float mn = fmaxf(m[r], bm);
+      // a query row whose keys in this block are all masked keeps its state
+      const float corr = mn == -INFINITY ? 1.f : expf(m[r] - mn);
+      float psum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float p = s[r][c] == -INFINITY ? 0.f : expf(s[r][c] - mn);
+        pt[(tk + 8 * c) * ATP_PPITCH + tq + 16 * r] = p;
+        psum += p;
+      }
+#pragma unroll
+      for (int off = 4; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
+      sum[r] = sum[r] * corr + psum;
+      m[r] = mn;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) o[r][i][c] *= corr;
     }
-    float bm = -INFINITY;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int jj = g + 8 * u;
-      s[u] = (jj < nk && j0 + jj <= qpos) ? s[u] * scale : -INFINITY;
-      bm = fmaxf(bm, s[u]);
-    }
-#pragma unroll
-    for (int off = 4; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
-    const float mn = fmaxf(m, bm);
-    // a query row whose keys in this block are all masked keeps its state
-    const float corr = mn == -INFINITY ? 1.f : expf(m - mn);
-    float psum = 0.f;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float p = s[u] == -INFINITY ? 0.f : expf(s[u] - mn);
-      ps[row * (ATP_KB + 1) + g + 8 * u] = p;
-      psum += p;
-    }
-#pragma unroll
-    for (int off = 4; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
-    sum = sum * corr + psum;
-    m = mn;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) o[i][c] *= corr;
-    __syncwarp();                                    // the row's probabilities come from its 8 lanes
-    const float* pr = ps + row * (ATP_KB + 1);
+    __syncthreads();                                 // every row's probabilities are in place
+    // ---- P V: queries tq + 16 r, dimensions 32 i + 4 tk .. + 3 ----
+#pragma unroll 2
     for (int j = 0; j < nk; ++j) {
-      const float p = pr[j];
+      float p[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) p[r] = pt[j * ATP_PPITCH + tq + 16 * r];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float4 v = *reinterpret_cast<const float4*>(vs + j * ATP_PITCH + 32 * i + 4 * g);
-        o[i][0] += p * v.x; o[i][1] += p * v.y; o[i][2] += p * v.z; o[i][3] += p * v.w;
+        const float4 v = *reinterpret_cast<const float4*>(vs + j * ATP_PITCH + 32 * i + 4 * tk);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          o[r][i][0] += p[r] * v.x; o[r][i][1] += p[r] * v.y; o[r][i][2] += p[r] * v.z; o[r][i][3] += p[r] * v.w;
+        }
       }
     }
     __syncthreads();                                 // every thread is done with this block's buffers
   }
-  if (row < nq) {
-    const float inv = 1.0f / sum;
-    float* dst = A + ((size_t)b * L + l0 + row) * HD + h * ATT_D + 4 * g;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      *reinterpret_cast<float4*>(dst + 32 * i) = make_float4(o[i][0] * inv, o[i][1] * inv, o[i][2] * inv, o[i][3] * inv);
+  for (int r = 0; r < 4; ++r) {
+    const int row = tq + 16 * r;
+    if (row < nq) {
+      const float inv = 1.0f / sum[r];
+      float* dst = A + ((size_t)b * L + l0 + row) * HD + h * ATT_D + 4 * tk;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<float4*>(dst + 32 * i) =
+            make_float4(o[r][i][0] * inv, o[r][i][1] * inv, o[r][i][2] * inv, o[r][i][3] * inv);
+    }
   }
 }
 
@@ -287,7 +317,7 @@ cudaError_t run_attention(const float* Q, const float* Kc, const float* Vc, int 
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(attention_prefill_kernel), ATP_SMEM);
   if (e != cudaSuccess) return e;
   return launch_pdl(attention_prefill_kernel, dim3((unsigned)((L + ATP_QB - 1) / ATP_QB), (unsigned)heads, (unsigned)B),
-                    dim3(256), ATP_SMEM, st, 1u, Q, Kc, Vc, L, t0, HD, T_cap, scale, A);
+                    dim3(ATP_THREADS), ATP_SMEM, st, 1u, Q, Kc, Vc, L, t0, HD, T_cap, scale, A);
 }
 
 }  // namespace bitnet
