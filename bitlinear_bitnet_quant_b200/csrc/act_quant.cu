@@ -669,6 +669,163 @@ hadamard_quant_i4_split_kernel(const TIn* __restrict__ X, const float* __restric
 }
 
 // ---------------------------------------------------------------------------
+// RMSNorm + Hadamard + int4 for K = 8192 in one block of b = 8192 (the H-
+// BitLinear input of the 2048 x 8192 workload), one token per CTA of 256
+// threads, on packed fp32 pairs (add / sub / mul .f32x2: half the arithmetic
+// instructions of the scalar stages, the same roundings).  Every mapping keeps
+// element bit 0 inside a thread's 64-bit register pair, so a pair is the unit
+// of the stages that do not touch bit 0 and of the shared-memory traffic:
+//   mapping A: thread t holds elements 32t .. 32t+31 (bits 0-4 in-thread):
+//              the loads, the sum of squares, the norm, stage 0 (the one stage
+//              inside a pair, scalar) and stages 1-4 (packed);
+//   mapping B: in-thread bits 0 and 5-8, thread = bits 1-4 and 9-12: stages 5-8;
+//   mapping C: in-thread bits 0 and 9-12, thread = bits 1-8: stages 9-12, the
+//              normalisation c_b, the absmax and the codes (a pair is a byte).
+// The row sits in shared memory as 32-element lines whose 16-byte slots
+// (bits 2-4) are XOR-swizzled by bits 5-7: the mapping-A float4 stores and the
+// mapping-B/C float2 accesses are all conflict-free.  Every value is the one
+// the other Hadamard kernels produce.
+// ---------------------------------------------------------------------------
+constexpr int HP_K = 8192;
+constexpr int HP_T = 256;
+
+BN_DEV int hp_phys(int e) { return e ^ (((e >> 5) & 7) << 2); }
+
+// Butterflies on pairs: stages whose element bit is in-thread bit 1 + i of the
+// pair index's bit i, for pair-index strides 1, 2, 4, 8 (four stages).
+BN_DEV void fwht_pairs16(uint64_t (&p)[16]) {
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if ((j & h) == 0) {
+        const uint64_t a = p[j], b = p[j + h];
+        p[j] = f2_add(a, b);
+        p[j + h] = f2_sub(a, b);
+      }
+    }
+  }
+}
+
+template <typename TIn, int PRE>
+__global__ void __launch_bounds__(HP_T, 4)
+hadamard_quant_i4_pair_kernel(const TIn* __restrict__ X, const float* __restrict__ B,
+                              const float* __restrict__ gamma, float eps, float cb, uint8_t* __restrict__ Xq4,
+                              float* __restrict__ s_x, float* __restrict__ T_dbg) {
+  constexpr int NW = HP_T / 32;
+  __shared__ __align__(16) float hs[HP_K];
+  __shared__ float red[NW];
+  pdl_launch_dependents();
+  pdl_wait();                                // X may come from, and Xq4 may still be read by, the previous kernel
+  const int m = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  float v[32];
+  {
+    const size_t off = (size_t)m * HP_K + (size_t)t * 32;
+    constexpr int E = InVec<TIn>::E;
+#pragma unroll
+    for (int q = 0; q < 32 / E; ++q) {
+      float tmp[E];
+      load_chunk<PRE, TIn, E>(X + off + q * E, B + off + q * E, nullptr, tmp);
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[q * E + e] = tmp[e];
+    }
+  }
+  // ---- sum of squares: in-thread tree (first level fused), lanes, warps in order ----
+  {
+    float sq[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      float a, b;
+      f2_unpack(f2_mul(f2_pack(v[2 * c], v[2 * c + 1]), f2_pack(v[2 * c], v[2 * c + 1])), a, b);
+      sq[c] = __fadd_rn(a, b);
+    }
+    const float part = warp_tree_sum(tree_sum<16>(sq));
+    if (lane == 0) red[warp] = part;
+  }
+  __syncthreads();
+  float w[NW];
+#pragma unroll
+  for (int i = 0; i < NW; ++i) w[i] = red[i];
+  const float ss = tree_sum<NW>(w);
+  const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)HP_K), eps)));
+  // ---- norm, stage 0 (inside each pair), stages 1-4 (mapping A) ----
+  uint64_t p[16];
+  {
+    const uint64_t rr = f2_pack(r, r);
+    const float* gp = gamma + (size_t)t * 32;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      uint64_t x = f2_mul(f2_pack(v[2 * j], v[2 * j + 1]), rr);
+      if (gamma != nullptr) x = f2_mul(x, f2_pack(__ldg(gp + 2 * j), __ldg(gp + 2 * j + 1)));
+      float a, b;
+      f2_unpack(x, a, b);
+      p[j] = f2_pack(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+  }
+  fwht_pairs16(p);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int e = 32 * t + 4 * q;
+    *reinterpret_cast<ulonglong2*>(hs + hp_phys(e)) = make_ulonglong2(p[2 * q], p[2 * q + 1]);
+  }
+  __syncthreads();
+  // ---- stages 5-8 (mapping B: pair j holds elements (t & 15) << 1 | j << 5 | (t >> 4) << 9, +1) ----
+  const int eb = ((t & 15) << 1) | ((t >> 4) << 9);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) p[j] = *reinterpret_cast<const uint64_t*>(hs + hp_phys(eb | (j << 5)));
+  fwht_pairs16(p);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) *reinterpret_cast<uint64_t*>(hs + hp_phys(eb | (j << 5))) = p[j];
+  __syncthreads();
+  // ---- stages 9-12 (mapping C: pair j holds elements t << 1 | j << 9, +1) ----
+#pragma unroll
+  for (int j = 0; j < 16; ++j) p[j] = *reinterpret_cast<const uint64_t*>(hs + hp_phys((t << 1) | (j << 9)));
+  fwht_pairs16(p);
+  float amax = 0.f;
+  {
+    const uint64_t cc = f2_pack(cb, cb);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      p[j] = f2_mul(p[j], cc);
+      float a, b;
+      f2_unpack(p[j], a, b);
+      amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+    }
+  }
+  amax = warp_max(amax);
+  __syncthreads();                           // every thread has read red[] (the sum of squares)
+  if (lane == 0) red[warp] = amax;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < NW; ++i) amax = fmaxf(amax, red[i]);
+  const float sc = __fdiv_rn(7.0f, fmaxf(amax, 1e-5f));
+  if (T_dbg != nullptr) {
+    float* dst = T_dbg + (size_t)m * HP_K;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      float a, b;
+      f2_unpack(p[j], a, b);
+      *reinterpret_cast<float2*>(dst + ((t << 1) | (j << 9))) = make_float2(a, b);
+    }
+  }
+  // ---- codes: pair j is byte t + 256 j (the even element in the low nibble) ----
+  {
+    // The products are packed; the rounding additions stay scalar: a packed
+    // multiply followed by a packed add may be fused into one packed fma,
+    // which would round t * s + 1.5 * 2^23 once instead of twice.
+    const uint64_t ss2 = f2_pack(sc, sc);
+    uint8_t* dst = Xq4 + (size_t)m * (HP_K / 2) + t;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      float a, b;
+      f2_unpack(f2_mul(p[j], ss2), a, b);
+      dst[256 * j] = (uint8_t)pair_nibbles(rint_low_bits(a), rint_low_bits(b));
+    }
+  }
+  if (t == 0) s_x[m] = sc;
+}
+
+// ---------------------------------------------------------------------------
 // RMSNorm + Hadamard + int4 for blocks of b = 2^L <= 512 elements, one warp per
 // block and one CTA per token (K / b <= 32 warps; e.g. K = 5632 in 11 blocks of
 // 512, the down projection's input).  Lane j holds the E = b / 32 consecutive
@@ -848,6 +1005,13 @@ static cudaError_t launch_h4(const void* X, const float* B, int M, int K, const 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // K = 8192 in one block: the packed-pair kernel.
+  if constexpr (L == 13) {
+    if (K == HP_K) {
+      return launch_pdl(hadamard_quant_i4_pair_kernel<TIn, PRE>, dim3((unsigned)M), dim3(HP_T), 0, st, 1u,
+                        static_cast<const TIn*>(X), B, gamma, eps, cb, Xq4, s_x, T_dbg);
+    }
+  }
   // K = 2048 / 4096 / 8192 / 16384, blocks of 1024 or more: one token per CTA
   // of K / 32 threads, 32 elements per thread.
   if constexpr (L >= 10) {

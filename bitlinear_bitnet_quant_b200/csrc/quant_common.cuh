@@ -66,4 +66,32 @@ BN_DEV uint32_t pair_nibbles(uint32_t lo, uint32_t hi) {
   return r;
 }
 
+// Two fp32 values in one 64-bit register and the sm_100 packed arithmetic on
+// them (add / sub / mul .rn.f32x2): each half is rounded exactly as the scalar
+// __fadd_rn / __fsub_rn / __fmul_rn of the same operands, so a packed stage
+// gives the scalar stage's values at half the instructions.  A packed multiply
+// whose result feeds a packed add can be contracted into a packed fma (one
+// rounding): keep an add that must see the rounded product scalar.
+BN_DEV uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+BN_DEV void f2_unpack(uint64_t r, float& lo, float& hi) { asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r)); }
+BN_DEV uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+BN_DEV uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+BN_DEV uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 }  // namespace bitnet

@@ -181,10 +181,11 @@ def test_hadamard_quant_many_tokens(M, K, b, dtype):
 
 @pytest.mark.parametrize("M,K,b,dtype,use_gamma", [(640, 4096, 0, "bf16", False), (600, 8192, 1024, "f32", False),
                                                    (700, 16384, 8192, "bf16", True), (620, 8192, 0, "f32", True),
-                                                   (900, 4096, 2048, "f32", False)])
+                                                   (900, 4096, 2048, "f32", False), (300, 8192, 0, "bf16", True)])
 def test_hadamard_quant_split_kernel(M, K, b, dtype, use_gamma):
     """Many tokens at K = 4096 / 8192 / 16384 with blocks of 1024 or more: the
-    kernel that spreads a token over K/32 threads (three index-bit groups)."""
+    kernels that spread a token over K/32 threads (three index-bit groups;
+    packed fp32 pairs for one block of 8192)."""
     rng = np.random.default_rng(M + K + b)
     x = wl.add_channel_outliers(rng, wl.student_t(rng, (M, K)), 0.005, 50.0)
     x[0] = 0
@@ -617,7 +618,8 @@ def test_add_quant_act(M, K, use_gamma):
     assert np.array_equal(host(q), q_o)
 
 
-@pytest.mark.parametrize("M,K,b", [(3, 5632, 0), (32, 5632, 0), (4, 2048, 0), (7, 8192, 1024), (2, 1024, 32)])
+@pytest.mark.parametrize("M,K,b", [(3, 5632, 0), (32, 5632, 0), (4, 2048, 0), (7, 8192, 1024), (2, 1024, 32),
+                                   (5, 8192, 0)])
 def test_glu_hadamard_quant_act(M, K, b):
     """Squared-ReLU gated unit folded into the Hadamard int4 quantiser: codes
     and scales equal bitnet_relu2_glu followed by bitnet_hadamard_quant_act."""
