@@ -132,25 +132,34 @@ attention_decode_kernel(const float* __restrict__ Q, const float* __restrict__ K
 }
 
 // ---------------------------------------------------------------------------
-// many queries per sequence (prefill): one CTA of 128 threads per (block of 64
-// queries, head, sequence).  Key blocks of 32 keys and their values are double-
-// buffered in shared memory by 16-byte asynchronous copies.  Register blocking:
-// thread (q, k) (q < 16, k < 8) computes the scores of queries q + 16 r and keys
-// k + 8 c (r, c < 4) as outer products of float4 reads (8 reads per 64 multiply-
-// adds, all broadcast or conflict-free), keeps the running softmax of its four
-// query rows with the row's 8 lanes (shuffles), and accumulates P V for its four
-// queries and 16 dimensions 32 i + 4 k .. + 3 (i < 4).
+// many queries per sequence (prefill): one CTA of 256 threads per (block of 64
+// queries, head, sequence), as two key groups of 128 threads: group g takes
+// the key blocks g, g + 2, g + 4, ... of 32 keys, each with its own double-
+// buffered keys and values (16-byte asynchronous copies) and its own running
+// softmax; the two partial softmaxes are merged at the end.  Register
+// blocking inside a group: thread (q, k) (q < 16, k < 8) computes the scores
+// of queries q + 16 r and keys k + 8 c (r, c < 4) as outer products of float4
+// reads (8 reads per 64 multiply-adds, all broadcast or conflict-free), keeps
+// the running softmax of its four query rows with the row's 8 lanes
+// (shuffles), and accumulates P V for its four queries and 16 dimensions
+// 32 i + 4 k .. + 3 (i < 4).
 // ---------------------------------------------------------------------------
 constexpr int ATP_QB = 64;
 constexpr int ATP_KB = 32;
-constexpr int ATP_THREADS = 128;
+constexpr int ATP_GT = 128;                        // threads per key group
+constexpr int ATP_G = 2;                           // key groups per CTA
+constexpr int ATP_THREADS = ATP_GT * ATP_G;
 constexpr int ATP_PITCH = ATT_D + 4;               // floats per staged row
 constexpr int ATP_PPITCH = ATP_QB + 4;             // probabilities, [key][query]
-constexpr size_t ATP_SMEM = (size_t)(ATP_QB + 4 * ATP_KB) * ATP_PITCH * 4 + (size_t)ATP_KB * ATP_PPITCH * 4;
+constexpr int ATP_GFLOATS = 4 * ATP_KB * ATP_PITCH + ATP_KB * ATP_PPITCH;   // a group's keys, values, probabilities
+constexpr size_t ATP_SMEM = ((size_t)ATP_QB * ATP_PITCH + (size_t)ATP_G * ATP_GFLOATS) * 4;
+static_assert(ATP_GT * (8 + 64) <= 4 * ATP_KB * ATP_PITCH, "a group's softmax state fits its key/value buffers");
 
-// 16-byte asynchronous copies of key/value rows j0 .. j0+31 (rows past nk zero).
-BN_DEV void att_stage_kv(const float* kbase, const float* vbase, int HD, int j0, int nk, float* ks, float* vs) {
-  for (int e = threadIdx.x; e < ATP_KB * (ATT_D / 4); e += ATP_THREADS) {
+// 16-byte asynchronous copies of key/value rows j0 .. j0+31 (rows past nk
+// zero) by the 128 threads of one key group (gt = thread inside the group).
+BN_DEV void att_stage_kv(const float* kbase, const float* vbase, int HD, int j0, int nk, float* ks, float* vs,
+                         int gt) {
+  for (int e = gt; e < ATP_KB * (ATT_D / 4); e += ATP_GT) {
     const int rr = e / (ATT_D / 4), cc = e - rr * (ATT_D / 4);
     const bool in = rr < nk;
     const size_t off = in ? (size_t)(j0 + rr) * HD + 4 * cc : 0;
@@ -160,12 +169,17 @@ BN_DEV void att_stage_kv(const float* kbase, const float* vbase, int HD, int j0,
   cp_async_commit();
 }
 
-__global__ void __launch_bounds__(ATP_THREADS, 2)
+// Barrier of one key group's 128 threads (barrier 1 + g).
+BN_DEV void att_group_sync(int g) { asm volatile("bar.sync %0, %1;" :: "r"(1 + g), "r"(ATP_GT) : "memory"); }
+
+__global__ void __launch_bounds__(ATP_THREADS, 1)
 attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ Kc, const float* __restrict__ Vc,
                          int L, int t0, int HD, int T_cap, float scale, float* __restrict__ A) {
   extern __shared__ float atp[];
+  const int tid = threadIdx.x;
+  const int g = tid / ATP_GT, gt = tid - g * ATP_GT;
   float* qs = atp;                                  // [64][PITCH]
-  float* kbuf = qs + ATP_QB * ATP_PITCH;            // [2][32][PITCH]
+  float* kbuf = qs + ATP_QB * ATP_PITCH + g * ATP_GFLOATS;   // [2][32][PITCH] of this group
   float* vbuf = kbuf + 2 * ATP_KB * ATP_PITCH;      // [2][32][PITCH]
   float* pt = vbuf + 2 * ATP_KB * ATP_PITCH;        // [32][PPITCH] probabilities of the current block
   pdl_launch_dependents();
@@ -173,19 +187,22 @@ attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ 
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int l0 = qb * ATP_QB;
   const int nq = L - l0 < ATP_QB ? L - l0 : ATP_QB;
-  const int tid = threadIdx.x;
-  const int tq = tid >> 3, tk = tid & 7;
+  const int tq = gt >> 3, tk = gt & 7;
   const float* kbase = Kc + (size_t)b * T_cap * HD + h * ATT_D;
   const float* vbase = Vc + (size_t)b * T_cap * HD + h * ATT_D;
   const int kend = t0 + l0 + nq;                     // keys 0 .. kend-1 are needed by the block
   const int nblk = (kend + ATP_KB - 1) / ATP_KB;
-  att_stage_kv(kbase, vbase, HD, 0, kend < ATP_KB ? kend : ATP_KB, kbuf, vbuf);
+  if (g < nblk) {
+    const int j0 = g * ATP_KB;
+    att_stage_kv(kbase, vbase, HD, j0, kend - j0 < ATP_KB ? kend - j0 : ATP_KB, kbuf, vbuf, gt);
+  }
   for (int e = tid; e < ATP_QB * (ATT_D / 4); e += ATP_THREADS) {
     const int rr = e / (ATT_D / 4), cc = e - rr * (ATT_D / 4);
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (rr < nq) v = *reinterpret_cast<const float4*>(Q + ((size_t)b * L + l0 + rr) * HD + h * ATT_D + 4 * cc);
     *reinterpret_cast<float4*>(qs + rr * ATP_PITCH + 4 * cc) = v;
   }
+  __syncthreads();                                   // the queries are in place for both groups
   float m[4], sum[4];
   float o[4][4][4];                                  // [query r][dimension group i][4]
 #pragma unroll
@@ -197,20 +214,20 @@ attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ 
 #pragma unroll
       for (int c = 0; c < 4; ++c) o[r][i][c] = 0.f;
   }
-  for (int blk = 0; blk < nblk; ++blk) {
+  for (int blk = g, it = 0; blk < nblk; blk += ATP_G, ++it) {
     const int j0 = blk * ATP_KB;
     const int nk = kend - j0 < ATP_KB ? kend - j0 : ATP_KB;
-    if (blk + 1 < nblk) {
-      const int j1 = j0 + ATP_KB;
+    if (blk + ATP_G < nblk) {
+      const int j1 = j0 + ATP_G * ATP_KB;
       att_stage_kv(kbase, vbase, HD, j1, kend - j1 < ATP_KB ? kend - j1 : ATP_KB,
-                   kbuf + ((blk + 1) & 1) * ATP_KB * ATP_PITCH, vbuf + ((blk + 1) & 1) * ATP_KB * ATP_PITCH);
+                   kbuf + ((it + 1) & 1) * ATP_KB * ATP_PITCH, vbuf + ((it + 1) & 1) * ATP_KB * ATP_PITCH, gt);
       asm volatile("cp.async.wait_group 1;" ::: "memory");
     } else {
       cp_async_wait_all();
     }
-    __syncthreads();                                 // this block's K, V (and the queries) are in place
-    const float* ks = kbuf + (blk & 1) * ATP_KB * ATP_PITCH;
-    const float* vs = vbuf + (blk & 1) * ATP_KB * ATP_PITCH;
+    att_group_sync(g);                               // this block's K and V are in place
+    const float* ks = kbuf + (it & 1) * ATP_KB * ATP_PITCH;
+    const float* vs = vbuf + (it & 1) * ATP_KB * ATP_PITCH;
     // ---- scores of queries tq + 16 r and keys tk + 8 c ----
     float s[4][4];
 #pragma unroll
@@ -262,7 +279,7 @@ attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ 
 #pragma unroll
         for (int c = 0; c < 4; ++c) o[r][i][c] *= corr;
     }
-    __syncthreads();                                 // every row's probabilities are in place
+    att_group_sync(g);                               // every row's probabilities are in place
     // ---- P V: queries tq + 16 r, dimensions 32 i + 4 tk .. + 3 ----
 #pragma unroll 2
     for (int j = 0; j < nk; ++j) {
@@ -278,18 +295,43 @@ attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ 
         }
       }
     }
-    __syncthreads();                                 // every thread is done with this block's buffers
+    att_group_sync(g);                               // every thread of the group is done with this block's buffers
   }
+  // ---- merge: group 1 hands its running max, sum and output to the same thread of group 0 ----
+  float* xch = atp + ATP_QB * ATP_PITCH + ATP_GFLOATS;   // group 1's key/value buffers (no copy in flight)
+  if (g == 1) {
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int row = tq + 16 * r;
-    if (row < nq) {
-      const float inv = 1.0f / sum[r];
-      float* dst = A + ((size_t)b * L + l0 + row) * HD + h * ATT_D + 4 * tk;
+    for (int r = 0; r < 4; ++r) {
+      xch[(8 * r) * ATP_GT + gt] = m[r];
+      xch[(8 * r + 1) * ATP_GT + gt] = sum[r];
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<float4*>(dst + 32 * i) =
-            make_float4(o[r][i][0] * inv, o[r][i][1] * inv, o[r][i][2] * inv, o[r][i][3] * inv);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) xch[(32 + 16 * r + 4 * i + c) * ATP_GT + gt] = o[r][i][c];
+  }
+  __syncthreads();
+  if (g == 1) return;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const float m1 = xch[(8 * r) * ATP_GT + gt], s1 = xch[(8 * r + 1) * ATP_GT + gt];
+    const float mn = fmaxf(m[r], m1);
+    const float c0 = m[r] == -INFINITY ? 0.f : expf(m[r] - mn);
+    const float c1 = m1 == -INFINITY ? 0.f : expf(m1 - mn);
+    const float tot = sum[r] * c0 + s1 * c1;
+    const int row = tq + 16 * r;
+    const float inv = 1.0f / tot;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float4 res;
+      res.x = (o[r][i][0] * c0 + xch[(32 + 16 * r + 4 * i + 0) * ATP_GT + gt] * c1) * inv;
+      res.y = (o[r][i][1] * c0 + xch[(32 + 16 * r + 4 * i + 1) * ATP_GT + gt] * c1) * inv;
+      res.z = (o[r][i][2] * c0 + xch[(32 + 16 * r + 4 * i + 2) * ATP_GT + gt] * c1) * inv;
+      res.w = (o[r][i][3] * c0 + xch[(32 + 16 * r + 4 * i + 3) * ATP_GT + gt] * c1) * inv;
+      if (row < nq)
+        *reinterpret_cast<float4*>(A + ((size_t)b * L + l0 + row) * HD + h * ATT_D + 4 * tk + 32 * i) = res;
     }
   }
 }
