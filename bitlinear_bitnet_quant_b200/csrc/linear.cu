@@ -109,25 +109,34 @@ linear_simt_kernel(const uint8_t* __restrict__ Xq, const float* __restrict__ s_x
 // operand B = the activation tile, brought by TMA into shared memory with the
 // 128-byte swizzle (int4 tiles are widened there by the converter warps);
 // D = int32 accumulators in tensor memory.
-//   warp 0    : TMA producer (and the per-token dequantisation scales)
+//   warp 0    : TMA producer of the weight tiles (and the per-token
+//               dequantisation scales)
 //   warp 1    : tensor-memory allocator and MMA issuer (one thread)
 //   warps 2-9 : converters, then the epilogue.  Warp w serves tensor-memory
 //               lanes 32*(w%4).. and half (w-2)/4 of the K bytes of a step
 //               (and of the token columns in the epilogue).
+//   warp 10   : TMA producer of the activation tiles.  Measured on B200, the
+//               tiles one warp issues land one after another (about 0.36 us
+//               each, whatever their size); two issuing warps halve the wait.
 // When the tiles alone leave SMs idle, K is split over a cluster of ksplit
 // CTAs (grid z); partial sums travel to the leader by one bulk copy each.
 // ===========================================================================
-constexpr int TC_THREADS = 320;
+constexpr int TC_THREADS = 352;
+constexpr int TC_XWARP = 10;                       // activation-tile producer
 constexpr int TC_CONV_THREADS = 256;
 constexpr int TC_BK = 128;
 
 // MB = 128 or 256 weight rows per CTA.  With 256, two M = 128 MMAs (two
 // accumulators, two A slices in tensor memory) share every activation tile:
 // half the activation bytes per MMA, at one CTA per SM (all 512 columns).
-// On B200 an SM takes in about 47-50 bytes per clock (measured with 16 KB
-// transfers, whatever the method), below the 80 bytes per clock that a
-// 128 x 128 tile needs at the int8 MMA rate: the bytes per MMA set the speed
-// of the 128-row tile.
+// Measured on B200 (clock64 stamps per K step): in the steady state the
+// 128 x 128 tile at two CTAs per SM issues a K step every ~850-900 cycles per
+// CTA against 256 of MMA work, with each activation tile landing ~2500 cycles
+// after its copy is issued; the SM then takes in ~45 bytes per clock of the
+// 80 that the MMA rate needs, while the shared memory also serves the MMA's
+// reads of the same tiles.  A CTA spends another ~2000 cycles before its
+// first MMA and ~6000 in the epilogue, which the CTA sharing its SM overlaps
+// only in part.
 template <int BN, int ACT_BITS, int MB = 128>
 struct TcCfg {
   static constexpr int RB = MB / 128;                          // row blocks = accumulators
@@ -153,6 +162,12 @@ struct TcCfg {
   static constexpr int S0 = S_SMEM < S_TMEM ? S_SMEM : S_TMEM;
   static constexpr int S = RB == 1 ? (S0 > 6 ? 6 : S0) : (S_SMEM > 8 ? 8 : S_SMEM);   // shared-memory stages
   static constexpr int ST = RB == 1 ? S : S_TMEM;                                      // tensor-memory A slots
+  // K steps per copy: consecutive stages are filled in pairs by one 3-D box
+  // each (measured on B200, the boxes one warp issues land one after another
+  // at about 0.36 us each whatever their size, so fewer, larger boxes feed an
+  // SM faster); a pair shares its full / empty barriers.
+  static constexpr int P = (S % 2 == 0 && S >= 4) ? 2 : 1;
+  static constexpr int SP = S / P;                                                     // pair stages
   static constexpr int COLS_NEEDED = DCOLS + ACOLS * ST;
   static constexpr int TMEM_COLS = COLS_NEEDED <= 32 ? 32 : COLS_NEEDED <= 64 ? 64 :
                                    COLS_NEEDED <= 128 ? 128 : COLS_NEEDED <= 256 ? 256 : 512;
@@ -204,7 +219,8 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
   // int4, activations widened); empty: stage free; acc: all MMAs done; sdq: scales ready;
   // red: split-K partials of the other ranks landed (leader only)
   // afree: the A slot's MMAs are done (used only when the A ring is shorter than the stage ring)
-  __shared__ __align__(8) uint64_t bar_wfull[S], bar_xfull[S], bar_empty[S], bar_conv[ST], bar_afree[ST];
+  constexpr int P = C::P, SP = C::SP;
+  __shared__ __align__(8) uint64_t bar_wfull[SP], bar_xfull[SP], bar_empty[SP], bar_conv[ST], bar_afree[ST];
   __shared__ __align__(8) uint64_t bar_acc, bar_sdq, bar_red;
   __shared__ uint32_t tmem_base_sh;
   __shared__ float sdq[BN];
@@ -212,7 +228,8 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
   auto xs = [&](int s) { return base + (size_t)s * C::XBYTES; };                          // 1024-aligned
   auto xraw = [&](int s) { return base + (size_t)S * C::XBYTES + (size_t)s * C::XRAW; };
-  auto ws = [&](int s) { return base + (size_t)S * (C::XBYTES + C::XRAW) + (size_t)s * C::WBYTES; };
+  // packed weights of pair stage p: [row block][step of the pair][128 rows][32 B]
+  auto wsp = [&](int p) { return base + (size_t)S * (C::XBYTES + C::XRAW) + (size_t)p * P * C::WBYTES; };
   // split-K partial sums, [slot][column][row] int32: in the leader, slot r-1 receives rank r;
   // in the other ranks, slot 0 stages the outgoing partial
   int32_t* red = reinterpret_cast<int32_t*>(base + (size_t)S * C::STAGE);
@@ -236,10 +253,10 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
   const int nk = (int)((int64_t)nk_all * (kr + 1) / ksplit) - kb;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&bar_wfull[s], 1);
-      mbar_init(&bar_xfull[s], 1);
-      mbar_init(&bar_empty[s], 1 + 8);
+    for (int p = 0; p < SP; ++p) {
+      mbar_init(&bar_wfull[p], 1);
+      mbar_init(&bar_xfull[p], 1);
+      mbar_init(&bar_empty[p], 1 + 8);
     }
     for (int a = 0; a < ST; ++a) {
       mbar_init(&bar_conv[a], 8);
@@ -267,28 +284,22 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
   // of this grid still has to allocate (later grids only wait on earlier ones).
   pdl_launch_dependents();
 
+  // pair j covers K steps jP .. jP+P-1 and uses pair stage j % SP in round j / SP
+  const int npairs = (nk + P - 1) / P;
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    const int pre = nk < S ? nk : S;
-    if (lane == 0) {
-      // weights do not depend on the previous kernel: start streaming them now
-      for (int i = 0; i < pre; ++i) {
-        mbar_arrive_expect_tx(&bar_wfull[i], C::WBYTES);
+    // ------------------------------------------------------------ weight producer
+    const int pre = npairs < SP ? npairs : SP;
+    auto load_w = [&](int j) {
+      const int p = j % SP;
+      mbar_arrive_expect_tx(&bar_wfull[p], (uint32_t)(P * C::WBYTES));
 #pragma unroll
-        for (int rb = 0; rb < RB; ++rb)
-          tma_load_2d(ws(i) + rb * (C::WBYTES / RB), tmW, &bar_wfull[i], (kb + i) * (TC_BK / 4), n0 + 128 * rb);
-      }
-    }
-    __syncwarp();
-    pdl_wait();                                    // activations and s_x come from the previous kernel
-    auto load_x = [&](int i) {
-      const int s = i % S;
-      mbar_arrive_expect_tx(&bar_xfull[s], XTX);
-      if constexpr (ACT_BITS == 8) tma_load_2d(xs(s), &tmX, &bar_xfull[s], (kb + i) * TC_BK, m0);
-      else tma_load_2d(xraw(s), &tmX, &bar_xfull[s], (kb + i) * (TC_BK / 2), m0);
+      for (int rb = 0; rb < RB; ++rb)
+        tma_load_3d(wsp(p) + rb * P * (C::WBYTES / RB), tmW, &bar_wfull[p], 0, n0 + 128 * rb, kb + j * P);
     };
     if (lane == 0)
-      for (int i = 0; i < pre; ++i) load_x(i);    // first: the activations are on the critical path
+      for (int j = 0; j < pre; ++j) load_w(j);   // weights do not depend on the previous kernel
+    __syncwarp();
+    pdl_wait();                                    // s_x comes from the previous kernel
     if (kr == 0) {
       if (lane == 0 && use_tma_store) tma_prefetch_desc(tmY);
       const float sw = ldg_nc_f32(s_w_ptr);
@@ -301,22 +312,32 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
     }
     if (lane == 0) {
       int issued = pre;
-      for (int i = pre; i < nk; ++i) {
-        const int s = i % S, r = i / S;
-        if (!mbar_wait(&bar_empty[s], (r - 1) & 1, DEV_ERR_TIMEOUT_EMPTY)) break;
-        mbar_arrive_expect_tx(&bar_wfull[s], C::WBYTES);
-#pragma unroll
-        for (int rb = 0; rb < RB; ++rb)
-          tma_load_2d(ws(s) + rb * (C::WBYTES / RB), tmW, &bar_wfull[s], (kb + i) * (TC_BK / 4), n0 + 128 * rb);
-        load_x(i);
-        issued = i + 1;
+      for (int j = pre; j < npairs; ++j) {
+        if (!mbar_wait(&bar_empty[j % SP], ((j / SP) - 1) & 1, DEV_ERR_TIMEOUT_EMPTY)) break;
+        load_w(j);
+        issued = j + 1;
       }
       // every copy issued has landed before the CTA may exit (returns at once
       // on the normal path, where the consumers have already waited for them)
-      for (int i = issued - S < 0 ? 0 : issued - S; i < issued; ++i) {
-        mbar_wait(&bar_wfull[i % S], (i / S) & 1, DEV_ERR_TIMEOUT_FULL, false);
-        mbar_wait(&bar_xfull[i % S], (i / S) & 1, DEV_ERR_TIMEOUT_FULL, false);
+      for (int j = issued - SP < 0 ? 0 : issued - SP; j < issued; ++j)
+        mbar_wait(&bar_wfull[j % SP], (j / SP) & 1, DEV_ERR_TIMEOUT_FULL, false);
+    }
+  } else if (warp == TC_XWARP) {
+    // ------------------------------------------------------------ activation producer
+    if (lane == 0) {
+      pdl_wait();                                  // the activations come from the previous kernel
+      int issued = 0;
+      for (int j = 0; j < npairs; ++j) {
+        const int p = j % SP;
+        if (j >= SP && !mbar_wait(&bar_empty[p], ((j / SP) - 1) & 1, DEV_ERR_TIMEOUT_EMPTY)) break;
+        mbar_arrive_expect_tx(&bar_xfull[p], (uint32_t)P * XTX);
+        // the pair's steps land in consecutive stages p P and p P + 1
+        if constexpr (ACT_BITS == 8) tma_load_3d(xs(p * P), &tmX, &bar_xfull[p], 0, m0, kb + j * P);
+        else tma_load_3d(xraw(p * P), &tmX, &bar_xfull[p], 0, m0, kb + j * P);
+        issued = j + 1;
       }
+      for (int j = issued - SP < 0 ? 0 : issued - SP; j < issued; ++j)
+        mbar_wait(&bar_xfull[j % SP], (j / SP) & 1, DEV_ERR_TIMEOUT_FULL, false);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -325,7 +346,7 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
       for (int i = 0; i < nk; ++i) {
         const int s = i % S, r = i / S;
         const int a = i % ST, ra = i / ST;
-        if (!mbar_wait(&bar_xfull[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
+        if (!mbar_wait(&bar_xfull[s / P], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
         if (!mbar_wait(&bar_conv[a], ra & 1, DEV_ERR_TIMEOUT_A)) break;
         tc_fence_after();
         const uint32_t xaddr = smem_u32(xs(s));
@@ -340,7 +361,9 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
             mma_i8_ts(tmem + (uint32_t)(BN * rb), aaddr, bdesc, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        if (i + S < nk) mma_commit(&bar_empty[s]);   // only stages that are refilled need releasing
+        // a pair stage is released after its last step's MMAs (the commit
+        // tracks every earlier MMA), and only if it is refilled
+        if (s % P == P - 1 && i - (P - 1) + S < nk) mma_commit(&bar_empty[s / P]);
         if (ST < S && i + ST < nk) mma_commit(&bar_afree[a]);
       }
       mma_commit(&bar_acc);
@@ -357,7 +380,8 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
     for (int i = 0; i < nk; ++i) {
       const int s = i % S, r = i / S;
       const int a = i % ST, ra = i / ST;
-      if (!mbar_wait_warp(&bar_wfull[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
+      const int c = s % P;                         // step inside the pair
+      if (!mbar_wait_warp(&bar_wfull[s / P], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
       tc_fence_after();
       // 64 weights of this row (of each row block) -> 16 tensor-memory columns
       // the tile arrives with the 32-byte swizzle: the two 16-byte halves of
@@ -366,10 +390,11 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
       uint4 w[RB];
 #pragma unroll
       for (int rb = 0; rb < RB; ++rb)
-        w[rb] = *reinterpret_cast<const uint4*>(ws(s) + 32 * (row + 128 * rb) + 16 * (h ^ ((row >> 2) & 1)));
+        w[rb] = *reinterpret_cast<const uint4*>(wsp(s / P) + (rb * P + c) * (C::WBYTES / RB) + 32 * row +
+                                                16 * (h ^ ((row >> 2) & 1)));
       if constexpr (ACT_BITS == 8) {
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_empty[s]);   // packed tile consumed
+        if (lane == 0 && c == P - 1) mbar_arrive(&bar_empty[s / P]);   // the pair's packed tiles consumed
       }
       if constexpr (ST < S) {
         // the A slot is free once the MMAs of step i - ST are done
@@ -389,20 +414,32 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
       }
       if constexpr (ACT_BITS == 4) {
         // int4 activation tile: widen to int8 (16*x) in the 128-byte-swizzled layout
-        if (!mbar_wait_warp(&bar_xfull[s], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
+        if (!mbar_wait_warp(&bar_xfull[s / P], r & 1, DEV_ERR_TIMEOUT_FULL)) break;
+        // all of a thread's 8-byte chunks are read before any is widened, so
+        // their shared-memory latencies overlap
+        constexpr int WI = (BN * 8 + TC_CONV_THREADS - 1) / TC_CONV_THREADS;
         uint8_t* dst = xs(s);
         const uint8_t* src = xraw(s);
-        for (int idx = ct; idx < BN * 8; idx += TC_CONV_THREADS) {
-          const int rr = idx >> 3, c = idx & 7;
-          const uint2 p = *reinterpret_cast<const uint2*>(src + 64 * rr + 8 * c);
-          uint32_t o0, o1, o2, o3;
-          widen8(p.x, o0, o1);
-          widen8(p.y, o2, o3);
-          *reinterpret_cast<uint4*>(dst + 128 * rr + 16 * (c ^ (rr & 7))) = make_uint4(o0, o1, o2, o3);
+        uint2 pk[WI];
+#pragma unroll
+        for (int u = 0; u < WI; ++u) {
+          const int idx = ct + u * TC_CONV_THREADS;
+          if (idx < BN * 8) pk[u] = *reinterpret_cast<const uint2*>(src + 64 * (idx >> 3) + 8 * (idx & 7));
+        }
+#pragma unroll
+        for (int u = 0; u < WI; ++u) {
+          const int idx = ct + u * TC_CONV_THREADS;
+          if (idx < BN * 8) {
+            const int rr = idx >> 3, c = idx & 7;
+            uint32_t o0, o1, o2, o3;
+            widen8(pk[u].x, o0, o1);
+            widen8(pk[u].y, o2, o3);
+            *reinterpret_cast<uint4*>(dst + 128 * rr + 16 * (c ^ (rr & 7))) = make_uint4(o0, o1, o2, o3);
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_empty[s]);
+        if (lane == 0 && c == P - 1) mbar_arrive(&bar_empty[s / P]);
       }
       // Hand every step to the MMA issuer as soon as its operands are in place
       // (measured on B200: holding steps back to batch the tensor-memory store
@@ -489,7 +526,7 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
         asm volatile("bar.sync 1, 256;" ::: "memory");
         if (ct == 0 && ok) {
           tma_store_2d(tmY, ostage, n0 + 128 * rb, m0);
-          bulk_wait_all();
+          bulk_wait_read();                        // the staging may be reused / released once read
         }
       }
       }
@@ -502,7 +539,7 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
-  if (ksplit > 1 && warp < 2) cluster_wait();     // pairs this warp's cluster_arrive
+  if (ksplit > 1 && (warp < 2 || warp == TC_XWARP)) cluster_wait();     // pairs this warp's cluster_arrive
 }
 
 // ===========================================================================
@@ -538,9 +575,21 @@ static bool make_map_2d(CUtensorMap* map, const void* ptr, CUtensorMapDataType d
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static bool make_map_bytes(CUtensorMap* map, const void* ptr, uint64_t inner_bytes, uint64_t rows,
-                           uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
-  return make_map_2d(map, ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, inner_bytes, rows, inner_bytes, box_inner, box_rows, sw);
+// Bytes [K steps][rows][step bytes] of a row-major [rows][row_bytes] matrix:
+// dimension 0 = the step_bytes of one K step, 1 = rows (stride row_bytes),
+// 2 = K steps (stride step_bytes); a box of `steps` K steps lands as
+// consecutive [box_rows][step_bytes] tiles.
+static bool make_map_steps(CUtensorMap* map, const void* ptr, uint64_t row_bytes, uint64_t rows, uint32_t step_bytes,
+                           uint32_t box_rows, uint32_t steps, CUtensorMapSwizzle sw) {
+  EncodeFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {step_bytes, rows, row_bytes / step_bytes};
+  cuuint64_t strides[2] = {row_bytes, step_bytes};
+  cuuint32_t box[3] = {step_bytes, box_rows, steps};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <typename T> struct MapType;
@@ -553,8 +602,8 @@ static cudaError_t launch_tc(LinGroup grp, const void* Xq, const float* s_x, int
   TcMaps maps;                                     // copied into the launch's parameters
   CUtensorMap tmX;
   const bool ok = ACT_BITS == 8
-      ? make_map_bytes(&tmX, Xq, (uint64_t)K, (uint64_t)M, TC_BK, BN, CU_TENSOR_MAP_SWIZZLE_128B)
-      : make_map_bytes(&tmX, Xq, (uint64_t)K / 2, (uint64_t)M, TC_BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
+      ? make_map_steps(&tmX, Xq, (uint64_t)K, (uint64_t)M, TC_BK, BN, C::P, CU_TENSOR_MAP_SWIZZLE_128B)
+      : make_map_steps(&tmX, Xq, (uint64_t)K / 2, (uint64_t)M, TC_BK / 2, BN, C::P, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
   // The output leaves through one TMA store per tile when rows are 16-byte
   // multiples; the diagnostics accumulators take the per-element path.
@@ -563,7 +612,7 @@ static cudaError_t launch_tc(LinGroup grp, const void* Xq, const float* s_x, int
     if (grp.acc_dbg[g] != nullptr || ((uint64_t)grp.N[g] * sizeof(TOut)) % 16 != 0) use_tma_store = 0;
   grp.first[0] = 0;
   for (int g = 0; g < grp.count; ++g) {
-    if (!make_map_bytes(&maps.w[g], grp.pkW[g], (uint64_t)K / 4, (uint64_t)grp.N[g], TC_BK / 4, 128,
+    if (!make_map_steps(&maps.w[g], grp.pkW[g], (uint64_t)K / 4, (uint64_t)grp.N[g], TC_BK / 4, 128, C::P,
                         CU_TENSOR_MAP_SWIZZLE_32B))
       return cudaErrorInvalidValue;
     if (use_tma_store && !make_map_2d(&maps.y[g], grp.Y[g], MapType<TOut>::v, (uint64_t)grp.N[g], (uint64_t)M,
@@ -619,8 +668,9 @@ static cudaError_t dispatch_tc(const LinGroup& grp, const void* Xq, const float*
   if (M <= 64) return launch_tc<64, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
   // 256 weight rows per CTA halve the activation bytes per MMA but hold a
   // whole SM.  Measured on B200 it runs the batched prefill product slower
-  // than the 128-row tile at two CTAs per SM (about 1700 cycles per K step
-  // against 512 of MMA work), so it is used only when asked for (kernel 4).
+  // than the 128-row tile at two CTAs per SM (about 1250 cycles per K step
+  // against 512 of MMA work, with the activation tiles landing only every
+  // ~1250 cycles), so it is used only when asked for (kernel 4).
   int sms = 148, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
