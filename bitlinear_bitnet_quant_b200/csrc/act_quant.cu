@@ -889,27 +889,37 @@ hadamard_quant_i4_warp_kernel(const TIn* __restrict__ X, const float* __restrict
 #pragma unroll
     for (int c = 0; c < E; ++c) v[c] = __fmul_rn(v[c], r);
   }
-  // ---- stages of stride 1 .. E/2 in registers, then E .. b/2 across lanes ----
+  // ---- stages of stride 1 .. E/2 in registers, then E .. b/2 across lanes,
+  // on packed fp32 pairs (elements 2j, 2j+1) except the stride-1 stage ----
+  uint64_t pv[E / 2];
 #pragma unroll
-  for (int h = 1; h < E; h <<= 1) {
+  for (int j = 0; j < E / 2; ++j) pv[j] = f2_pack(__fadd_rn(v[2 * j], v[2 * j + 1]), __fsub_rn(v[2 * j], v[2 * j + 1]));
 #pragma unroll
-    for (int c = 0; c < E; ++c) {
-      if ((c & h) == 0) {
-        const float a = v[c], b = v[c + h];
-        v[c] = __fadd_rn(a, b);
-        v[c + h] = __fsub_rn(a, b);
+  for (int h = 1; h < E / 2; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < E / 2; ++j) {
+      if ((j & h) == 0) {
+        const uint64_t a = pv[j], b = pv[j + h];
+        pv[j] = f2_add(a, b);
+        pv[j + h] = f2_sub(a, b);
       }
     }
   }
 #pragma unroll
   for (int lb = 1; lb < 32; lb <<= 1) {
-    const bool upper = (lane & lb) != 0;
+    // the lower lane keeps v + other, the upper other - v: (+-1) * v + other
+    const float sg = (lane & lb) != 0 ? -1.0f : 1.0f;
+    const uint64_t sg2 = f2_pack(sg, sg);
 #pragma unroll
-    for (int c = 0; c < E; ++c) {
-      const float other = __shfl_xor_sync(0xffffffffu, v[c], lb);
-      v[c] = upper ? __fsub_rn(other, v[c]) : __fadd_rn(v[c], other);
+    for (int j = 0; j < E / 2; ++j) {
+      float a, b;
+      f2_unpack(pv[j], a, b);
+      const float oa = __shfl_xor_sync(0xffffffffu, a, lb), ob = __shfl_xor_sync(0xffffffffu, b, lb);
+      pv[j] = f2_fma(sg2, pv[j], f2_pack(oa, ob));
     }
   }
+#pragma unroll
+  for (int j = 0; j < E / 2; ++j) f2_unpack(pv[j], v[2 * j], v[2 * j + 1]);
   // ---- normalise, absmax over the token ----
   float amax = 0.f;
 #pragma unroll

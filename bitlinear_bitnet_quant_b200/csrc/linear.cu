@@ -25,6 +25,11 @@ template <typename T> BN_DEV void store_out(T* p, float v);
 template <> BN_DEV void store_out<float>(float* p, float v) { *p = v; }
 template <> BN_DEV void store_out<__nv_bfloat16>(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
+// float(a) for |a| < 2^22 without the (quarter-rate) conversion instruction:
+// a + 0x4B400000 is the bit pattern of 1.5 * 2^23 + a (consecutive fp32
+// values are 1 apart there), and the subtraction is exact.
+BN_DEV float small_int_to_float(int a) { return __fsub_rn(__int_as_float(a + 0x4B400000), 12582912.0f); }
+
 BN_DEV float dequant_scale(float sx, float sw) {
   return __fmul_rn(__fdiv_rn(1.0f, sx), __fdiv_rn(1.0f, sw));
 }
@@ -452,6 +457,8 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
 
     // ------------------------------------------------------------ epilogue
     constexpr int SHIFT = ACT_BITS == 8 ? 6 : 10;
+    // |acc| <= qmax * K: below 2^22 the cheap exact conversion applies
+    const bool small_acc = (int64_t)(ACT_BITS == 8 ? 127 : 8) * K < (int64_t)(1 << 22);
     const int cbeg = h * C::HALF;                // this warp's token columns
     const bool acc_ok = mbar_wait_warp(&bar_acc, 0, DEV_ERR_TIMEOUT_ACC);
     tc_fence_after();
@@ -502,7 +509,7 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
 #pragma unroll
             for (int jj = 0; jj < NC; ++jj) {
               const int acc = (int)v[g][jj] >> SHIFT;
-              float y = __fmul_rn((float)acc, sdq[c0 + jj]);
+              float y = __fmul_rn(small_acc ? small_int_to_float(acc) : (float)acc, sdq[c0 + jj]);
               if (!ok) y = 0.f;
               store_out(ostage + (size_t)(c0 + jj) * 128 + row, y);
             }
