@@ -140,8 +140,9 @@ def tensor_peak(ctx) -> tuple:
 
 
 def profiled_traffic(kernel_tag: str):
-    """Per-launch DRAM bytes from the committed ncu summary, if it was taken
-    on the current kernel sources (else None)."""
+    """DRAM bytes per launch (per step for the stacked-layer workloads, whose
+    roofline covers every linear launch of a step) from the committed ncu
+    summary, if it was taken on the current kernel sources (else None)."""
     path = os.path.join(ROOT, "profiles", f"{kernel_tag}.txt")
     try:
         kv = {}
@@ -152,7 +153,7 @@ def profiled_traffic(kernel_tag: str):
                     kv[k.strip()] = v.strip()
         if kv.get("kernel_source_hash") != kernel_source_hash():
             return None
-        return float(kv["dram_bytes_per_launch"])
+        return float(kv["dram_bytes_per_launch"] if "dram_bytes_per_launch" in kv else kv["dram_bytes_per_step"])
     except Exception:
         return None
 
