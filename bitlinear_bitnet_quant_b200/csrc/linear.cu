@@ -25,6 +25,17 @@ template <typename T> BN_DEV void store_out(T* p, float v);
 template <> BN_DEV void store_out<float>(float* p, float v) { *p = v; }
 template <> BN_DEV void store_out<__nv_bfloat16>(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
+// The epilogue's store of one output into the staged tile.  bf16: round to
+// nearest even on the bit pattern with integer operations (the conversion
+// instruction issues at a quarter of the rate); equal to __float2bfloat16_rn
+// for every non-NaN input, and the dequantised outputs are never NaN.
+template <typename T> BN_DEV void stage_out(T* p, float v);
+template <> BN_DEV void stage_out<float>(float* p, float v) { *p = v; }
+template <> BN_DEV void stage_out<__nv_bfloat16>(__nv_bfloat16* p, float v) {
+  const uint32_t u = __float_as_uint(v);
+  *reinterpret_cast<uint16_t*>(p) = (uint16_t)((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
+}
+
 // float(a) for |a| < 2^22 without the (quarter-rate) conversion instruction:
 // a + 0x4B400000 is the bit pattern of 1.5 * 2^23 + a (consecutive fp32
 // values are 1 apart there), and the subtraction is exact.
@@ -228,7 +239,7 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
   __shared__ __align__(8) uint64_t bar_wfull[SP], bar_xfull[SP], bar_empty[SP], bar_conv[ST], bar_afree[ST];
   __shared__ __align__(8) uint64_t bar_acc, bar_sdq, bar_red;
   __shared__ uint32_t tmem_base_sh;
-  __shared__ float sdq[BN];
+  __shared__ __align__(16) float sdq[BN];
 
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
   auto xs = [&](int s) { return base + (size_t)s * C::XBYTES; };                          // 1024-aligned
@@ -506,12 +517,29 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
             for (int jj = 0; jj < NC; ++jj) v[g][jj] += (uint32_t)red[((pr - 1) * BN + c0 + jj) * 128 + row];
           }
           if (use_tma_store) {
+            // the chunk's scales in registers (c0 is a multiple of 16), and the
+            // conversion chosen once per chunk: measured on B200, the per-value
+            // scale reads, conversion instructions and select made this loop
+            // ~2/3 of the epilogue
+            float sq[NC];
 #pragma unroll
-            for (int jj = 0; jj < NC; ++jj) {
-              const int acc = (int)v[g][jj] >> SHIFT;
-              float y = __fmul_rn(small_acc ? small_int_to_float(acc) : (float)acc, sdq[c0 + jj]);
-              if (!ok) y = 0.f;
-              store_out(ostage + (size_t)(c0 + jj) * 128 + row, y);
+            for (int q4 = 0; q4 < NC / 4; ++q4) {
+              const float4 f = *reinterpret_cast<const float4*>(sdq + c0 + 4 * q4);
+              sq[4 * q4] = f.x; sq[4 * q4 + 1] = f.y; sq[4 * q4 + 2] = f.z; sq[4 * q4 + 3] = f.w;
+            }
+            if (!ok) {
+#pragma unroll
+              for (int jj = 0; jj < NC; ++jj) sq[jj] = 0.f;
+            }
+            TOut* dst = ostage + (size_t)c0 * 128 + row;
+            if (small_acc) {
+#pragma unroll
+              for (int jj = 0; jj < NC; ++jj)
+                stage_out(dst + jj * 128, __fmul_rn(small_int_to_float((int)v[g][jj] >> SHIFT), sq[jj]));
+            } else {
+#pragma unroll
+              for (int jj = 0; jj < NC; ++jj)
+                stage_out(dst + jj * 128, __fmul_rn((float)((int)v[g][jj] >> SHIFT), sq[jj]));
             }
           } else if (ok && n < N) {
 #pragma unroll
