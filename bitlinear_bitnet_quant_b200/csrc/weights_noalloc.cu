@@ -12,12 +12,12 @@
 // The array lives for as long as the library is loaded, on every device that
 // uses it.  Host code cannot use the array's name as a device address, so the
 // first call on each device looks the address up with cudaGetSymbolAddress
-// (with that device current) and caches it; do that first call before any
-// stream capture.  The cached address belongs to the device's primary context:
-// after cudaDeviceReset, or under a context the caller created itself, it no
-// longer names the array, and this entry point must not be called.  All calls share the one array: the counters are cleared at
-// the start of each call, and two calls whose kernels overlap on the GPU (for
-// example on two streams) race on it.
+// (with that device current) and caches it.  The cached address belongs to
+// the device's primary context: after cudaDeviceReset, or under a context the
+// caller created itself, it no longer names the array, and this entry point
+// must not be called.  All calls share the one array: the counters are cleared
+// at the start of each call, and two calls whose kernels overlap on the GPU
+// (for example on two streams) race on it.
 #include <cuda_runtime.h>
 #include <stdint.h>
 

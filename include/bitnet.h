@@ -108,10 +108,10 @@ BITNET_API int bitnet_quantize_weights(const void* W, int w_dtype, int64_t N, in
  * device that uses it until the library is unloaded.  The caller still owns W,
  * pkW and s_w.  No cudaMalloc, cudaFree or allocating routine is called.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.  The address is cached for the device's
- *     primary context: do not call this entry point after cudaDeviceReset or
- *     under a context the caller created itself (cuCtxCreate).
+ *     (cudaGetSymbolAddress, with that device current).  The address is
+ *     cached for the device's primary context: do not call this entry point
+ *     after cudaDeviceReset or under a context the caller created itself
+ *     (cuCtxCreate).
  *   - Every call shares the one array and clears it before use; calls whose
  *     kernels overlap on the GPU (e.g. on two streams) race on it.
  *   - Limit: N*K <= BITNET_NOALLOC_MAX_WEIGHTS (what the fixed 64-bit counters
