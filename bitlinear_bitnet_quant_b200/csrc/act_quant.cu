@@ -1026,9 +1026,11 @@ static cudaError_t launch_h4(const void* X, const float* B, int M, int K, const 
   // of K / 32 threads, 32 elements per thread.
   if constexpr (L >= 10) {
     const int W = K == 2048 ? 1 : K == 4096 ? 2 : K == 8192 ? 3 : K == 16384 ? 4 : 0;
-    // 64 or 128 threads per token only with enough tokens to fill the SMs (a few
-    // tokens go faster on the one-CTA-per-token kernel's 256 threads)
-    if (W != 0 && L <= 10 + W && (W >= 3 || M >= sms)) {
+    // 64 or 128 threads per token only with many tokens: measured on B200 at
+    // 512 tokens of K = 2048 (the O projection's input) the one-CTA-per-token
+    // kernel's 256 threads take 5.3 us per launch against 7.7 us here (two
+    // warps per token leave the SMs short of warps)
+    if (W != 0 && L <= 10 + W && (W >= 3 || M >= 16 * sms)) {
       const size_t ssmem = (size_t)(K + K / 32) * sizeof(float) + (size_t)K / 2;
       const unsigned grid = (unsigned)M;
 #define BN_HS(WW)                                                                                           \

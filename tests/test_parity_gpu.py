@@ -181,7 +181,8 @@ def test_hadamard_quant_many_tokens(M, K, b, dtype):
 
 @pytest.mark.parametrize("M,K,b,dtype,use_gamma", [(640, 4096, 0, "bf16", False), (600, 8192, 1024, "f32", False),
                                                    (700, 16384, 8192, "bf16", True), (620, 8192, 0, "f32", True),
-                                                   (900, 4096, 2048, "f32", False), (300, 8192, 0, "bf16", True)])
+                                                   (900, 4096, 2048, "f32", False), (300, 8192, 0, "bf16", True),
+                                                   (2400, 4096, 0, "bf16", False)])
 def test_hadamard_quant_split_kernel(M, K, b, dtype, use_gamma):
     """Many tokens at K = 4096 / 8192 / 16384 with blocks of 1024 or more: the
     kernels that spread a token over K/32 threads (three index-bit groups;
