@@ -187,7 +187,7 @@ bitlinear_fused_kernel(const TIn* __restrict__ X, int M, int K, const float* __r
   const int xpitch = K + 64, spitch = K + 16;
   const uint32_t row_bytes = (uint32_t)K + 16u;        // codes and the scale
 
-  uint8_t* wsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fuse_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* wsm = smem_align(fuse_smem_raw, 1024u);
   const size_t wbytes = (size_t)ROWS * K / 4, rbytes = dec_red_bytes<TG, RG>();
   uint8_t* xbuf = wsm + (wbytes > rbytes ? wbytes : rbytes);
   uint8_t* stage = xbuf + (size_t)M * xpitch;

@@ -106,6 +106,16 @@ BN_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// p advanced to the next multiple of `align` (a power of two) bytes of the
+// shared window, by pointer arithmetic on the shared array itself: the
+// compiler then still knows that the result addresses shared memory (a round
+// trip through an integer would make every access through it a generic one).
+template <typename T>
+BN_DEV T* smem_align(T* p, uint32_t align) {
+  const uint32_t pad = (align - (smem_u32(p) & (align - 1u))) & (align - 1u);
+  return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(p) + pad);
+}
+
 BN_DEV uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));

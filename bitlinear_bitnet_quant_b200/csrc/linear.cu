@@ -241,7 +241,7 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
   __shared__ uint32_t tmem_base_sh;
   __shared__ __align__(16) float sdq[BN];
 
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* base = smem_align(dsmem_raw, 1024u);
   auto xs = [&](int s) { return base + (size_t)s * C::XBYTES; };                          // 1024-aligned
   auto xraw = [&](int s) { return base + (size_t)S * C::XBYTES + (size_t)s * C::XRAW; };
   // packed weights of pair stage p: [row block][step of the pair][128 rows][32 B]

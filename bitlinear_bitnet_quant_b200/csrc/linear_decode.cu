@@ -62,7 +62,7 @@ linear_decode_kernel(const __grid_constant__ LinGroup grp, const uint8_t* __rest
   __shared__ float sdq[TOK];
   __shared__ uint16_t lut5[W5 ? 243 : 1];
 
-  uint8_t* wsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dec_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* wsm = smem_align(dec_smem_raw, 1024u);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int nseg = K / 512;

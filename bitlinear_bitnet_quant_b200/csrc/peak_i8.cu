@@ -23,7 +23,7 @@ peak_i8_kernel(int n_mma, unsigned long long* __restrict__ cycles, unsigned long
   extern __shared__ uint8_t pk_raw[];
   __shared__ __align__(8) uint64_t bar_done;
   __shared__ uint32_t tmem_base_sh;
-  uint8_t* b = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pk_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* b = smem_align(pk_raw, 1024u);
   for (int i = threadIdx.x; i < BN * 128 / 4; i += PK_THREADS)
     reinterpret_cast<uint32_t*>(b)[i] = 0x9E3779B9u * (uint32_t)(i + 1);
   fence_proxy_async_smem();
