@@ -184,11 +184,11 @@ int bitnet_hadamard_quant_act(const void* X, int x_dtype, int64_t M, int64_t K, 
 }
 
 // kernel: 0 = automatic, 1 = CUDA-core dp4a, 2 = tcgen05, 3 = warp-MMA decode,
-// 4 = tcgen05 with 256 weight rows per CTA
+// 4 = tcgen05 with 256 weight rows per CTA, 5 = persistent tcgen05 (int8)
 static int linear_impl(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                        int64_t M, int64_t N, int64_t K, void* Y, int y_dtype, int32_t* acc_dbg, int kernel,
                        void* stream) {
-  if (kernel < 0 || kernel > 4) return BITNET_ERR_SHAPE;
+  if (kernel < 0 || kernel > 5) return BITNET_ERR_SHAPE;
   if (act_bits != 8 && act_bits != 4) return BITNET_ERR_DTYPE;
   if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
   if (M < 0 || M > (int64_t(1) << 30) || N < 1 || N > (int64_t(1) << 30) || K < 128 || K > 65536 ||
@@ -200,6 +200,7 @@ static int linear_impl(const void* Xq, int act_bits, const float* s_x, const uin
       (reinterpret_cast<uintptr_t>(s_x) & 3u) || (reinterpret_cast<uintptr_t>(s_w) & 3u))
     return BITNET_ERR_ALIGN;
   if (kernel == 3 && !bitnet::decode_path_applies((int)M, (int)K)) return BITNET_ERR_SHAPE;
+  if (kernel == 5 && (act_bits != 8 || M <= 64 || (K / 128) % 2 != 0)) return BITNET_ERR_SHAPE;
   int d = check_device();
   if (d != BITNET_OK) return d;
   if (!bitnet::tensor_map_encoder_available()) return BITNET_ERR_UNSUPPORTED;

@@ -578,6 +578,269 @@ linear_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CU
 }
 
 // ===========================================================================
+// Persistent variant of the int8 tcgen05 kernel (selectable per call, kernel
+// 5): one CTA per SM loops over the 128 x 128 tiles (static round robin), with
+// two accumulators in tensor memory and four epilogue warps of its own, so a
+// tile's epilogue and the next tile's start overlap the K loop instead of
+// adding to it.  Measured on B200 its K steps come no faster than those of one
+// CTA of the two-per-SM kernel (~800 cycles), so it is slower overall.
+//   warp 0     : weight-tile producer (two K steps per 3-D copy)
+//   warp 1     : tensor-memory allocator (all 512 columns) and MMA issuer
+//   warps 2-9  : converters (packed weights -> int8 in tensor memory)
+//   warp 10    : activation-tile producer
+//   warps 11-14: epilogue (tensor-memory lane quarter = warp % 4)
+// Tensor memory: accumulators at columns 0 and 128, eight A slots of 32 from
+// 256 (all 512 columns).  Shared memory: eight activation stages (16 KB), four
+// weight pair stages (8 KB), the output staging tile (128 x 128 outputs): as
+// many bytes in flight per SM as two CTAs of the non-persistent kernel hold.
+// ===========================================================================
+constexpr int PT_THREADS = 480;
+constexpr int PT_S = 8;                          // K-step stages (pairs of two)
+constexpr int PT_SP = PT_S / 2;
+constexpr int PT_ST = 8;                         // tensor-memory A slots
+constexpr int PT_XBYTES = 128 * 128;
+constexpr int PT_WBYTES = 128 * 32;
+constexpr int PT_EPI_WARP0 = 11;
+
+template <typename TOut>
+constexpr size_t pt_smem_bytes() {
+  return (size_t)PT_S * PT_XBYTES + (size_t)PT_S * PT_WBYTES + (size_t)128 * 128 * sizeof(TOut) + 1024;
+}
+
+template <typename TOut>
+__global__ void __launch_bounds__(PT_THREADS, 1)
+linear_tc_persistent_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ CUtensorMap tmX,
+                            const __grid_constant__ LinGroup grp, int use_tma_store, const float* __restrict__ s_x,
+                            int M, int K) {
+  constexpr int S = PT_S, SP = PT_SP, ST = PT_ST;
+  extern __shared__ uint8_t dsmem_raw[];
+  __shared__ __align__(8) uint64_t bar_wfull[SP], bar_xfull[SP], bar_empty[SP], bar_conv[ST];
+  __shared__ __align__(8) uint64_t bar_accf[2], bar_acce[2], bar_fin;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ __align__(16) float sdq[128];
+
+  uint8_t* base = smem_align(dsmem_raw, 1024u);
+  auto xs = [&](int st) { return base + (size_t)st * PT_XBYTES; };
+  auto wsp = [&](int pp) { return base + (size_t)S * PT_XBYTES + (size_t)pp * 2 * PT_WBYTES; };
+  TOut* ostage = reinterpret_cast<TOut*>(base + (size_t)S * (PT_XBYTES + PT_WBYTES));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntn = grp.first[grp.count];                    // weight-row tiles over the group
+  const int ntm = (M + 127) / 128;                         // token tiles
+  const int total = ntn * ntm;
+  const int ntl = blockIdx.x < total ? (total - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;   // tiles of this CTA
+  const int nk = K / TC_BK, npt = nk / 2;                  // K steps and pairs per tile (nk even)
+  const int npairs = ntl * npt;
+  auto tile_of = [&](int lt, int& gi, int& n0, int& m0) {
+    const int tt = (int)blockIdx.x + lt * (int)gridDim.x;
+    const int ni = tt % ntn;
+    gi = group_of(grp, ni);
+    n0 = (ni - grp.first[gi]) * 128;
+    m0 = (tt / ntn) * 128;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < SP; ++q) {
+      mbar_init(&bar_wfull[q], 1);
+      mbar_init(&bar_xfull[q], 1);
+      mbar_init(&bar_empty[q], 1 + 8);
+    }
+    for (int a = 0; a < ST; ++a) mbar_init(&bar_conv[a], 8);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar_accf[b], 1);
+      mbar_init(&bar_acce[b], 4);
+    }
+    mbar_init(&bar_fin, 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ weight producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int gj = 0; gj < npairs; ++gj) {
+        const int lt = gj / npt, j = gj - lt * npt, q = gj % SP;
+        int gi, n0, m0;
+        tile_of(lt, gi, n0, m0);
+        if (gj >= SP && !mbar_wait(&bar_empty[q], ((gj / SP) - 1) & 1, DEV_ERR_TIMEOUT_EMPTY)) break;
+        mbar_arrive_expect_tx(&bar_wfull[q], 2u * PT_WBYTES);
+        tma_load_3d(wsp(q), &maps.w[gi], &bar_wfull[q], 0, n0, 2 * j);
+        issued = gj + 1;
+      }
+      for (int gj = issued - SP < 0 ? 0 : issued - SP; gj < issued; ++gj)
+        mbar_wait(&bar_wfull[gj % SP], (gj / SP) & 1, DEV_ERR_TIMEOUT_FULL, false);
+    }
+  } else if (warp == TC_XWARP) {
+    // ------------------------------------------------------------ activation producer
+    if (lane == 0) {
+      pdl_wait();                                  // the activations come from the previous kernel
+      int issued = 0;
+      for (int gj = 0; gj < npairs; ++gj) {
+        const int lt = gj / npt, j = gj - lt * npt, q = gj % SP;
+        int gi, n0, m0;
+        tile_of(lt, gi, n0, m0);
+        if (gj >= SP && !mbar_wait(&bar_empty[q], ((gj / SP) - 1) & 1, DEV_ERR_TIMEOUT_EMPTY)) break;
+        mbar_arrive_expect_tx(&bar_xfull[q], 2u * PT_XBYTES);
+        tma_load_3d(xs(2 * q), &tmX, &bar_xfull[q], 0, m0, 2 * j);
+        issued = gj + 1;
+      }
+      for (int gj = issued - SP < 0 ? 0 : issued - SP; gj < issued; ++gj)
+        mbar_wait(&bar_xfull[gj % SP], (gj / SP) & 1, DEV_ERR_TIMEOUT_FULL, false);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_i8(128, 128);
+      bool ok = true;
+      for (int lt = 0; lt < ntl && ok; ++lt) {
+        const int b = lt & 1;
+        // the epilogue has read this accumulator's previous tile
+        if (lt >= 2 && !mbar_wait(&bar_acce[b], ((lt >> 1) - 1) & 1, DEV_ERR_TIMEOUT_ACC)) break;
+        tc_fence_after();
+        for (int i = 0; i < nk; ++i) {
+          const int gs = lt * nk + i, st = gs % S, gj = gs >> 1, a = gs % ST;
+          if (!mbar_wait(&bar_xfull[st >> 1], (gj / SP) & 1, DEV_ERR_TIMEOUT_FULL) ||
+              !mbar_wait(&bar_conv[a], (gs / ST) & 1, DEV_ERR_TIMEOUT_A)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t xaddr = smem_u32(xs(st));
+#pragma unroll
+          for (int kk = 0; kk < TC_BK / 32; ++kk)
+            mma_i8_ts(tmem + 128u * b, tmem + 256u + 32u * a + 8u * kk, smem_desc_k_sw128(xaddr + kk * 32), IDESC,
+                      (i > 0 || kk > 0) ? 1u : 0u);
+          // a pair stage is released after its second step's MMAs, if it is refilled
+          if ((st & 1) && gj + SP < npairs) mma_commit(&bar_empty[st >> 1]);
+        }
+        if (ok) mma_commit(&bar_accf[b]);
+      }
+      mma_commit(&bar_fin);
+      mbar_wait(&bar_fin, 0, DEV_ERR_TIMEOUT_ACC, false);   // no MMA in flight at teardown
+    }
+  } else if (warp < PT_EPI_WARP0) {
+    // ------------------------------------------------------------ converters
+    const int q4 = warp & 3;                      // tensor-memory lane quarter
+    const int h = (warp - 2) >> 2;                // which half of the K bytes of a step
+    const int row = 32 * q4 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16);
+    for (int gs = 0; gs < ntl * nk; ++gs) {
+      const int st = gs % S, gj = gs >> 1, a = gs % ST, c = st & 1;
+      if (!mbar_wait_warp(&bar_wfull[st >> 1], (gj / SP) & 1, DEV_ERR_TIMEOUT_FULL)) break;
+      tc_fence_after();
+      const uint4 w = *reinterpret_cast<const uint4*>(wsp(st >> 1) + c * PT_WBYTES + 32 * row +
+                                                      16 * (h ^ ((row >> 2) & 1)));
+      __syncwarp();
+      if (lane == 0 && c == 1) mbar_arrive(&bar_empty[st >> 1]);   // the pair's packed tiles consumed
+      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+      uint32_t av[16];
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) av[4 * g + jj] = unpack4(wv[g], jj);
+      tmem_st16(lane_base + (uint32_t)(256 + 32 * a + 16 * h), av);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_conv[a]);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q4 = warp & 3;
+    const int row = 32 * q4 + lane;               // output feature inside the tile
+    const int et = threadIdx.x - 32 * PT_EPI_WARP0;   // 0..127
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16);
+    const bool small_acc = (int64_t)127 * K < (int64_t)(1 << 22);
+    pdl_wait();                                   // s_x comes from the previous kernel
+    for (int lt = 0; lt < ntl; ++lt) {
+      int gi, n0, m0;
+      tile_of(lt, gi, n0, m0);
+      const int N = grp.N[gi];
+      TOut* __restrict__ Y = static_cast<TOut*>(grp.Y[gi]);
+      int32_t* __restrict__ acc_dbg = grp.acc_dbg[gi];
+      // the previous tile's staged outputs have been read by its store, and its scales are no longer used
+      asm volatile("bar.sync 3, 128;" ::: "memory");
+      {
+        const int m = m0 + et;
+        sdq[et] = m < M ? dequant_scale(ldg_f32(s_x + m), ldg_nc_f32(grp.s_w[gi])) : 0.f;
+      }
+      const int b = lt & 1;
+      const bool ok = mbar_wait_warp(&bar_accf[b], (lt >> 1) & 1, DEV_ERR_TIMEOUT_ACC);
+      tc_fence_after();
+      asm volatile("bar.sync 3, 128;" ::: "memory");     // the tile's scales are in place
+      const int n = n0 + row;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t v[2][16];
+        load_cols<16, 2>(lane_base + (uint32_t)(128 * b + c0), v);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const int cc = c0 + 16 * g;
+          float sq[16];
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const float4 f = *reinterpret_cast<const float4*>(sdq + cc + 4 * k4);
+            sq[4 * k4] = f.x; sq[4 * k4 + 1] = f.y; sq[4 * k4 + 2] = f.z; sq[4 * k4 + 3] = f.w;
+          }
+          if (use_tma_store) {
+            TOut* dst = ostage + (size_t)cc * 128 + row;
+            if (small_acc) {
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj)
+                stage_out(dst + jj * 128, __fmul_rn(small_int_to_float((int)v[g][jj] >> 6), sq[jj]));
+            } else {
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj) stage_out(dst + jj * 128, __fmul_rn((float)((int)v[g][jj] >> 6), sq[jj]));
+            }
+          } else if (ok && n < N) {
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int m = m0 + cc + jj;
+              if (m < M) {
+                const int acc = (int)v[g][jj] >> 6;
+                if (acc_dbg) acc_dbg[(size_t)m * N + n] = acc;
+                store_out(Y + (size_t)m * N + n, __fmul_rn((float)acc, sq[jj]));
+              }
+            }
+          }
+        }
+      }
+      // every read of this accumulator is done: the MMAs of tile lt + 2 may use it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_acce[b]);
+      if (use_tma_store) {
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 3, 128;" ::: "memory");
+        if (et == 0 && ok) {
+          tma_store_2d(&maps.y[gi], ostage, n0, m0);
+          bulk_wait_read();                        // the staging is reused by the next tile
+        }
+      }
+      // no early exit: the four warps take the same barriers whatever their waits returned
+      // (after a give-up every later wait returns at once)
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ===========================================================================
 // host side
 // ===========================================================================
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -693,11 +956,56 @@ static cudaError_t launch_tc(LinGroup grp, const void* Xq, const float* s_x, int
                     s_x, M, K, ksplit);
 }
 
+// The persistent int8 kernel (128 x 128 tiles, one CTA per SM over all tiles).
+template <typename TOut>
+static cudaError_t launch_tc_persistent(LinGroup grp, const void* Xq, const float* s_x, int M, int K,
+                                        cudaStream_t st) {
+  TcMaps maps;
+  CUtensorMap tmX;
+  if (!make_map_steps(&tmX, Xq, (uint64_t)K, (uint64_t)M, TC_BK, 128, 2, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  int use_tma_store = 1;
+  for (int g = 0; g < grp.count; ++g)
+    if (grp.acc_dbg[g] != nullptr || ((uint64_t)grp.N[g] * sizeof(TOut)) % 16 != 0) use_tma_store = 0;
+  grp.first[0] = 0;
+  for (int g = 0; g < grp.count; ++g) {
+    if (!make_map_steps(&maps.w[g], grp.pkW[g], (uint64_t)K / 4, (uint64_t)grp.N[g], TC_BK / 4, 128, 2,
+                        CU_TENSOR_MAP_SWIZZLE_32B))
+      return cudaErrorInvalidValue;
+    if (use_tma_store && !make_map_2d(&maps.y[g], grp.Y[g], MapType<TOut>::v, (uint64_t)grp.N[g], (uint64_t)M,
+                                      (uint64_t)grp.N[g] * sizeof(TOut), 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    if (!use_tma_store) maps.y[g] = tmX;           // unused
+    grp.first[g + 1] = grp.first[g] + (grp.N[g] + 127) / 128;
+  }
+  for (int g = grp.count; g < GROUP_MAX; ++g) {
+    maps.w[g] = maps.w[0];
+    maps.y[g] = maps.y[0];
+    grp.first[g + 1] = grp.first[grp.count];
+  }
+  int sms = 148, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int total = grp.first[grp.count] * ((M + 127) / 128);
+  const int grid = total < sms ? total : sms;
+  if (grid == 0) return cudaSuccess;
+  const size_t smem = pt_smem_bytes<TOut>();
+  auto kern = linear_tc_persistent_kernel<TOut>;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3((unsigned)grid), dim3(PT_THREADS), smem, st, 1u, maps, tmX, grp, use_tma_store, s_x,
+                    M, K);
+}
+
 // rows: 0 = choose the weight rows per CTA, 128 or 256 = that tile.
 template <int ACT_BITS, typename TOut>
 static cudaError_t dispatch_tc(const LinGroup& grp, const void* Xq, const float* s_x, int M, int K, int rows,
                                cudaStream_t st) {
   if (rows == 256) return launch_tc<128, ACT_BITS, TOut, 256>(grp, Xq, s_x, M, K, st);
+  if (rows == -1) {                   // the persistent kernel, asked for (int8, > 64 tokens, even K steps)
+    if constexpr (ACT_BITS == 8) return launch_tc_persistent<TOut>(grp, Xq, s_x, M, K, st);
+    return cudaErrorInvalidValue;
+  }
   if (M <= 16) return launch_tc<16, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
   if (M <= 32) return launch_tc<32, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
   if (M <= 64) return launch_tc<64, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
@@ -706,13 +1014,11 @@ static cudaError_t dispatch_tc(const LinGroup& grp, const void* Xq, const float*
   // than the 128-row tile at two CTAs per SM (about 1250 cycles per K step
   // against 512 of MMA work, with the activation tiles landing only every
   // ~1250 cycles), so it is used only when asked for (kernel 4).
-  int sms = 148, dev = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int tiles256 = 0;
-  for (int g = 0; g < grp.count; ++g) tiles256 += (grp.N[g] + 255) / 256;
-  tiles256 *= (M + 127) / 128;
-  (void)tiles256;                     // measured on B200: the 256-row tile is slower (see the tile's notes)
+  // The persistent kernel (kernel 5) hides each tile's start and epilogue
+  // behind the next tile's K loop, but at one CTA per SM its K steps come no
+  // faster than one CTA's of this kernel: measured on B200 it runs the batched
+  // prefill product in 242 us (6 or 8 stages) against 205 us here, so it is
+  // not chosen automatically.
   return launch_tc<128, ACT_BITS, TOut, 128>(grp, Xq, s_x, M, K, st);
 }
 
@@ -737,7 +1043,7 @@ cudaError_t run_linear_group(const LinGroup& grp, const void* Xq, int act_bits, 
                              int y_bf16, int path, cudaStream_t st);
 
 // path: 0 = automatic, 1 = SIMT, 2 = tcgen05, 3 = warp-MMA decode kernel, 4 = tcgen05 with
-// 256 weight rows per CTA
+// 256 weight rows per CTA, 5 = persistent tcgen05 (int8)
 cudaError_t run_linear(const void* Xq, int act_bits, const float* s_x, const uint8_t* pkW, const float* s_w,
                        int M, int N, int K, void* Y, int y_bf16, int32_t* acc_dbg, int path, cudaStream_t st) {
   // up to 32 tokens: one pass over the weights with warp-level MMA
@@ -771,7 +1077,7 @@ cudaError_t run_linear_group(const LinGroup& grp, const void* Xq, int act_bits, 
   if ((path == 0 || path == 3) && decode_path_applies(M, K))
     return run_linear_decode_group(grp, Xq, act_bits, s_x, M, K, y_bf16, st);
   if (path == 3) return cudaErrorInvalidValue;
-  const int rows = path == 2 ? 128 : path == 4 ? 256 : 0;
+  const int rows = path == 2 ? 128 : path == 4 ? 256 : path == 5 ? -1 : 0;
   if (act_bits == 8) {
     return y_bf16 ? dispatch_tc<8, __nv_bfloat16>(grp, Xq, s_x, M, K, rows, st)
                   : dispatch_tc<8, float>(grp, Xq, s_x, M, K, rows, st);

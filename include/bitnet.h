@@ -283,8 +283,10 @@ BITNET_API int bitnet_relu2_glu(const float* gate, const float* up, float* out, 
  *                            3 = warp-MMA decode kernel (BITNET_ERR_SHAPE for
  *                            shapes it does not cover: M > 32, K % 512 != 0 or
  *                            K > 16384), 4 = tcgen05 kernel with 256 weight
- *                            rows per CTA (the automatic choice for large
- *                            products, forced here at any shape).
+ *                            rows per CTA, 5 = persistent tcgen05 kernel (one
+ *                            CTA per SM over 128 x 128 tiles; int8 codes,
+ *                            M > 64 and an even K / 128, else
+ *                            BITNET_ERR_SHAPE).
  *   bitnet_bitlinear_kernel: 0-3 = the int8 quantiser, then that linear
  *                            kernel; 4 = the fused single kernel described at
  *                            bitnet_bitlinear (BITNET_ERR_SHAPE outside its range).

@@ -165,8 +165,9 @@ def test_kernel_choice_is_per_call(L):
     values outside the documented ones are refused before anything is enqueued."""
     lk = lambda kernel, **kw: L.bitnet_linear_kernel(ALIGNED, 8, ALIGNED, ALIGNED, ALIGNED, kw.get("M", 4), 256,
                                                      kw.get("K", 256), ALIGNED, 0, None, kernel, None)
-    assert lk(5) == 2 and lk(-1) == 2
+    assert lk(6) == 2 and lk(-1) == 2
     assert lk(3, M=33, K=512) == 2 and lk(3, K=384) == 2          # outside the decode kernel's range
+    assert lk(5) == 2 and lk(5, M=128, K=384) == 2                # persistent kernel: > 64 tokens, even K steps
     assert lk(1, M=0) == 0 and lk(2, M=0) == 0
     bk = lambda kernel, **kw: L.bitnet_bitlinear_kernel(ALIGNED, 1, kw.get("M", 4), kw.get("K", 512), None, 1e-6,
                                                         ALIGNED, ALIGNED, 256, ALIGNED, 0, ALIGNED, ALIGNED, kernel,

@@ -419,6 +419,45 @@ def test_linear_256_row_tile(M, N, K, act_bits, out):
     _check_linear(qx, qw, s_x, s_w, act_bits, out, path=4)
 
 
+@pytest.mark.parametrize("M,N,K,out", [(130, 520, 512, "f32"), (300, 1000, 1024, "bf16"), (65, 128, 256, "f32"),
+                                      (1000, 1200, 768, "bf16"), (4096, 640, 256, "f32")])
+def test_linear_persistent(M, N, K, out):
+    """The persistent tcgen05 kernel (one CTA per SM looping over 128 x 128
+    tiles, two accumulators, its own epilogue warps), forced at small and ragged
+    shapes: bit-exact accumulators (per-element epilogue) and outputs (staged,
+    one bulk store per tile)."""
+    qx, qw, s_x, s_w = _random_codes(M, N, K, 8, seed=M + 3 * N + K)
+    _check_linear(qx, qw, s_x, s_w, 8, out, path=5)
+    xq, pk = dev(qx), dev(O.pack_ternary(qw))
+    od = torch.float32 if out == "f32" else torch.bfloat16
+    Y5, _ = api.bitnet_linear(xq, 8, dev(s_x), pk, dev(np.array([s_w], np.float32)), out_dtype=od, kernel=5)
+    Y2, _ = api.bitnet_linear(xq, 8, dev(s_x), pk, dev(np.array([s_w], np.float32)), out_dtype=od, kernel=2)
+    torch.cuda.synchronize()
+    assert api.bitnet_device_error() == 0
+    assert torch.equal(Y5, Y2)
+
+
+def test_linear_group_many_tiles():
+    """A group whose tiles fill several waves: every output equals the
+    oracle's product."""
+    rng = np.random.default_rng(77)
+    M, K, Ns = 1024, 512, (4096, 5632)
+    qx = rng.integers(-128, 128, size=(M, K)).astype(np.int8)
+    s_x = rng.uniform(0.5, 200, size=M).astype(np.float32)
+    mats, ws = [], []
+    for N in Ns:
+        qw = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+        s_w = np.float32(rng.uniform(5, 60))
+        mats.append((qw, s_w))
+        ws.append((dev(O.pack_ternary(qw)), dev(np.array([s_w], np.float32))))
+    Ys = api.bitnet_linear_group(dev(qx), 8, dev(s_x), ws, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert api.bitnet_device_error() == 0
+    for (qw, s_w), Y in zip(mats, Ys):
+        _, y_o = O.linear(qx, s_x, qw, s_w)
+        assert np.array_equal(host(Y).view(np.uint32), y_o.view(np.uint32))
+
+
 # ------------------------------------------------------- fused BitLinear ----
 
 def _check_bitlinear(M, N, K, dtype, use_gamma, out, path=0, seed=0):
