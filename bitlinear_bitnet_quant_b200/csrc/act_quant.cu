@@ -966,11 +966,25 @@ static cudaError_t dispatch_q8(const void* X, const float* B, float* H, int M, i
   int C = K / E, PC = 1;
   while (PC < C) PC <<= 1;
 #define BN_Q8(NT, IT) launch_q8<TIn, NT, IT, PRE>(X, B, H, M, K, gamma, eps, Xq, s_x, st)
+  // 512 chunks a token (K = 2048 fp32, 4096 bf16) with few tokens (up to four
+  // per SM): more threads a token shorten its serial part.  Measured on B200,
+  // per launch: 512 x 2048 fp32 with the residual add 4.8 -> 4.1 us (512
+  // threads), without it 3.2 -> 3.1 us (256); 32 x 2048 with the add 2.4 ->
+  // 2.0 us (256).  Many tokens keep 128 threads (4096 x 4096 bf16: 9.7 us,
+  // against 13.4 with 256).  Every choice gives the same balanced tree over
+  // the chunk index, hence the same bits.
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const bool few = M <= 4 * sms;
   if (PC <= 1024) {
     switch (PC <= 128 ? 1 : PC / 128) {
       case 1: return BN_Q8(128, 1);
       case 2: return BN_Q8(128, 2);
-      case 4: return BN_Q8(128, 4);
+      case 4:
+        if (few && PRE == PRE_ADD && M > 64) return BN_Q8(512, 1);
+        if (few) return BN_Q8(256, 2);
+        return BN_Q8(128, 4);
       case 8: return BN_Q8(128, 8);
     }
   } else {

@@ -89,7 +89,8 @@ def test_quantize_weights_edge_cases():
 @pytest.mark.parametrize("M,K,dtype,use_gamma", [
     (1, 16, "f32", False), (3, 48, "bf16", True), (17, 256, "f32", False), (8, 256, "f32", True),
     (16, 2560, "bf16", False), (129, 4096, "bf16", False), (5, 2048, "bf16", True),
-    (7, 5632, "bf16", False), (2, 16384, "bf16", False), (3, 16384, "f32", True), (33, 1040, "f32", False)])
+    (7, 5632, "bf16", False), (2, 16384, "bf16", False), (3, 16384, "f32", True), (33, 1040, "f32", False),
+    (40, 2048, "f32", True), (600, 2048, "f32", False), (700, 4096, "bf16", True)])
 def test_quant_act(M, K, dtype, use_gamma):
     x = wl.add_entry_outliers(np.random.default_rng(M * K), wl.gaussian(np.random.default_rng(K), (M, K)),
                               0.005, 30.0)
@@ -642,7 +643,7 @@ def test_chain_24_layers():
 
 
 @pytest.mark.parametrize("M,K,use_gamma", [(3, 2048, False), (32, 2048, True), (5, 16, False), (17, 5632, False),
-                                             (2, 16384, True)])
+                                             (2, 16384, True), (300, 2048, True), (512, 2048, False)])
 def test_add_quant_act(M, K, use_gamma):
     """Residual add folded into the int8 quantiser: H, codes and scales equal
     bitnet_add followed by bitnet_quant_act, bit for bit."""
