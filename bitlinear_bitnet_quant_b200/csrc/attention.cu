@@ -182,31 +182,71 @@ BN_DEV void att_group_sync(int g) {
   else asm volatile("bar.sync 2, %0;" :: "n"(ATP_GT) : "memory");
 }
 
+// Running softmax state of RQ query rows of one thread: max, sum and the
+// unnormalised P V of its 16 dimensions.
+template <int RQ>
+struct AttState {
+  float m[RQ], sum[RQ];
+  float o[RQ][4][4];                                 // [query r][dimension group i][4]
+};
+
+template <int RQ>
+BN_DEV void att_state_init(AttState<RQ>& st) {
+#pragma unroll
+  for (int r = 0; r < RQ; ++r) {
+    st.m[r] = -INFINITY;
+    st.sum[r] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) st.o[r][i][c] = 0.f;
+  }
+}
+
+// st <- the merge of st and the state stored at x (field f at x[f * ATP_GT]):
+// both rescaled to the larger max (exact in real arithmetic), an empty state
+// (max -inf) weighing nothing.
+template <int RQ, typename Ld>
+BN_DEV void att_state_merge(AttState<RQ>& st, Ld ld) {
+#pragma unroll
+  for (int r = 0; r < RQ; ++r) {
+    const float m1 = ld(2 * r), s1 = ld(2 * r + 1);
+    const float mn = fmaxf(st.m[r], m1);
+    const float c0 = st.m[r] == -INFINITY ? 0.f : expf(st.m[r] - mn);
+    const float c1 = m1 == -INFINITY ? 0.f : expf(m1 - mn);
+    st.sum[r] = st.sum[r] * c0 + s1 * c1;
+    st.m[r] = mn;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) st.o[r][i][c] = st.o[r][i][c] * c0 + ld(2 * RQ + 16 * r + 4 * i + c) * c1;
+  }
+}
+
+// Key blocks [kb0, kb1) of query block qb for the whole CTA: the queries are
+// staged, group g takes the blocks kb0 + g, kb0 + g + 2, ..., and at the end
+// group 1's state is merged into group 0's (st is valid in group 0 only).
+// Every thread of the CTA calls it with the same arguments.
 template <int RQ, int KC>
-__global__ void __launch_bounds__(ATP_THREADS, RQ <= 2 ? 2 : 1)
-attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ Kc, const float* __restrict__ Vc,
-                         int L, int t0, int HD, int T_cap, float scale, float* __restrict__ A) {
+BN_DEV void att_task(const float* __restrict__ Q, const float* __restrict__ kbase, const float* __restrict__ vbase,
+                     int b, int h, int L, int t0, int HD, float scale, int qb, int kb0, int kb1, float* atp,
+                     AttState<RQ>& st) {
   using C = AtpCfg<RQ, KC>;
   constexpr int QB = C::QB, KB = C::KB, PPITCH = C::PPITCH, GFLOATS = C::GFLOATS;
-  extern __shared__ float atp[];
   const int tid = threadIdx.x;
   const int g = tid / ATP_GT, gt = tid - g * ATP_GT;
+  const int tq = gt >> 3, tk = gt & 7;
   float* qs = atp;                                  // [QB][PITCH]
   float* kbuf = qs + QB * ATP_PITCH + g * GFLOATS;  // [2][KB][PITCH] of this group
   float* vbuf = kbuf + 2 * KB * ATP_PITCH;          // [2][KB][PITCH]
   float* pt = vbuf + 2 * KB * ATP_PITCH;            // [KB][PPITCH] probabilities of the current block
-  pdl_launch_dependents();
-  pdl_wait();
-  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int l0 = qb * QB;
   const int nq = L - l0 < QB ? L - l0 : QB;
-  const int tq = gt >> 3, tk = gt & 7;
-  const float* kbase = Kc + (size_t)b * T_cap * HD + h * ATT_D;
-  const float* vbase = Vc + (size_t)b * T_cap * HD + h * ATT_D;
-  const int kend = t0 + l0 + nq;                     // keys 0 .. kend-1 are needed by the block
-  const int nblk = (kend + KB - 1) / KB;
-  if (g < nblk) {
-    const int j0 = g * KB;
+  const int kend = t0 + l0 + nq;                     // keys 0 .. kend-1 are visible to the block
+  __syncthreads();                                   // the previous task is done with every buffer
+  att_state_init(st);
+  if (kb0 + g < kb1) {
+    const int j0 = (kb0 + g) * KB;
     att_stage_kv<KB>(kbase, vbase, HD, j0, kend - j0 < KB ? kend - j0 : KB, kbuf, vbuf, gt);
   }
   for (int e = tid; e < QB * (ATT_D / 4); e += ATP_THREADS) {
@@ -216,21 +256,10 @@ attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ 
     *reinterpret_cast<float4*>(qs + rr * ATP_PITCH + 4 * cc) = v;
   }
   __syncthreads();                                   // the queries are in place for both groups
-  float m[RQ], sum[RQ];
-  float o[RQ][4][4];                                 // [query r][dimension group i][4]
-#pragma unroll
-  for (int r = 0; r < RQ; ++r) {
-    m[r] = -INFINITY;
-    sum[r] = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) o[r][i][c] = 0.f;
-  }
-  for (int blk = g, it = 0; blk < nblk; blk += ATP_G, ++it) {
+  for (int blk = kb0 + g, it = 0; blk < kb1; blk += ATP_G, ++it) {
     const int j0 = blk * KB;
     const int nk = kend - j0 < KB ? kend - j0 : KB;
-    if (blk + ATP_G < nblk) {
+    if (blk + ATP_G < kb1) {
       const int j1 = j0 + ATP_G * KB;
       att_stage_kv<KB>(kbase, vbase, HD, j1, kend - j1 < KB ? kend - j1 : KB,
                        kbuf + ((it + 1) & 1) * KB * ATP_PITCH, vbuf + ((it + 1) & 1) * KB * ATP_PITCH, gt);
@@ -242,11 +271,11 @@ attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ 
     const float* ks = kbuf + (it & 1) * KB * ATP_PITCH;
     const float* vs = vbuf + (it & 1) * KB * ATP_PITCH;
     // ---- scores of queries tq + 16 r and keys tk + 8 c ----
-    float s[RQ][KC];
+    float sc[RQ][KC];
 #pragma unroll
     for (int r = 0; r < RQ; ++r)
 #pragma unroll
-      for (int c = 0; c < KC; ++c) s[r][c] = 0.f;
+      for (int c = 0; c < KC; ++c) sc[r][c] = 0.f;
 #pragma unroll 4
     for (int dd = 0; dd < ATT_D; dd += 4) {
       float4 qv[RQ], kv[KC];
@@ -258,7 +287,7 @@ attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ 
       for (int r = 0; r < RQ; ++r)
 #pragma unroll
         for (int c = 0; c < KC; ++c)
-          s[r][c] += qv[r].x * kv[c].x + qv[r].y * kv[c].y + qv[r].z * kv[c].z + qv[r].w * kv[c].w;
+          sc[r][c] += qv[r].x * kv[c].x + qv[r].y * kv[c].y + qv[r].z * kv[c].z + qv[r].w * kv[c].w;
     }
     // ---- running softmax of the query rows (the row's 8 lanes: xor 1, 2, 4) ----
 #pragma unroll
@@ -268,84 +297,146 @@ attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ 
 #pragma unroll
       for (int c = 0; c < KC; ++c) {
         const int jj = tk + 8 * c;
-        s[r][c] = (jj < nk && j0 + jj <= qpos) ? s[r][c] * scale : -INFINITY;
-        bm = fmaxf(bm, s[r][c]);
+        sc[r][c] = (jj < nk && j0 + jj <= qpos) ? sc[r][c] * scale : -INFINITY;
+        bm = fmaxf(bm, sc[r][c]);
       }
 #pragma unroll
       for (int off = 4; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
-      const float mn = fmaxf(m[r], bm);
+      const float mn = fmaxf(st.m[r], bm);
       // a query row whose keys in this block are all masked keeps its state
-      const float corr = mn == -INFINITY ? 1.f : expf(m[r] - mn);
+      const float corr = mn == -INFINITY ? 1.f : expf(st.m[r] - mn);
       float psum = 0.f;
 #pragma unroll
       for (int c = 0; c < KC; ++c) {
-        const float p = s[r][c] == -INFINITY ? 0.f : expf(s[r][c] - mn);
-        pt[(tk + 8 * c) * PPITCH + tq + 16 * r] = p;
-        psum += p;
+        const float pp = sc[r][c] == -INFINITY ? 0.f : expf(sc[r][c] - mn);
+        pt[(tk + 8 * c) * PPITCH + tq + 16 * r] = pp;
+        psum += pp;
       }
 #pragma unroll
       for (int off = 4; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
-      sum[r] = sum[r] * corr + psum;
-      m[r] = mn;
+      st.sum[r] = st.sum[r] * corr + psum;
+      st.m[r] = mn;
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) o[r][i][c] *= corr;
+        for (int c = 0; c < 4; ++c) st.o[r][i][c] *= corr;
     }
     att_group_sync(g);                               // every row's probabilities are in place
     // ---- P V: queries tq + 16 r, dimensions 32 i + 4 tk .. + 3 ----
 #pragma unroll 2
     for (int j = 0; j < nk; ++j) {
-      float p[RQ];
+      float pr[RQ];
 #pragma unroll
-      for (int r = 0; r < RQ; ++r) p[r] = pt[j * PPITCH + tq + 16 * r];
+      for (int r = 0; r < RQ; ++r) pr[r] = pt[j * PPITCH + tq + 16 * r];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float4 v = *reinterpret_cast<const float4*>(vs + j * ATP_PITCH + 32 * i + 4 * tk);
 #pragma unroll
         for (int r = 0; r < RQ; ++r) {
-          o[r][i][0] += p[r] * v.x; o[r][i][1] += p[r] * v.y; o[r][i][2] += p[r] * v.z; o[r][i][3] += p[r] * v.w;
+          st.o[r][i][0] += pr[r] * v.x; st.o[r][i][1] += pr[r] * v.y;
+          st.o[r][i][2] += pr[r] * v.z; st.o[r][i][3] += pr[r] * v.w;
         }
       }
     }
     att_group_sync(g);                               // every thread of the group is done with this block's buffers
   }
-  // ---- merge: group 1 hands its running max, sum and output to the same thread of group 0 ----
+  // ---- group 1 hands its state to the same thread of group 0 ----
   float* xch = atp + QB * ATP_PITCH + GFLOATS;       // group 1's key/value buffers (no copy in flight)
   if (g == 1) {
 #pragma unroll
     for (int r = 0; r < RQ; ++r) {
-      xch[(2 * r) * ATP_GT + gt] = m[r];
-      xch[(2 * r + 1) * ATP_GT + gt] = sum[r];
-    }
-#pragma unroll
-    for (int r = 0; r < RQ; ++r)
+      xch[(2 * r) * ATP_GT + gt] = st.m[r];
+      xch[(2 * r + 1) * ATP_GT + gt] = st.sum[r];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) xch[(2 * RQ + 16 * r + 4 * i + c) * ATP_GT + gt] = o[r][i][c];
+        for (int c = 0; c < 4; ++c) xch[(2 * RQ + 16 * r + 4 * i + c) * ATP_GT + gt] = st.o[r][i][c];
+    }
   }
   __syncthreads();
-  if (g == 1) return;
+  if (g == 0) att_state_merge<RQ>(st, [&](int f) { return xch[f * ATP_GT + gt]; });
+}
+
+// Group 0 writes the normalised output rows of query block qb.
+template <int RQ, int KC>
+BN_DEV void att_write(const AttState<RQ>& st, float* __restrict__ A, int b, int h, int L, int HD, int qb) {
+  using C = AtpCfg<RQ, KC>;
+  const int gt = threadIdx.x, tq = gt >> 3, tk = gt & 7;
+  const int l0 = qb * C::QB;
+  const int nq = L - l0 < C::QB ? L - l0 : C::QB;
 #pragma unroll
   for (int r = 0; r < RQ; ++r) {
-    const float m1 = xch[(2 * r) * ATP_GT + gt], s1 = xch[(2 * r + 1) * ATP_GT + gt];
-    const float mn = fmaxf(m[r], m1);
-    const float c0 = m[r] == -INFINITY ? 0.f : expf(m[r] - mn);
-    const float c1 = m1 == -INFINITY ? 0.f : expf(m1 - mn);
-    const float tot = sum[r] * c0 + s1 * c1;
     const int row = tq + 16 * r;
-    const float inv = 1.0f / tot;
+    const float inv = 1.0f / st.sum[r];
+    if (row < nq) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float* x1 = xch + (2 * RQ + 16 * r + 4 * i) * ATP_GT + gt;
-      float4 res;
-      res.x = (o[r][i][0] * c0 + x1[0 * ATP_GT] * c1) * inv;
-      res.y = (o[r][i][1] * c0 + x1[1 * ATP_GT] * c1) * inv;
-      res.z = (o[r][i][2] * c0 + x1[2 * ATP_GT] * c1) * inv;
-      res.w = (o[r][i][3] * c0 + x1[3 * ATP_GT] * c1) * inv;
-      if (row < nq)
-        *reinterpret_cast<float4*>(A + ((size_t)b * L + l0 + row) * HD + h * ATT_D + 4 * tk + 32 * i) = res;
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<float4*>(A + ((size_t)b * L + l0 + row) * HD + h * ATT_D + 4 * tk + 32 * i) =
+            make_float4(st.o[r][i][0] * inv, st.o[r][i][1] * inv, st.o[r][i][2] * inv, st.o[r][i][3] * inv);
+    }
+  }
+}
+
+// Causal prefill over clusters of two CTAs per (pair of query blocks, head,
+// sequence): query block qa = p (light) and qz = nqb - 1 - p (heavy) have
+// nblk(qa) + nblk(qz) key blocks between them, split evenly: CTA 0 takes the
+// first s key blocks of qz and then all of qa, CTA 1 the rest of qz.  CTA 0
+// stores its partial state of qz into CTA 1's shared memory (distributed
+// shared memory), and CTA 1 merges it into its own before writing qz.  (When
+// qa == qz, the middle block of an odd count, its keys are split in half.)
+template <int RQ, int KC>
+__global__ void __launch_bounds__(ATP_THREADS, 1)
+attention_prefill_kernel(const float* __restrict__ Q, const float* __restrict__ Kc, const float* __restrict__ Vc,
+                         int L, int t0, int HD, int T_cap, float scale, float* __restrict__ A) {
+  using C = AtpCfg<RQ, KC>;
+  constexpr int QB = C::QB, KB = C::KB;
+  extern __shared__ float atp[];
+  float* pex = atp + (C::SMEM / 4);                  // [2 RQ + 16 RQ][ATP_GT]: the partner's partial state
+  pdl_launch_dependents();
+  cluster_arrive();                                  // both CTAs of the pair run before any remote store
+  cluster_wait();
+  pdl_wait();
+  const int rank = blockIdx.x & 1, p = blockIdx.x >> 1, h = blockIdx.y, b = blockIdx.z;
+  const int nqb = (L + QB - 1) / QB;
+  const int qa = p, qz = nqb - 1 - p;
+  auto nblk = [&](int q) {
+    const int l0 = q * QB;
+    return (t0 + l0 + (L - l0 < QB ? L - l0 : QB) + KB - 1) / KB;
+  };
+  const int wz = nblk(qz);
+  const int s = qa == qz ? wz / 2 : (wz - nblk(qa) > 0 ? (wz - nblk(qa)) / 2 : 0);
+  const float* kbase = Kc + (size_t)b * T_cap * HD + h * ATT_D;
+  const float* vbase = Vc + (size_t)b * T_cap * HD + h * ATT_D;
+  const int gt = threadIdx.x;
+  AttState<RQ> st;
+  if (rank == 0) {
+    att_task<RQ, KC>(Q, kbase, vbase, b, h, L, t0, HD, scale, qz, 0, s, atp, st);
+    if (gt < ATP_GT) {                               // group 0 stores its state into the partner's buffer
+      const uint32_t dst = cluster_map(smem_u32(pex), 1);
+#pragma unroll
+      for (int r = 0; r < RQ; ++r) {
+        st_cluster_u32(dst + 4u * ((2 * r) * ATP_GT + gt), __float_as_uint(st.m[r]));
+        st_cluster_u32(dst + 4u * ((2 * r + 1) * ATP_GT + gt), __float_as_uint(st.sum[r]));
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            st_cluster_u32(dst + 4u * ((2 * RQ + 16 * r + 4 * i + c) * ATP_GT + gt), __float_as_uint(st.o[r][i][c]));
+      }
+    }
+    cluster_arrive();                                // releases the stores to the partner
+    if (qa != qz) {
+      att_task<RQ, KC>(Q, kbase, vbase, b, h, L, t0, HD, scale, qa, 0, nblk(qa), atp, st);
+      if (gt < ATP_GT) att_write<RQ, KC>(st, A, b, h, L, HD, qa);
+    }
+    cluster_wait();
+  } else {
+    att_task<RQ, KC>(Q, kbase, vbase, b, h, L, t0, HD, scale, qz, s, wz, atp, st);
+    cluster_arrive();
+    cluster_wait();                                  // the partner's state is in place
+    if (gt < ATP_GT) {
+      att_state_merge<RQ>(st, [&](int f) { return pex[f * ATP_GT + gt]; });
+      att_write<RQ, KC>(st, A, b, h, L, HD, qz);
     }
   }
 }
@@ -376,10 +467,13 @@ cudaError_t run_attention(const float* Q, const float* Kc, const float* Vc, int 
   // the shared-memory reads per multiply-add, twice the blocks and barriers).
   using C = AtpCfg<4, 4>;
   auto kern = attention_prefill_kernel<4, 4>;
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), C::SMEM);
+  const size_t smem = C::SMEM + (size_t)ATP_GT * 18 * 4 * sizeof(float);   // + the partner's partial state
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3((unsigned)((L + C::QB - 1) / C::QB), (unsigned)heads, (unsigned)B),
-                    dim3(ATP_THREADS), C::SMEM, st, 1u, Q, Kc, Vc, L, t0, HD, T_cap, scale, A);
+  const int nqb = (L + C::QB - 1) / C::QB;
+  const int pairs = (nqb + 1) / 2;
+  return launch_pdl(kern, dim3((unsigned)(2 * pairs), (unsigned)heads, (unsigned)B), dim3(ATP_THREADS), smem, st,
+                    dim3(2, 1, 1), Q, Kc, Vc, L, t0, HD, T_cap, scale, A);
 }
 
 }  // namespace bitnet

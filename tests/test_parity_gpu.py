@@ -724,11 +724,13 @@ def _rand_rows(rng, n, HD, scale=0.6):
 
 
 @pytest.mark.parametrize("B,L,t0,heads", [(1, 64, 0, 16), (2, 40, 0, 16), (3, 20, 37, 2), (32, 1, 512, 16),
-                                          (4, 5, 100, 4), (2, 1, 0, 16)])
+                                          (4, 5, 100, 4), (2, 1, 0, 16), (1, 512, 0, 16), (1, 300, 0, 2),
+                                          (2, 130, 70, 4), (1, 200, 0, 4)])
 def test_rope_append_and_attention(B, L, t0, heads):
     """RoPE of Q and K, the cache append, and causal attention over the cache,
-    on the prefill kernel (16 or more queries per sequence) and the decode
-    kernel (fewer)."""
+    on the prefill kernel (16 or more queries per sequence: pairs of query
+    blocks sharing their keys over two CTAs, an odd middle block split in half)
+    and the decode kernel (fewer)."""
     rng = np.random.default_rng(B * 1000 + L * 10 + t0)
     HD = heads * 128
     T_cap = t0 + L + 3
