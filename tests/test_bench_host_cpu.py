@@ -65,9 +65,22 @@ def test_profiled_traffic_only_for_current_sources(tmp_path, monkeypatch):
         f"# header: with a colon\nkernel: k\nkernel_source_hash: {h}\ndram_bytes_per_launch: 4485632\n")
     assert bench.profiled_traffic("linear_x") == 4485632.0
     assert bench.profiled_traffic("linear_missing") is None
+    # the stacked-layer summaries give the bytes of every linear launch of a step
+    (tmp_path / "profiles" / "linear_y.txt").write_text(
+        f"kernel: all launches of a step\nkernel_source_hash: {h}\ndram_bytes_per_step: 412703232\n")
+    assert bench.profiled_traffic("linear_y") == 412703232.0
     (csrc / "a.cu").write_text("// kernel a, changed\n")
     assert bench.kernel_source_hash() != h
-    assert bench.profiled_traffic("linear_x") is None
+    assert bench.profiled_traffic("linear_x") is None and bench.profiled_traffic("linear_y") is None
+
+
+def test_targets_cover_the_decode_and_prefill_configs():
+    """The decode GEMV (>= 70 % of HBM) and the prefill GEMM (>= 50 % of int8)
+    targets are attached to exactly those bench lines."""
+    assert set(bench.TARGET_FRAC) == {"decode_m1", "decode_m4", "decode_m16", "prefill"}
+    assert all(bench.TARGET_FRAC[k] == 0.70 for k in ("decode_m1", "decode_m4", "decode_m16"))
+    assert bench.TARGET_FRAC["prefill"] == 0.50
+    assert set(bench.TARGET_FRAC) <= set(bench.WORKLOADS)
 
 
 def test_all_cores_cpu_baseline_line():
